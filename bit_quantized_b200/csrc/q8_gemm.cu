@@ -1,0 +1,716 @@
+// W8A8 GEMMs on the sm_100a tensor cores (tcgen05) with TMEM accumulators,
+// TMA-fed shared-memory pipelines and a fused dequant epilogue.
+//
+// What is computed ("大模型量化" (Xilyfe), INT32 accumulator section; the
+// quantized matmul of the "大模型量化技术" overview, section 2.1, read with
+// R = S (Q - Z); Transformers FP8 / FBGEMM page, section 5.3):
+//   INT8  acc[m,n] = sum_k xq[m,k] wq[n,k]              (int32 in TMEM)
+//         y = fl32(fl32(fl32(acc - Z[n] rowsum[m]) * Sx[m]) * Sw[n])
+//   FP8   acc = sum_k e4m3 x e4m3                        (fp32 in TMEM)
+//         y = fl32(fl32(acc * Sx[m]) * Sw[n])
+//   LLM.int8 (bitsandbytes LLM.int8 page, 核心思想): a second fp32 TMEM
+//         accumulator takes the fp16 outlier columns, y = fl32(y_int8 + y16)
+//   then y = fl32(y + bias[n]) and Y = bf16_rne(y).
+//
+// Two kernels share the same warp roles (192 threads):
+//   warp 0      TMA producer: one elected lane streams 128-byte-deep K slices
+//               of both operands into a ring of shared-memory stages;
+//   warp 1      allocates TMEM; one elected lane issues tcgen05.mma;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp reads its
+//               own 32-lane quarter of TMEM), dequant, bf16 stores.
+//
+// gemm_tile_kernel    persistent over 128 x BN output tiles, activations as
+//                     the MMA's M side; TMEM accumulators double-buffered so
+//                     the epilogue of one tile overlaps the next tile's MMAs.
+// gemm_decode_kernel  small token counts (decode): weights on the MMA's M side
+//                     (128 output channels per CTA) and the tokens as N, with
+//                     K split across the CTAs of a thread-block cluster whose
+//                     partial accumulators are summed through distributed
+//                     shared memory in a fixed rank order (exact for int32).
+//
+// No TMA multicast is used anywhere: each CTA loads its own tiles and the
+// 126 MB L2 provides the reuse across CTAs.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "q8_device.cuh"
+#include "q8_internal.h"
+
+namespace q8 {
+namespace {
+
+constexpr int kBM = 128;        // MMA M (TMEM lanes)
+constexpr int kBKB = 128;       // bytes of K per pipeline stage (one 128-byte swizzle row)
+constexpr int kThreads = 192;
+constexpr int kSmemBudget = 200 * 1024;
+
+enum GemmKind { kS8S8 = 0, kS8U8 = 1, kE4M3 = 2 };
+
+struct EpiParams {
+    int m, n;
+    const float* sx;
+    const int32_t* rowsum;
+    const float* sw;
+    const float* zw;
+    const float* bias;
+    __nv_bfloat16* y;
+    int64_t ldy;
+    void* acc_debug;
+    float* y16_debug;
+    const int32_t* outlier_count;
+    int* status;
+};
+
+template <int BN, bool MIXED>
+struct TileCfg {
+    static constexpr int A_BYTES = kBM * kBKB;
+    static constexpr int B_BYTES = BN * kBKB;
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int STAGES_RAW = kSmemBudget / STAGE;
+    static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+    static constexpr int BUF_COLS = MIXED ? 2 * BN : BN;     // int32 acc (+ fp32 outlier acc)
+    static constexpr int USED_COLS = 2 * BUF_COLS;
+    static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64
+                                   : USED_COLS <= 128 ? 128 : USED_COLS <= 256 ? 256 : 512;
+    static constexpr int SMEM = STAGES * STAGE + 1024;
+    static_assert(USED_COLS <= 512, "TMEM holds 512 columns");
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+};
+
+template <int KIND>
+constexpr uint32_t main_idesc(int n_mma) {
+    // kind::i8: A = activations (s8), B = weights (s8 or u8), int32 accumulate.
+    // kind::f8f6f4: both E4M3, fp32 accumulate.
+    return KIND == kE4M3 ? make_idesc(1, 0, 0, kBM, n_mma)
+                         : make_idesc(2, 1, KIND == kS8U8 ? 0 : 1, kBM, n_mma);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Dequant of one accumulator value (int32 path).
+__device__ __forceinline__ float dequant_int(int32_t acc, float zw, int32_t rs, float sx, float sw,
+                                             bool has_zp) {
+    int64_t c = static_cast<int64_t>(acc);
+    if (has_zp) c -= static_cast<int64_t>(zw) * static_cast<int64_t>(rs);
+    float v = __ll2float_rn(c);
+    v = __fmul_rn(v, sx);
+    return __fmul_rn(v, sw);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+    const __nv_bfloat16 lo = __float2bfloat16_rn(a), hi = __float2bfloat16_rn(b);
+    return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
+// ============================================================================
+// Persistent tile kernel
+// ============================================================================
+template <int BN, int KIND, bool MIXED>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmA16,
+                 const __grid_constant__ CUtensorMap tmB16, const EpiParams p, int num_kb,
+                 int tiles_m, int tiles_n) {
+    using C = TileCfg<BN, MIXED>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], 4);
+        }
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+
+    int n16_kb = 0;
+    if constexpr (MIXED) n16_kb = (*p.outlier_count + 63) / 64;
+    const int total_kb = num_kb + n16_kb;
+    const int num_tiles = tiles_m * tiles_n;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (elect_one()) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            if constexpr (MIXED) {
+                tma_prefetch_desc(&tmA16);
+                tma_prefetch_desc(&tmB16);
+            }
+            uint32_t issued = 0;             // stages that ever received a load
+            uint32_t last_par = 0;           // parity of each stage's last load
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int tm = tile % tiles_m, tn = tile / tiles_m;
+                for (int kb = 0; kb < total_kb; ++kb) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + stage * C::STAGE;
+                    uint8_t* sb = sa + C::A_BYTES;
+                    mbar_arrive_expect_tx(&full_bar[stage], C::STAGE);
+                    if (!MIXED || kb < num_kb) {
+                        tma_load_2d(sa, &tmA, &full_bar[stage], kb * kBKB, tm * kBM);
+                        tma_load_2d(sb, &tmB, &full_bar[stage], kb * kBKB, tn * BN);
+                    } else {
+                        const int k16 = (kb - num_kb) * 64;
+                        tma_load_2d(sa, &tmA16, &full_bar[stage], k16, tm * kBM);
+                        tma_load_2d(sb, &tmB16, &full_bar[stage], k16, tn * BN);
+                    }
+                    issued |= 1u << stage;
+                    last_par = (last_par & ~(1u << stage)) | (phase << stage);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+            if (!ok) {
+                // Abort: let every load already issued land before the CTA exits.
+                for (int s = 0; s < C::STAGES; ++s)
+                    if (issued & (1u << s)) mbar_wait(&full_bar[s], (last_par >> s) & 1, nullptr, nullptr);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (elect_one()) {
+            const uint32_t idesc = main_idesc<KIND>(BN);
+            const uint32_t idesc16 = make_idesc(1, 0, 0, kBM, BN);  // f16 x f16 -> f32
+            int stage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t bphase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!mbar_wait(&tempty_bar[buf], bphase ^ 1, &abort_sh, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_main = tmem_base + buf * C::BUF_COLS;
+                for (int kb = 0; kb < total_kb; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, &abort_sh, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_addr(smem + stage * C::STAGE);
+                    const uint64_t ad = sdesc_kmajor_sw128(sa);
+                    const uint64_t bd = sdesc_kmajor_sw128(sa + C::A_BYTES);
+                    if (!MIXED || kb < num_kb) {
+#pragma unroll
+                        for (int ks = 0; ks < kBKB / 32; ++ks) {
+                            if constexpr (KIND == kE4M3)
+                                mma_issue<kKindF8>(d_main, ad + 2 * ks, bd + 2 * ks, idesc, (kb | ks) != 0);
+                            else
+                                mma_issue<kKindI8>(d_main, ad + 2 * ks, bd + 2 * ks, idesc, (kb | ks) != 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < kBKB / 32; ++ks)
+                            mma_issue<kKindF16>(d_main + BN, ad + 2 * ks, bd + 2 * ks, idesc16,
+                                                ((kb - num_kb) | ks) != 0);
+                    }
+                    tc_commit(&empty_bar[stage]);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&tfull_bar[buf]);
+                buf ^= 1;
+                if (buf == 0) bphase ^= 1;
+            }
+            if (!ok) {
+                // Abort: wait for the MMAs already issued before TMEM is freed.
+                tc_commit(&drain_bar);
+                mbar_wait(&drain_bar, 0, nullptr, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue
+        const int q = warp & 3;  // this warp's TMEM lane quarter
+        const bool has_zp = p.zw != nullptr;
+        int buf = 0;
+        uint32_t bphase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            const int tm = tile % tiles_m, tn = tile / tiles_m;
+            if (!mbar_wait(&tfull_bar[buf], bphase, &abort_sh, p.status)) break;
+            tc_fence_after();
+            const int row = tm * kBM + q * 32 + lane;
+            const bool row_ok = row < p.m;
+            const float sx = row_ok ? p.sx[row] : 0.f;
+            const int32_t rs = (row_ok && has_zp) ? p.rowsum[row] : 0;
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::BUF_COLS;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                __syncwarp();
+                uint32_t r[32];
+                tmem_ld32(tb + c * 32, r);
+                uint32_t r16[32];
+                if constexpr (MIXED) {
+                    if (n16_kb > 0) tmem_ld32(tb + BN + c * 32, r16);
+                }
+                tmem_ld_wait();
+                const int n0 = tn * BN + c * 32;
+                if (row_ok && n0 < p.n) {
+                const int nv = (p.n - n0) >= 32 ? 32 : (p.n - n0);   // 16 or 32
+                float out[32];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (4 * j >= nv) break;
+                    const float4 sw4 = *reinterpret_cast<const float4*>(p.sw + n0 + 4 * j);
+                    float4 zw4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = zw4;
+                    if (has_zp) zw4 = *reinterpret_cast<const float4*>(p.zw + n0 + 4 * j);
+                    if (p.bias) b4 = *reinterpret_cast<const float4*>(p.bias + n0 + 4 * j);
+                    const float swv[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
+                    const float zwv[4] = {zw4.x, zw4.y, zw4.z, zw4.w};
+                    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 4 * j + e;
+                        float v;
+                        if constexpr (KIND == kE4M3) {
+                            v = __fmul_rn(__fmul_rn(__uint_as_float(r[i]), sx), swv[e]);
+                        } else {
+                            v = dequant_int(static_cast<int32_t>(r[i]), zwv[e], rs, sx, swv[e], has_zp);
+                        }
+                        if constexpr (MIXED) {
+                            const float y16 = n16_kb > 0 ? __uint_as_float(r16[i]) : 0.0f;
+                            v = __fadd_rn(v, y16);
+                        }
+                        if (p.bias) v = __fadd_rn(v, bv[e]);
+                        out[i] = v;
+                    }
+                }
+                uint4* yp = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(row) * p.ldy + n0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (8 * j >= nv) break;
+                    yp[j] = make_uint4(pack_bf16(out[8 * j], out[8 * j + 1]),
+                                       pack_bf16(out[8 * j + 2], out[8 * j + 3]),
+                                       pack_bf16(out[8 * j + 4], out[8 * j + 5]),
+                                       pack_bf16(out[8 * j + 6], out[8 * j + 7]));
+                }
+                if (p.acc_debug) {
+                    uint4* ap = reinterpret_cast<uint4*>(static_cast<uint32_t*>(p.acc_debug) +
+                                                         static_cast<int64_t>(row) * p.n + n0);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (4 * j >= nv) break;
+                        ap[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+                    }
+                }
+                if constexpr (MIXED) {
+                    if (p.y16_debug) {
+                        uint4* dp = reinterpret_cast<uint4*>(p.y16_debug + static_cast<int64_t>(row) * p.n + n0);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            if (4 * j >= nv) break;
+                            if (n16_kb > 0)
+                                dp[j] = make_uint4(r16[4 * j], r16[4 * j + 1], r16[4 * j + 2], r16[4 * j + 3]);
+                            else
+                                dp[j] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
+                }
+                }  // row_ok && n0 < p.n
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+            buf ^= 1;
+            if (buf == 0) bphase ^= 1;
+        }
+        __syncwarp();
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ============================================================================
+// Decode kernel: weights as the MMA's M side, tokens as N, split-K in a cluster
+// ============================================================================
+template <int NT, int KIND>
+struct DecodeCfg {
+    static constexpr int A_BYTES = kBM * kBKB;   // 128 weight rows
+    static constexpr int B_BYTES = NT * kBKB;    // NT token rows
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int RED_BYTES = NT * kBM * 4;
+    static constexpr int STAGES_RAW = (kSmemBudget - RED_BYTES) / STAGE;
+    static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+    static constexpr int TMEM_COLS = NT < 32 ? 32 : NT;
+    static constexpr int SMEM = STAGES * STAGE + RED_BYTES + 1024;
+};
+
+template <int NT, int KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                   const EpiParams p, int num_kb, int kb_per_split, int splits) {
+    using C = DecodeCfg<NT, KIND>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint32_t* red = reinterpret_cast<uint32_t*>(smem + C::STAGES * C::STAGE);  // [NT][128]
+    __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar;
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int tn = blockIdx.x;                       // 128 output channels
+    const uint32_t rank = cluster_ctarank();         // split index along K
+    const int kb0 = static_cast<int>(rank) * kb_per_split;
+    const int kb1 = min(num_kb, kb0 + kb_per_split);
+    const int my_kb = kb1 > kb0 ? kb1 - kb0 : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&tfull_bar, 1);
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+
+    if (warp == 0) {
+        if (elect_one()) {
+            tma_prefetch_desc(&tmW);
+            tma_prefetch_desc(&tmX);
+            uint32_t issued = 0, last_par = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sa = smem + stage * C::STAGE;
+                mbar_arrive_expect_tx(&full_bar[stage], C::STAGE);
+                tma_load_2d(sa, &tmW, &full_bar[stage], kb * kBKB, tn * kBM);
+                tma_load_2d(sa + C::A_BYTES, &tmX, &full_bar[stage], kb * kBKB, 0);
+                issued |= 1u << stage;
+                last_par = (last_par & ~(1u << stage)) | (phase << stage);
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            if (!ok)
+                for (int s = 0; s < C::STAGES; ++s)
+                    if (issued & (1u << s)) mbar_wait(&full_bar[s], (last_par >> s) & 1, nullptr, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (elect_one()) {
+            // A = weights (u8 or s8 for INT8, E4M3), B = tokens.
+            const uint32_t idesc = KIND == kE4M3 ? make_idesc(1, 0, 0, kBM, NT)
+                                                 : make_idesc(2, KIND == kS8U8 ? 0 : 1, 1, kBM, NT);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int i = 0; i < my_kb; ++i) {
+                if (!mbar_wait(&full_bar[stage], phase, &abort_sh, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = smem_addr(smem + stage * C::STAGE);
+                const uint64_t ad = sdesc_kmajor_sw128(sa);
+                const uint64_t bd = sdesc_kmajor_sw128(sa + C::A_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < kBKB / 32; ++ks) {
+                    if constexpr (KIND == kE4M3)
+                        mma_issue<kKindF8>(tmem_base, ad + 2 * ks, bd + 2 * ks, idesc, (i | ks) != 0);
+                    else
+                        mma_issue<kKindI8>(tmem_base, ad + 2 * ks, bd + 2 * ks, idesc, (i | ks) != 0);
+                }
+                tc_commit(&empty_bar[stage]);
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            tc_commit(ok ? &tfull_bar : &drain_bar);
+            if (!ok) mbar_wait(&drain_bar, 0, nullptr, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // Epilogue warps: TMEM partial -> own shared memory, laid out [token][channel].
+        const int q = warp & 3;
+        const int ch = q * 32 + lane;
+        bool have = my_kb > 0 && mbar_wait(&tfull_bar, 0, &abort_sh, p.status);
+        if (have) tc_fence_after();
+        __syncwarp();
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+        for (int c = 0; c < NT; c += 16) {
+            uint32_t r[16];
+            tmem_ld16(tb + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) red[(c + i) * kBM + ch] = have ? r[i] : 0u;
+        }
+        __syncwarp();
+    }
+
+    // Partials of the whole cluster are visible after this barrier.
+    __syncthreads();
+    cluster_sync();
+
+    if (warp >= 2) {
+        // Rank r finishes the tokens t with t % splits == r, summing the ranks'
+        // partials in rank order.
+        const int q = warp & 3;
+        const int ch = q * 32 + lane;
+        const int n = tn * kBM + ch;
+        const bool has_zp = p.zw != nullptr;
+        const bool col_ok = n < p.n;
+        const float sw = col_ok ? p.sw[n] : 0.f;
+        const float zw = (col_ok && has_zp) ? p.zw[n] : 0.f;
+        const float bias = (col_ok && p.bias) ? p.bias[n] : 0.f;
+        for (int t = static_cast<int>(rank); t < NT && t < p.m; t += splits) {
+            const uint32_t local = smem_addr(&red[t * kBM + ch]);
+            uint32_t acc_bits;
+            float v;
+            if constexpr (KIND == kE4M3) {
+                float s = 0.f;
+                for (int r = 0; r < splits; ++r)
+                    s = __fadd_rn(s, __uint_as_float(ld_shared_cluster_u32(map_shared_rank(local, r))));
+                acc_bits = __float_as_uint(s);
+                v = __fmul_rn(__fmul_rn(s, p.sx[t]), sw);
+            } else {
+                int32_t s = 0;
+                for (int r = 0; r < splits; ++r)
+                    s += static_cast<int32_t>(ld_shared_cluster_u32(map_shared_rank(local, r)));
+                acc_bits = static_cast<uint32_t>(s);
+                v = dequant_int(s, zw, has_zp ? p.rowsum[t] : 0, p.sx[t], sw, has_zp);
+            }
+            if (p.bias) v = __fadd_rn(v, bias);
+            if (col_ok) {
+                p.y[static_cast<int64_t>(t) * p.ldy + n] = __float2bfloat16_rn(v);
+                if (p.acc_debug)
+                    static_cast<uint32_t*>(p.acc_debug)[static_cast<int64_t>(t) * p.n + n] = acc_bits;
+            }
+        }
+    }
+
+    // Keep this CTA's shared memory alive until every rank has read it.
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ============================================================================
+// Host side
+// ============================================================================
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D K-major tile map with 128-byte swizzle: inner extent `inner` elements of
+// `esize` bytes, `outer` rows `ld_bytes` apart, box of (box_inner, box_outer).
+bool make_map(CUtensorMap* m, const void* base, bool fp16, uint64_t inner, uint64_t outer,
+              uint64_t ld_bytes, uint32_t box_inner, uint32_t box_outer) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {ld_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+template <int BN, int KIND, bool MIXED>
+q8_status run_tile(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
+    using C = TileCfg<BN, MIXED>;
+    CUtensorMap tA, tB, tA16, tB16;
+    if (!make_map(&tA, a.a_codes, false, a.k, a.m, a.lda, kBKB, kBM) ||
+        !make_map(&tB, a.b_codes, false, a.k, a.n, a.ldb, kBKB, BN))
+        return Q8_ERR_CUDA;
+    if constexpr (MIXED) {
+        if (!make_map(&tA16, a.xo, true, a.k16_cap, a.m, a.ldxo * 2, 64, kBM) ||
+            !make_map(&tB16, a.wo, true, a.k16_cap, a.n, a.ldwo * 2, 64, BN))
+            return Q8_ERR_CUDA;
+    } else {
+        tA16 = tA;
+        tB16 = tB;
+    }
+    auto kern = gemm_tile_kernel<BN, KIND, MIXED>;
+    if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
+    const int tiles_m = static_cast<int>((a.m + kBM - 1) / kBM);
+    const int tiles_n = static_cast<int>((a.n + BN - 1) / BN);
+    const int tiles = tiles_m * tiles_n;
+    const int num_kb = static_cast<int>((a.k + kBKB - 1) / kBKB);
+    const int grid = tiles < sm_count() ? tiles : sm_count();
+    kern<<<grid, kThreads, C::SMEM, s>>>(tA, tB, tA16, tB16, ep, num_kb, tiles_m, tiles_n);
+    return cudaGetLastError() == cudaSuccess ? Q8_OK : Q8_ERR_LAUNCH;
+}
+
+template <int NT, int KIND>
+q8_status run_decode(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
+    using C = DecodeCfg<NT, KIND>;
+    CUtensorMap tW, tX;
+    if (!make_map(&tW, a.b_codes, false, a.k, a.n, a.ldb, kBKB, kBM) ||
+        !make_map(&tX, a.a_codes, false, a.k, a.m, a.lda, kBKB, NT))
+        return Q8_ERR_CUDA;
+    auto kern = gemm_decode_kernel<NT, KIND>;
+    if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
+    const int tiles_n = static_cast<int>((a.n + kBM - 1) / kBM);
+    const int num_kb = static_cast<int>((a.k + kBKB - 1) / kBKB);
+    // Split K so that the grid covers the SMs once, at most 8 CTAs per cluster,
+    // with every split non-empty.
+    int want = sm_count() / tiles_n;
+    if (want < 1) want = 1;
+    if (want > 8) want = 8;
+    if (want > num_kb) want = num_kb;
+    const int per = (num_kb + want - 1) / want;
+    const int splits = (num_kb + per - 1) / per;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_n), static_cast<unsigned>(splits), 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = static_cast<unsigned>(splits);
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tW, tX, ep, num_kb, per, splits) != cudaSuccess)
+        return Q8_ERR_LAUNCH;
+    return Q8_OK;
+}
+
+template <int KIND>
+q8_status dispatch_kind(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
+    if (a.m <= 16) return run_decode<16, KIND>(a, ep, s);
+    if (a.m <= 32) return run_decode<32, KIND>(a, ep, s);
+    if (a.m <= 64) return run_decode<64, KIND>(a, ep, s);
+    // Output tiles of 128 x 256 unless that leaves most SMs idle.
+    const int64_t tiles256 = ((a.m + 127) / 128) * ((a.n + 255) / 256);
+    if (tiles256 >= sm_count()) return run_tile<256, KIND, false>(a, ep, s);
+    return run_tile<128, KIND, false>(a, ep, s);
+}
+
+}  // namespace
+
+q8_status launch_linear(const LinearArgs& a, cudaStream_t s) {
+    if (a.m == 0 || a.n == 0) return Q8_OK;
+    EpiParams ep;
+    ep.m = static_cast<int>(a.m);
+    ep.n = static_cast<int>(a.n);
+    ep.sx = a.sx;
+    ep.rowsum = a.rowsum;
+    ep.sw = a.sw;
+    ep.zw = a.zw;
+    ep.bias = a.bias;
+    ep.y = a.y;
+    ep.ldy = a.ldy;
+    ep.acc_debug = a.acc_debug;
+    ep.y16_debug = a.y16_debug;
+    ep.outlier_count = a.outlier_count;
+    ep.status = device_status_ptr();
+    if (a.outlier_count != nullptr) {
+        if (a.kind == kS8U8) return run_tile<128, kS8U8, true>(a, ep, s);
+        return run_tile<128, kS8S8, true>(a, ep, s);
+    }
+    switch (a.kind) {
+        case kS8S8: return dispatch_kind<kS8S8>(a, ep, s);
+        case kS8U8: return dispatch_kind<kS8U8>(a, ep, s);
+        case kE4M3: return dispatch_kind<kE4M3>(a, ep, s);
+    }
+    return Q8_ERR_DTYPE;
+}
+
+}  // namespace q8

@@ -1,0 +1,75 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/q8.h"
+
+namespace q8 {
+
+// Device address of the current device's status word (set up once per device).
+int* device_status_ptr();
+
+// ---- quantize kernels (q8_quant.cu)
+enum RowOp { kOpActInt8 = 0, kOpActFp8 = 1, kOpWeightAsym = 2, kOpWeightSym = 3, kOpWeightFp8 = 4 };
+
+struct RowQuantArgs {
+    const void* src;       // rows x k input (f16 / bf16 / f32)
+    q8_dtype src_dtype;
+    int64_t rows, k, ld;   // ld in elements
+    int op;                // RowOp
+    bool codes_u8;         // asymmetric weights stored as uint8 (q + 128)
+    float clip_ub;         // fp8 activations: > 0 clips the row absmax
+    const uint8_t* skip;   // [k] columns left out (LLM.int8 outliers); may be null
+    void* codes;           // rows x k, row stride k
+    float* scale;          // [rows]
+    float* zero_point;     // [rows] or null
+    int32_t* rowsum;       // [rows] or null
+    // LLM.int8 gather of the outlier columns (only with skip)
+    const int32_t* outlier_idx;
+    const int32_t* outlier_count;
+    __half* x_outlier;     // rows x ldo, or null
+    int64_t ldo;
+};
+
+cudaError_t launch_row_quant(const RowQuantArgs& a, cudaStream_t s);
+
+cudaError_t launch_outlier_columns(const void* X, q8_dtype dt, int64_t m, int64_t k, int64_t ldx,
+                                   float threshold, uint8_t* mask, int32_t* idx, int32_t* count,
+                                   cudaStream_t s);
+
+// W16o[n, j] for j < round_up(count, 64): the fp16 outlier columns of the weight
+// (from W16 when given, else dequantized from the codes); zeros past count.
+cudaError_t launch_gather_weight_outliers(const q8_weight& w, const __half* W16,
+                                          const int32_t* idx, const int32_t* count,
+                                          __half* W16o, int64_t ldo, cudaStream_t s);
+
+cudaError_t launch_dequant(const q8_weight& w, q8_dtype out_dtype, void* out, cudaStream_t s);
+
+// ---- GEMMs (q8_gemm.cu)
+struct LinearArgs {
+    int64_t m, n, k;
+    const void* a_codes;  int64_t lda;     // activations m x k
+    const void* b_codes;  int64_t ldb;     // weights n x k
+    int kind;                              // 0: int8 x int8, 1: int8 x uint8, 2: e4m3 x e4m3
+    const float* sx;
+    const int32_t* rowsum;                 // null when zw is null
+    const float* sw;
+    const float* zw;                       // null: no zero point
+    const float* bias;
+    __nv_bfloat16* y;  int64_t ldy;
+    void* acc_debug;                       // m x n (row stride n), or null
+    // LLM.int8 outlier stream (all null for plain W8A8)
+    const __half* xo; int64_t ldxo;        // m x ldxo fp16 gathered outlier columns
+    const __half* wo; int64_t ldwo;        // n x ldwo fp16 outlier weight columns
+    const int32_t* outlier_count;          // device
+    int64_t k16_cap;                       // columns the outlier buffers hold
+    float* y16_debug;                      // m x n, or null
+};
+
+q8_status launch_linear(const LinearArgs& a, cudaStream_t s);
+
+}  // namespace q8

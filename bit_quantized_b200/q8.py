@@ -1,0 +1,290 @@
+"""Thin Python binding of libq8.so (include/q8.h), same names as the C ABI.
+
+Argument marshalling only: each function checks that tensors are CUDA tensors
+of the expected dtype, allocates outputs with torch when the caller does not
+pass them, and calls the C entry point with raw device pointers and the
+current torch CUDA stream.  Every step of the computation runs in the
+library's kernels; there is no fallback.  If libq8.so is missing, importing
+this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libq8.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m bit_quantized_b200.build` "
+        "(the q8 CUDA library has no fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+# ---------------------------------------------------------------- C types
+
+Q8_OK, Q8_ERR_NULL, Q8_ERR_SHAPE, Q8_ERR_ALIGN, Q8_ERR_DTYPE, Q8_ERR_SCHEME = range(6)
+Q8_ERR_UNSUPPORTED_ARCH, Q8_ERR_LAUNCH, Q8_ERR_DEVICE_TIMEOUT, Q8_ERR_WORKSPACE, Q8_ERR_CUDA = range(6, 11)
+Q8_S8, Q8_U8, Q8_E4M3, Q8_F16, Q8_BF16, Q8_F32, Q8_S32 = range(7)
+Q8_ASYM_INT8, Q8_SYM_INT8, Q8_FP8_E4M3 = range(3)
+Q8_OP_LINEAR_W8A8, Q8_OP_LINEAR_INT8_MIXED = 0, 1
+
+EXPORTED = [
+    "q8_quantize_weight", "q8_dequantize_weight", "q8_quantize_act", "q8_outlier_quantize_act",
+    "q8_linear_w8a8", "q8_linear_int8_mixed", "q8_workspace_size", "q8_status_string",
+    "q8_get_device_status", "q8_clear_device_status", "q8_device_check", "q8_version",
+]
+
+
+class CWeight(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("code_dtype", ctypes.c_int),
+                ("scale", ctypes.c_void_p), ("zero_point", ctypes.c_void_p),
+                ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("ld", ctypes.c_int64)]
+
+
+class CAct(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("code_dtype", ctypes.c_int),
+                ("scale", ctypes.c_void_p), ("rowsum", ctypes.c_void_p),
+                ("m", ctypes.c_int64), ("k", ctypes.c_int64), ("ld", ctypes.c_int64)]
+
+
+_i64, _int, _f, _vp, _sz = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+_SIG = {
+    "q8_quantize_weight": ([_vp, _int, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp], _int),
+    "q8_dequantize_weight": ([ctypes.POINTER(CWeight), _int, _vp, _vp], _int),
+    "q8_quantize_act": ([_vp, _int, _i64, _i64, _i64, _int, _f, _vp, _vp, _vp, _vp], _int),
+    "q8_outlier_quantize_act": ([_vp, _int, _i64, _i64, _i64, _f, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _vp, _i64, _vp], _int),
+    "q8_linear_w8a8": ([ctypes.POINTER(CAct), ctypes.POINTER(CWeight), _vp, _vp, _i64, _vp, _vp,
+                        _sz, _vp], _int),
+    "q8_linear_int8_mixed": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeight), _vp, _f, _vp,
+                              _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
+    "q8_workspace_size": ([_int, _i64, _i64, _i64], _sz),
+    "q8_status_string": ([_int], ctypes.c_char_p),
+    "q8_get_device_status": ([_vp, _vp], _int),
+    "q8_clear_device_status": ([_vp], _int),
+    "q8_device_check": ([], _int),
+    "q8_version": ([], _int),
+}
+for _name, (_args, _res) in _SIG.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+
+def lib():
+    """The loaded ctypes library (raw C entry points)."""
+    return _lib
+
+
+class Q8Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {q8_status_string(status)} (status {status})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != Q8_OK:
+        raise Q8Error(status, where)
+
+
+def q8_status_string(status: int) -> str:
+    return _lib.q8_status_string(int(status)).decode()
+
+
+def q8_version() -> int:
+    return int(_lib.q8_version())
+
+
+def q8_device_check() -> int:
+    return int(_lib.q8_device_check())
+
+
+def q8_workspace_size(op: int, m: int, n: int, k: int) -> int:
+    return int(_lib.q8_workspace_size(op, m, n, k))
+
+
+# ---------------------------------------------------------------- helpers
+
+_FLOAT_DT = {torch.float16: Q8_F16, torch.bfloat16: Q8_BF16, torch.float32: Q8_F32}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be 2-D with unit column stride")
+    return t
+
+
+@dataclasses.dataclass
+class QWeight:
+    """A per-output-channel quantized weight (device tensors)."""
+    codes: torch.Tensor          # n x k int8 / uint8 / float8_e4m3fn
+    scale: torch.Tensor          # [n] fp32
+    zero_point: Optional[torch.Tensor]  # [n] fp32 (integer-valued) or None
+    code_dtype: int
+
+    def c(self) -> CWeight:
+        n, k = self.codes.shape
+        return CWeight(self.codes.data_ptr(), self.code_dtype, self.scale.data_ptr(),
+                       None if self.zero_point is None else self.zero_point.data_ptr(),
+                       n, k, self.codes.stride(0))
+
+
+@dataclasses.dataclass
+class QAct:
+    """A per-token quantized activation (device tensors)."""
+    codes: torch.Tensor          # m x k int8 / float8_e4m3fn
+    scale: torch.Tensor          # [m] fp32
+    rowsum: Optional[torch.Tensor]  # [m] int32 or None
+    code_dtype: int
+
+    def c(self) -> CAct:
+        m, k = self.codes.shape
+        return CAct(self.codes.data_ptr(), self.code_dtype, self.scale.data_ptr(),
+                    None if self.rowsum is None else self.rowsum.data_ptr(), m, k,
+                    self.codes.stride(0))
+
+
+# ---------------------------------------------------------------- entry points
+
+_SCHEME = {"asym": Q8_ASYM_INT8, "sym": Q8_SYM_INT8, "fp8": Q8_FP8_E4M3}
+_CODES = {"s8": (Q8_S8, torch.int8), "u8": (Q8_U8, torch.uint8),
+          "e4m3": (Q8_E4M3, torch.float8_e4m3fn)}
+
+
+def q8_quantize_weight(W: torch.Tensor, scheme: str = "asym", codes: str = "s8",
+                       stream=None) -> QWeight:
+    """Per-output-channel weight quantization (see q8_quantize_weight in q8.h)."""
+    _cuda(W, "W")
+    n, k = W.shape
+    cdt, tdt = _CODES[codes]
+    q = torch.empty((n, k), dtype=tdt, device=W.device)
+    S = torch.empty(n, dtype=torch.float32, device=W.device)
+    Z = torch.empty(n, dtype=torch.float32, device=W.device) if scheme == "asym" else None
+    _check(_lib.q8_quantize_weight(_ptr(W), _FLOAT_DT[W.dtype], n, k, W.stride(0),
+                                   _SCHEME[scheme], cdt, _ptr(q), _ptr(S), _ptr(Z),
+                                   _stream(stream)), "q8_quantize_weight")
+    return QWeight(q, S, Z, cdt)
+
+
+def q8_dequantize_weight(w: QWeight, out_dtype=torch.float32, stream=None) -> torch.Tensor:
+    out = torch.empty(w.codes.shape, dtype=out_dtype, device=w.codes.device)
+    cw = w.c()
+    _check(_lib.q8_dequantize_weight(ctypes.byref(cw), _FLOAT_DT[out_dtype], _ptr(out),
+                                     _stream(stream)), "q8_dequantize_weight")
+    return out
+
+
+def q8_quantize_act(X: torch.Tensor, scheme: str = "int8", clip_ub: float = 0.0,
+                    out: Optional[QAct] = None, stream=None) -> QAct:
+    """Dynamic per-token quantization: scheme "int8" (symmetric, row sums) or "fp8"."""
+    _cuda(X, "X")
+    m, k = X.shape
+    if out is None:
+        if scheme == "int8":
+            out = QAct(torch.empty((m, k), dtype=torch.int8, device=X.device),
+                       torch.empty(m, dtype=torch.float32, device=X.device),
+                       torch.empty(m, dtype=torch.int32, device=X.device), Q8_S8)
+        else:
+            out = QAct(torch.empty((m, k), dtype=torch.float8_e4m3fn, device=X.device),
+                       torch.empty(m, dtype=torch.float32, device=X.device), None, Q8_E4M3)
+    _check(_lib.q8_quantize_act(_ptr(X), _FLOAT_DT[X.dtype], m, k, X.stride(0),
+                                Q8_SYM_INT8 if scheme == "int8" else Q8_FP8_E4M3, float(clip_ub),
+                                _ptr(out.codes), _ptr(out.scale), _ptr(out.rowsum),
+                                _stream(stream)), "q8_quantize_act")
+    return out
+
+
+def q8_outlier_quantize_act(X: torch.Tensor, threshold: float = 6.0, gather: bool = True,
+                            stream=None) -> dict:
+    """LLM.int8 outlier columns + regular-stream INT8 quantization."""
+    _cuda(X, "X")
+    m, k = X.shape
+    dev = X.device
+    kp = (k + 63) // 64 * 64
+    r = {
+        "codes": torch.empty((m, k), dtype=torch.int8, device=dev),
+        "scale": torch.empty(m, dtype=torch.float32, device=dev),
+        "rowsum": torch.empty(m, dtype=torch.int32, device=dev),
+        "mask": torch.empty(k, dtype=torch.uint8, device=dev),
+        "idx": torch.empty(k, dtype=torch.int32, device=dev),
+        "count": torch.empty(1, dtype=torch.int32, device=dev),
+        "x_outlier": torch.empty((m, kp), dtype=torch.float16, device=dev) if gather else None,
+    }
+    _check(_lib.q8_outlier_quantize_act(
+        _ptr(X), _FLOAT_DT[X.dtype], m, k, X.stride(0), float(threshold), _ptr(r["codes"]),
+        _ptr(r["scale"]), _ptr(r["rowsum"]), _ptr(r["mask"]), _ptr(r["idx"]), _ptr(r["count"]),
+        _ptr(r["x_outlier"]), kp, _stream(stream)), "q8_outlier_quantize_act")
+    return r
+
+
+def q8_linear_w8a8(x: QAct, w: QWeight, bias: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None, acc_debug: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """W8A8 linear with the dequant epilogue; returns the bf16 M x N output."""
+    m, n = x.codes.shape[0], w.codes.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=x.codes.device)
+    cx, cw = x.c(), w.c()
+    _check(_lib.q8_linear_w8a8(ctypes.byref(cx), ctypes.byref(cw), _ptr(bias), _ptr(out),
+                               out.stride(0), _ptr(acc_debug), None, 0, _stream(stream)),
+           "q8_linear_w8a8")
+    return out
+
+
+def q8_linear_int8_mixed(X: torch.Tensor, w: QWeight, threshold: float = 6.0,
+                         W16: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
+                         out: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None, debug: bool = False,
+                         stream=None):
+    """LLM.int8 mixed-decomposition linear.  Returns Y, or (Y, debug dict) with debug=True."""
+    _cuda(X, "X")
+    m, k = X.shape
+    n = w.codes.shape[0]
+    dev = X.device
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    need = q8_workspace_size(Q8_OP_LINEAR_INT8_MIXED, m, n, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    dbg = None
+    if debug:
+        dbg = {"mask": torch.empty(k, dtype=torch.uint8, device=dev),
+               "count": torch.empty(1, dtype=torch.int32, device=dev),
+               "acc": torch.empty((m, n), dtype=torch.int32, device=dev),
+               "y16": torch.empty((m, n), dtype=torch.float32, device=dev)}
+    cw = w.c()
+    _check(_lib.q8_linear_int8_mixed(
+        _ptr(X), _FLOAT_DT[X.dtype], m, k, X.stride(0), ctypes.byref(cw), _ptr(W16),
+        float(threshold), _ptr(bias), _ptr(out), out.stride(0),
+        _ptr(dbg["mask"]) if dbg else None, _ptr(dbg["count"]) if dbg else None,
+        _ptr(dbg["acc"]) if dbg else None, _ptr(dbg["y16"]) if dbg else None,
+        _ptr(workspace), workspace.numel(), _stream(stream)), "q8_linear_int8_mixed")
+    return (out, dbg) if debug else out
+
+
+def q8_get_device_status(stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check(_lib.q8_get_device_status(ctypes.cast(ctypes.pointer(v), ctypes.c_void_p),
+                                     _stream(stream)), "q8_get_device_status")
+    return int(v.value)
+
+
+def q8_clear_device_status(stream=None) -> None:
+    _check(_lib.q8_clear_device_status(_stream(stream)), "q8_clear_device_status")

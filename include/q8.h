@@ -1,0 +1,282 @@
+/*
+ * q8.h -- C ABI of the B200 (sm_100a) 8-bit quantized linear layer.
+ *
+ * The library computes the hot path of an 8-bit quantized nn.Linear:
+ *   - per-output-channel weight quantization (asymmetric or symmetric INT8, FP8 E4M3);
+ *   - dynamic per-token activation quantization (symmetric INT8 with row sums,
+ *     or FP8 E4M3 with an upper-bound clip);
+ *   - the W8A8 GEMM with INT32 / FP32 accumulation and a dequant epilogue;
+ *   - the LLM.int8 mixed decomposition (outlier feature columns in fp16).
+ *
+ * Notation follows the pages' linear map Q = round(R / S) + Z, R = S (Q - Z):
+ * `scale` is S, the dequant multiplier, and `zero_point` is Z, an integer held
+ * in fp32.  Page short names used in the citations:
+ *   [Fabric]   "8-Bit LLM Quantization with Lightning Fabric" (mlqm.cn)
+ *   [CSDN]     "大模型量化技术" overview (devpress.csdn.net), sections 2.1-2.3
+ *   [FBGEMM]   "Transformers FP8 (W8A8) 量化实战：基于 FBGEMM", sections 5.1-5.3, 6
+ *   [LLM.int8] "Transformers 单 GPU 高效推理：bitsandbytes LLM.int8 8-bit 混合精度量化"
+ *   [Xilyfe]   "大模型量化" (xilyfe.github.io): symmetric, asymmetric, INT32 accumulator
+ *
+ * Conventions shared by every entry point
+ *   Layout      all matrices are row-major 2-D: X is M x K (tokens x features),
+ *               W is N x K (out x in, the nn.Linear layout of [FBGEMM] 5.1),
+ *               Y is M x N.  Leading dimensions are in elements.  Callers flatten
+ *               leading batch dims first ([FBGEMM] 5.2-5.3: x.view(-1, K), then
+ *               the result is viewed back to (*x.shape[:-1], -1)).
+ *   Memory      every pointer is DEVICE memory owned by the caller, unless a
+ *               parameter says "host".  The library allocates nothing: scratch
+ *               comes from the caller's `workspace` (see q8_workspace_size).
+ *   Streams     every call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *               the legacy default stream) and never synchronizes the host,
+ *               except q8_get_device_status.
+ *   Sizes       K % 32 == 0, N % 16 == 0, M >= 0; M, N, K <= 2^31 - 1;
+ *               INT8 GEMMs need K <= 32768 (INT32 accumulator bound).
+ *               M == 0 is a valid empty call that launches nothing.
+ *   Alignment   every pointer 16-byte aligned; every leading dimension a
+ *               multiple of 16 bytes.
+ *   Values      inputs must be finite; NaN and Inf inputs give unspecified codes.
+ *   Rounding    round-half-to-even everywhere; q = rne(fl32(x / S)) with an
+ *               IEEE fp32 division, so codes are bit-exact with a scalar
+ *               reference; S is floored at 1e-8 ([Xilyfe] QuantConfig eps).
+ *   Errors      every call returns a q8_status and never prints, throws or
+ *               aborts.  Arguments are validated on the host before anything is
+ *               launched, so an error return means nothing was enqueued.
+ *               Device-side waits are bounded (about one second); a wait that
+ *               runs out records Q8_ERR_DEVICE_TIMEOUT in a per-device status
+ *               word read by q8_get_device_status.
+ *   Hardware    compute capability 10.0 (B200, sm_100a) only; anything else
+ *               returns Q8_ERR_UNSUPPORTED_ARCH after argument validation.
+ */
+#ifndef Q8_H_
+#define Q8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define Q8_VERSION 1
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st *q8_stream_t;
+
+typedef enum {
+    Q8_OK = 0,
+    Q8_ERR_NULL = 1,             /* a required pointer is NULL */
+    Q8_ERR_SHAPE = 2,            /* a size or leading dimension is out of range */
+    Q8_ERR_ALIGN = 3,            /* a pointer or leading dimension is not 16-byte aligned */
+    Q8_ERR_DTYPE = 4,            /* unsupported dtype, or dtypes that do not fit together */
+    Q8_ERR_SCHEME = 5,           /* unsupported scheme, or scheme / code dtype mismatch */
+    Q8_ERR_UNSUPPORTED_ARCH = 6, /* the current device is not compute capability 10.0 */
+    Q8_ERR_LAUNCH = 7,           /* a kernel launch failed */
+    Q8_ERR_DEVICE_TIMEOUT = 8,   /* a bounded device wait ran out (q8_get_device_status) */
+    Q8_ERR_WORKSPACE = 9,        /* workspace NULL or smaller than q8_workspace_size */
+    Q8_ERR_CUDA = 10             /* another CUDA runtime error (no device, bad stream, ...) */
+} q8_status;
+
+typedef enum {
+    Q8_S8 = 0,    /* int8 codes */
+    Q8_U8 = 1,    /* uint8 codes (asymmetric weights stored as q + 128) */
+    Q8_E4M3 = 2,  /* OCP FP8 E4M3FN codes (max 448, no infinities) */
+    Q8_F16 = 3,   /* IEEE binary16 */
+    Q8_BF16 = 4,  /* bfloat16 */
+    Q8_F32 = 5,
+    Q8_S32 = 6
+} q8_dtype;
+
+typedef enum {
+    Q8_ASYM_INT8 = 0, /* per-row min-max, S = (max - min)/255, Z = rne(-min/S) - 128 */
+    Q8_SYM_INT8 = 1,  /* per-row absmax, S = absmax/127, Z = 0, codes in [-127, 127] */
+    Q8_FP8_E4M3 = 2   /* per-row absmax, S = absmax/448, codes E4M3 saturating */
+} q8_scheme;
+
+/* A quantized weight: N x K codes (row stride `ld` elements) with one scale per
+ * row and, for asymmetric codes, one zero point per row.  For Q8_U8 codes the
+ * zero point is in the uint8 convention (Z + 128), so S (q - zero_point) is
+ * the dequantized value in both conventions. */
+typedef struct {
+    const void *codes;
+    q8_dtype code_dtype;          /* Q8_S8, Q8_U8 or Q8_E4M3 */
+    const float *scale;           /* [n] */
+    const float *zero_point;      /* [n] integer-valued; NULL for symmetric / FP8 */
+    int64_t n, k, ld;
+} q8_weight;
+
+/* A quantized activation: M x K codes with one scale per row and, for INT8,
+ * the int32 row sums of the codes (needed when the weight has a zero point). */
+typedef struct {
+    const void *codes;
+    q8_dtype code_dtype;          /* Q8_S8 or Q8_E4M3 */
+    const float *scale;           /* [m] */
+    const int32_t *rowsum;        /* [m]; may be NULL when the weight has no zero point */
+    int64_t m, k, ld;
+} q8_act;
+
+/*
+ * Per-output-channel weight quantization, one row of W at a time.
+ * [Fabric] 2.1, 2.3 and 3.3 (one scale and zero point per output row);
+ * [Xilyfe] asymmetric section (s = 255/(alpha-beta), z = round(-s beta) - 128)
+ * and symmetric section (s = 127/alpha); [CSDN] 2.3 min-max calibration;
+ * [FBGEMM] 5.1 (e4m3 weight, fp32 weight_scale per output channel).
+ *
+ *   W           device, n x k, w_dtype Q8_F16, Q8_BF16 or Q8_F32, row stride ldw.
+ *   scheme      Q8_ASYM_INT8 (code_dtype Q8_S8 or Q8_U8), Q8_SYM_INT8 (Q8_S8),
+ *               Q8_FP8_E4M3 (Q8_E4M3).
+ *   codes       device, n x k output, row stride k.
+ *   scale       device [n] output.
+ *   zero_point  device [n] output for Q8_ASYM_INT8 (required); ignored (may be
+ *               NULL) for the other schemes.
+ * Asymmetric, per row with beta = min, alpha = max:
+ *   S = max(fl32(fl32(alpha - beta) / 255), 1e-8);
+ *   Z = clamp(rne(fl32(-beta / S)) - 128, -128, 127);
+ *   q = clamp(rne(fl32(w / S)) + Z, -128, 127)   (stored + 128 for Q8_U8, Z too).
+ * Symmetric: S = max(fl32(absmax / 127), 1e-8); q = clamp(rne(fl32(w / S)), -127, 127).
+ * FP8: S = max(fl32(absmax / 448), 1e-8); q = e4m3_rne_satfinite(fl32(w / S)).
+ */
+q8_status q8_quantize_weight(const void *W, q8_dtype w_dtype, int64_t n, int64_t k,
+                             int64_t ldw, q8_scheme scheme, q8_dtype code_dtype,
+                             void *codes, float *scale, float *zero_point,
+                             q8_stream_t stream);
+
+/*
+ * Dequantize a weight back to floating point for debugging, out = S (q - Z)
+ * ([Fabric] 3.3 dequantize_weight; [Xilyfe] "量化是什么": r = S (q - Z)).
+ * fp32 order: d = fl32(q - Z), v = fl32(S * d), then RNE to out_dtype.
+ *   out   device, w->n x w->k, out_dtype Q8_F32, Q8_F16 or Q8_BF16, row stride w->k.
+ */
+q8_status q8_dequantize_weight(const q8_weight *w, q8_dtype out_dtype, void *out,
+                               q8_stream_t stream);
+
+/*
+ * Dynamic per-token activation quantization, every call.
+ * [Xilyfe] symmetric section and dynamic-quantization paragraph; [FBGEMM] 5.2
+ * (quantize_fp8_per_row with the activation_scale_ub clip) and 6 (ub 1200.0).
+ *
+ *   X        device, m x k, x_dtype Q8_F16, Q8_BF16 or Q8_F32, row stride ldx.
+ *   scheme   Q8_SYM_INT8: S = max(fl32(absmax/127), 1e-8),
+ *              q = clamp(rne(fl32(x/S)), -127, 127), codes int8;
+ *            Q8_FP8_E4M3: alpha = min(absmax, clip_ub) when clip_ub > 0,
+ *              S = max(fl32(alpha/448), 1e-8), q = e4m3_rne_satfinite(fl32(x/S)).
+ *   clip_ub  FP8 only; <= 0 means no clip.
+ *   codes    device, m x k output (int8 or e4m3), row stride k.
+ *   scale    device [m] output.
+ *   rowsum   device [m] int32 output, sum_k q (INT8 only; may be NULL).
+ */
+q8_status q8_quantize_act(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
+                          int64_t ldx, q8_scheme scheme, float clip_ub, void *codes,
+                          float *scale, int32_t *rowsum, q8_stream_t stream);
+
+/*
+ * LLM.int8 outlier detection fused with the regular stream's quantization
+ * ([LLM.int8] 核心思想 and BitsAndBytesConfig: llm_int8_threshold = 6.0).
+ * A feature column k is an outlier when some token has |X[m, k]| > threshold
+ * (strictly); threshold <= 0 turns the decomposition off.  Then, per token,
+ * alpha is the absmax over the non-outlier columns and the INT8 codes of
+ * outlier columns are 0 (the regular stream is "the rest").
+ *
+ *   X             device, m x k fp16 (Q8_F16), row stride ldx.
+ *   codes         device, m x k int8 output, row stride k.
+ *   scale         device [m] output;  rowsum device [m] int32 output.
+ *   mask          device [k] uint8 output: 1 for outlier columns.
+ *   idx           device [k] int32 output: outlier columns ascending in
+ *                 idx[0 .. *count); entries past *count are unspecified.
+ *   count         device int32 output (stays on the device).
+ *   x_outlier     device, m x ldo fp16 output: x_outlier[m, j] = X[m, idx[j]]
+ *                 for j < *count and 0 for count <= j < round_up(count, 64);
+ *                 may be NULL.  ldo >= round_up(k, 64) and a multiple of 8.
+ * The column pass reads all m rows, so the outlier set depends on the batch.
+ */
+q8_status q8_outlier_quantize_act(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
+                                  int64_t ldx, float threshold, void *codes, float *scale,
+                                  int32_t *rowsum, uint8_t *mask, int32_t *idx,
+                                  int32_t *count, void *x_outlier, int64_t ldo,
+                                  q8_stream_t stream);
+
+/*
+ * W8A8 linear: Y = dequant(x) dequant(w)^T (+ bias), bf16 out.
+ * INT8 ([Xilyfe] INT32 accumulator section; [CSDN] 2.1 quantized matmul read
+ * with R = S (Q - Z)):
+ *   acc[m, n] = sum_k xq[m, k] wq[n, k]                  (tensor cores, int32)
+ *   y = fl32(fl32(fl32(acc - Z[n] rowsum[m]) * Sx[m]) * Sw[n]);  y = fl32(y + bias[n])
+ * FP8 ([FBGEMM] 5.3 f8f8bf16_rowwise, then + bias):
+ *   acc = sum_k e4m3(xq) e4m3(wq) (tensor cores, fp32);  y = fl32(fl32(acc*Sx)*Sw) (+bias)
+ * Y[m, n] = bf16_rne(y).
+ *
+ *   x          INT8 (Q8_S8) with x->rowsum required when w->zero_point is set,
+ *              or FP8 (Q8_E4M3); x->k == w->k.
+ *   w          Q8_S8 / Q8_U8 (with or without zero point) for INT8 x;
+ *              Q8_E4M3 for FP8 x.
+ *   bias       device [n] fp32, or NULL.
+ *   Y          device, m x n bf16 output, row stride ldy >= n.
+ *   acc_debug  device, m x n int32 (INT8) or fp32 (FP8) raw accumulator
+ *              output (row stride n), or NULL.
+ *   workspace  unused by this call today; pass q8_workspace_size(Q8_OP_LINEAR_W8A8, ...)
+ *              bytes (currently 0; NULL accepted).
+ */
+q8_status q8_linear_w8a8(const q8_act *x, const q8_weight *w, const float *bias, void *Y,
+                         int64_t ldy, void *acc_debug, void *workspace, size_t ws_bytes,
+                         q8_stream_t stream);
+
+/*
+ * LLM.int8 mixed-decomposition linear ([LLM.int8] 核心思想; BitsAndBytesConfig
+ * llm_int8_threshold, llm_int8_has_fp16_weight).  One call runs
+ * q8_outlier_quantize_act on X, the INT8 GEMM of the regular stream, and the
+ * fp16 GEMM of the outlier columns, merged before rounding:
+ *   y16[m, n] = sum_{j < count} X[m, idx[j]] W16[n, idx[j]]   (fp16 in, fp32 acc)
+ *   y = fl32(y_int8 + y16);  y = fl32(y + bias[n]);  Y = bf16_rne(y)
+ * with y_int8 the INT8 epilogue above without bias.
+ *
+ *   X              device, m x k fp16 (Q8_F16), row stride ldx.
+ *   w              INT8 weight (Q8_S8 or Q8_U8, zero point optional).
+ *   W16            device n x k fp16 original weight, row stride k, when the
+ *                  caller keeps it (llm_int8_has_fp16_weight); NULL (the default)
+ *                  uses fp16_rne(fl32(S[n] * fl32(q - Z))) for the outlier columns.
+ *   threshold      6.0 by default; <= 0 turns the decomposition off.
+ *   bias, Y, ldy   as q8_linear_w8a8.
+ *   outlier_mask   device [k] uint8 output, or NULL.
+ *   outlier_count  device int32 output, or NULL.
+ *   acc_debug      device m x n int32 raw INT8 accumulator, or NULL.
+ *   y16_debug      device m x n fp32 outlier-stream result, or NULL.
+ *   workspace      device scratch of at least
+ *                  q8_workspace_size(Q8_OP_LINEAR_INT8_MIXED, m, n, k) bytes,
+ *                  256-byte aligned; contents need no initialization.
+ */
+q8_status q8_linear_int8_mixed(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
+                               int64_t ldx, const q8_weight *w, const void *W16,
+                               float threshold, const float *bias, void *Y, int64_t ldy,
+                               uint8_t *outlier_mask, int32_t *outlier_count,
+                               int32_t *acc_debug, float *y16_debug, void *workspace,
+                               size_t ws_bytes, q8_stream_t stream);
+
+enum { Q8_OP_LINEAR_W8A8 = 0, Q8_OP_LINEAR_INT8_MIXED = 1 };
+
+/* Bytes of device workspace an operation needs for these sizes (host function,
+ * no device access).  The mixed operation sizes its outlier buffers for every
+ * column being an outlier, so no call can overflow them. */
+size_t q8_workspace_size(int op, int64_t m, int64_t n, int64_t k);
+
+/* Static, NUL-terminated description of a status code (host). */
+const char *q8_status_string(q8_status s);
+
+/* Waits for `stream`, then reads the current device's status word into *out
+ * (host pointer): Q8_OK, or the first device-side error recorded since the
+ * last clear (Q8_ERR_DEVICE_TIMEOUT). */
+q8_status q8_get_device_status(int32_t *out, q8_stream_t stream);
+
+/* Resets the current device's status word to Q8_OK (enqueued on `stream`). */
+q8_status q8_clear_device_status(q8_stream_t stream);
+
+/* Q8_OK when the current device can run this library, else
+ * Q8_ERR_UNSUPPORTED_ARCH or Q8_ERR_CUDA (host). */
+q8_status q8_device_check(void);
+
+/* Q8_VERSION of the built library (host). */
+int q8_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q8_H_ */

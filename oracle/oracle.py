@@ -72,6 +72,7 @@ def lib():
             "or_epilogue_int": [vp, vp, i64, vp, i64, vp, vp, vp, vp, vp, vp],
             "or_gemm_fp8": [vp, i64, vp, i64, i64, vp, i64, vp, i64, vp, vp, vp, vp, vp],
             "or_dequant_weight_f16": [vp, i32, i64, vp, vp, vp, i64, vp, i64, vp],
+            "or_dequant_weight": [vp, i32, i64, i64, i64, vp, vp, vp],
             "or_outlier_gemm": [vp, i64, vp, i64, vp, i64, vp, i64, vp, i64, vp],
             "or_merge": [vp, vp, i64, vp, i64, vp, vp],
         }
@@ -271,6 +272,17 @@ def dequant_weight_f16(wq, Sw, Zw, colidx, rows=None) -> np.ndarray:
     lib().or_dequant_weight_f16(_ptr(wq), int(wq.dtype == np.int8), wq.shape[1],
                                 _ptr(f32(Sw)), _ptr(f32(Zw)), _ptr(r), r.size, _ptr(ci),
                                 ci.size, _ptr(out))
+    return out
+
+
+def dequant_weight_codes(wq, kind: str, Sw, Zw=None) -> np.ndarray:
+    """fp32 S (q - Z) for every element.  kind: "s8", "u8" or "e4m3"."""
+    wq = np.ascontiguousarray(wq)
+    n, k = wq.shape
+    out = np.empty((n, k), np.float32)
+    f32 = lambda v: None if v is None else np.ascontiguousarray(v, dtype=np.float32)
+    lib().or_dequant_weight(_ptr(wq), {"s8": 0, "u8": 1, "e4m3": 2}[kind], n, k, wq.shape[1],
+                            _ptr(f32(Sw)), _ptr(f32(Zw)), _ptr(out))
     return out
 
 

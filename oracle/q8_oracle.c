@@ -482,6 +482,26 @@ void or_dequant_weight_f16(const void *q, int q_signed, int64_t ldq, const float
 }
 
 /*
+ * Dequantized weight in fp32, r = fl32(S[n] * fl32(q - Z[n])) for every element
+ * ([Xilyfe] "量化是什么": r = S (q - Z); [Fabric] 3.3 dequantize_weight).
+ * code_kind: 0 int8, 1 uint8, 2 E4M3 (decoded exactly); Z may be NULL.
+ */
+void or_dequant_weight(const void *q, int code_kind, int64_t n, int64_t k, int64_t ldq,
+                       const float *S, const float *Z, float *out) {
+    build_tables();
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            float code;
+            if (code_kind == 0) code = (float)((const int8_t *)q)[r * ldq + j];
+            else if (code_kind == 1) code = (float)((const uint8_t *)q)[r * ldq + j];
+            else code = (float)g_e4m3_signed[((const uint8_t *)q)[r * ldq + j]];
+            float d = Z ? code - Z[r] : code;
+            out[r * k + j] = S[r] * d;
+        }
+}
+
+/*
  * LLM.int8 outlier stream ([LLM.int8] 核心思想: columns beyond the threshold
  * are multiplied in fp16): y16[m, n] = fl32(sum_{j < count} X[m, idx[j]] *
  * W16[n, j]), products and sum in double.  X is the full M x K activation

@@ -1,0 +1,188 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+include/q8.h declares, and rejects bad arguments before touching a device.
+
+None of these launch a kernel.  Pointers passed here are never dereferenced:
+each call returns from host validation (or from the device check, which finds
+no usable sm_100a device on a CPU-only machine).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from bit_quantized_b200 import build as q8build
+
+q8build.build()
+from bit_quantized_b200 import q8  # noqa: E402
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "q8.h")
+FAKE = 0x10000          # 16-byte aligned, never dereferenced
+MIS = 0x10008           # 8-byte aligned only
+# Calls with valid arguments and fake pointers are made only where no GPU is
+# visible: there they stop at the device check; on a GPU they would launch.
+NO_GPU = not torch.cuda.is_available()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(q8_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(q8.LIB_PATH)
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(q8.EXPORTED) == names
+
+
+def test_version_matches_header():
+    m = re.search(r"#define Q8_VERSION (\d+)", open(HEADER).read())
+    assert q8.q8_version() == int(m.group(1))
+
+
+def test_status_strings():
+    for s in range(11):
+        assert q8.q8_status_string(s) not in ("", "unknown status")
+    assert q8.q8_status_string(99) == "unknown status"
+
+
+def test_workspace_size():
+    ws = q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, 512, 4096, 4096)
+    up = lambda v, a: (v + a - 1) // a * a
+    kp = 4096
+    want = (up(4096, 256) + up(4 * 4096, 256) + 256 + up(512 * 4096, 256) + 2 * up(4 * 512, 256)
+            + up(2 * 512 * kp, 256) + up(2 * 4096 * kp, 256))
+    assert ws == want
+    assert q8.q8_workspace_size(q8.Q8_OP_LINEAR_W8A8, 16, 4096, 4096) == 0
+    assert q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, 1, 16, 32) > 0
+
+
+L = q8.lib()
+_ns = None
+
+
+def qw(**kw):
+    args = dict(W=FAKE, w_dtype=q8.Q8_BF16, n=64, k=128, ldw=128, scheme=q8.Q8_ASYM_INT8,
+                code_dtype=q8.Q8_S8, codes=FAKE, scale=FAKE, zp=FAKE)
+    args.update(kw)
+    return L.q8_quantize_weight(args["W"], args["w_dtype"], args["n"], args["k"], args["ldw"],
+                                args["scheme"], args["code_dtype"], args["codes"], args["scale"],
+                                args["zp"], _ns)
+
+
+def test_quantize_weight_validation():
+    assert qw(W=None) == q8.Q8_ERR_NULL
+    assert qw(zp=None) == q8.Q8_ERR_NULL                       # asymmetric needs Z
+    assert qw(k=100, ldw=100) == q8.Q8_ERR_SHAPE               # K % 32
+    assert qw(ldw=64) == q8.Q8_ERR_SHAPE                       # ld < k
+    assert qw(n=-1) == q8.Q8_ERR_SHAPE
+    assert qw(w_dtype=q8.Q8_S8) == q8.Q8_ERR_DTYPE
+    assert qw(code_dtype=q8.Q8_E4M3) == q8.Q8_ERR_SCHEME
+    assert qw(scheme=q8.Q8_SYM_INT8, code_dtype=q8.Q8_U8) == q8.Q8_ERR_SCHEME
+    assert qw(scheme=7) == q8.Q8_ERR_SCHEME
+    assert qw(W=MIS) == q8.Q8_ERR_ALIGN
+    assert qw(ldw=132) == q8.Q8_ERR_ALIGN                      # 264 bytes
+    # valid arguments reach the device check: no sm_100a device here
+    if NO_GPU:
+        assert qw() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+    if NO_GPU:
+        assert qw(scheme=q8.Q8_SYM_INT8, zp=None) in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def qa(**kw):
+    args = dict(X=FAKE, x_dtype=q8.Q8_F16, m=16, k=256, ldx=256, scheme=q8.Q8_SYM_INT8, ub=0.0,
+                codes=FAKE, scale=FAKE, rowsum=FAKE)
+    args.update(kw)
+    return L.q8_quantize_act(args["X"], args["x_dtype"], args["m"], args["k"], args["ldx"],
+                             args["scheme"], args["ub"], args["codes"], args["scale"],
+                             args["rowsum"], _ns)
+
+
+def test_quantize_act_validation():
+    assert qa(codes=None) == q8.Q8_ERR_NULL
+    assert qa(k=48, ldx=48) == q8.Q8_ERR_SHAPE
+    assert qa(scheme=q8.Q8_ASYM_INT8) == q8.Q8_ERR_SCHEME
+    assert qa(x_dtype=q8.Q8_E4M3) == q8.Q8_ERR_DTYPE
+    assert qa(codes=MIS) == q8.Q8_ERR_ALIGN
+    if NO_GPU:
+        assert qa() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+    if NO_GPU:
+        assert qa(m=0) in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def _weight(code_dtype=q8.Q8_S8, zp=FAKE, n=64, k=128, ld=128):
+    return q8.CWeight(FAKE, code_dtype, FAKE, zp, n, k, ld)
+
+
+def _act(code_dtype=q8.Q8_S8, m=16, k=128, ld=128, rowsum=FAKE):
+    return q8.CAct(FAKE, code_dtype, FAKE, rowsum, m, k, ld)
+
+
+def lin(x=None, w=None, Y=FAKE, ldy=64):
+    x = x or _act()
+    w = w or _weight()
+    return L.q8_linear_w8a8(ctypes.byref(x), ctypes.byref(w), None, Y, ldy, None, None, 0, _ns)
+
+
+def test_linear_w8a8_validation():
+    assert lin(Y=None) == q8.Q8_ERR_NULL
+    assert lin(x=_act(rowsum=None)) == q8.Q8_ERR_NULL          # zero point needs row sums
+    assert lin(x=_act(k=256, ld=256)) == q8.Q8_ERR_SHAPE       # K mismatch
+    assert lin(w=_weight(n=40)) == q8.Q8_ERR_SHAPE             # N % 16
+    assert lin(ldy=32) == q8.Q8_ERR_SHAPE
+    assert lin(x=_act(code_dtype=q8.Q8_E4M3)) == q8.Q8_ERR_DTYPE   # fp8 x int8
+    assert lin(w=_weight(code_dtype=q8.Q8_E4M3)) == q8.Q8_ERR_SCHEME  # fp8 with zero point
+    assert lin(x=_act(k=65536, ld=65536), w=_weight(k=65536, ld=65536)) == q8.Q8_ERR_SHAPE
+    assert lin(Y=MIS) == q8.Q8_ERR_ALIGN
+    assert lin(ldy=68) == q8.Q8_ERR_ALIGN
+    if NO_GPU:
+        assert lin() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+    fx = _act(code_dtype=q8.Q8_E4M3, rowsum=None)
+    if NO_GPU:
+        assert lin(x=fx, w=_weight(code_dtype=q8.Q8_E4M3, zp=None)) in (
+            q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def mixed(w=None, ws=FAKE, ws_bytes=None, x_dtype=q8.Q8_F16, m=16, k=128, W16=None):
+    w = w or _weight(k=k, ld=k)
+    if ws_bytes is None:
+        ws_bytes = q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, m, w.n, k)
+    return L.q8_linear_int8_mixed(FAKE, x_dtype, m, k, k, ctypes.byref(w), W16, 6.0, None, FAKE,
+                                  w.n, None, None, None, None, ws, ws_bytes, _ns)
+
+
+def test_linear_int8_mixed_validation():
+    assert mixed(ws=None) == q8.Q8_ERR_WORKSPACE
+    assert mixed(ws_bytes=100) == q8.Q8_ERR_WORKSPACE
+    assert mixed(ws=FAKE + 16) == q8.Q8_ERR_ALIGN              # workspace must be 256-aligned
+    assert mixed(x_dtype=q8.Q8_BF16) == q8.Q8_ERR_DTYPE
+    assert mixed(w=_weight(code_dtype=q8.Q8_E4M3, zp=None)) == q8.Q8_ERR_DTYPE
+    assert mixed(W16=MIS) == q8.Q8_ERR_ALIGN
+    if NO_GPU:
+        assert mixed() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def test_outlier_act_validation():
+    f = L.q8_outlier_quantize_act
+    args = [FAKE, q8.Q8_F16, 16, 128, 128, 6.0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, _ns]
+    a = list(args); a[10] = None
+    assert f(*a) == q8.Q8_ERR_NULL
+    a = list(args); a[13] = 64
+    assert f(*a) == q8.Q8_ERR_SHAPE                             # ldo < round_up(k, 64)
+    a = list(args); a[1] = q8.Q8_BF16
+    assert f(*a) == q8.Q8_ERR_DTYPE
+    a = list(args); a[12] = MIS
+    assert f(*a) == q8.Q8_ERR_ALIGN
+    if NO_GPU:
+        assert f(*args) in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def test_device_calls_report_no_device():
+    assert q8.q8_device_check() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH, q8.Q8_OK)
+    v = ctypes.c_int32(0)
+    assert L.q8_get_device_status(None, _ns) == q8.Q8_ERR_NULL

@@ -1,0 +1,243 @@
+"""GPU parity of the W8A8 and LLM.int8 linears against the CPU oracle.
+
+INT8 accumulators and INT8 W8A8 outputs are compared bit for bit; FP8 and
+mixed outputs within the bound in tests/parity.py.  Full-size workloads are
+compared on sampled rows and columns in the same launch configuration the
+benchmark uses; smaller shapes that span several tiles, ragged tails and the
+decode path are compared in full.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+from bit_quantized_b200 import q8  # noqa: E402
+
+DEV = "cuda:0"
+
+
+def _int8_case(x32, w32, scheme, codes, X_dev, W_dev, bias=None, rows=None, cols=None,
+               what=""):
+    """Runs quantize + linear on the GPU and checks codes, acc and Y against the oracle."""
+    qa = q8.q8_quantize_act(X_dev, "int8")
+    qw = q8.q8_quantize_weight(W_dev, scheme, codes)
+    m, n = X_dev.shape[0], W_dev.shape[0]
+    acc = torch.empty((m, n), dtype=torch.int32, device=DEV)
+    b_dev = None if bias is None else torch.from_numpy(bias).to(DEV)
+    Y = q8.q8_linear_w8a8(qa, qw, bias=b_dev, acc_debug=acc)
+    torch.cuda.synchronize()
+    xq, Sx, rs = O.quant_act_int8(x32)
+    wq, Sw, Zw = O.quant_weight(w32, scheme, codes)
+    r = np.arange(m) if rows is None else rows
+    c = np.arange(n) if cols is None else cols
+    acc_ref, y_ref, Y_ref = O.linear_w8a8_int8(xq, Sx, rs, wq, Sw, Zw, bias, r, c)
+    P.assert_equal(acc.cpu().numpy()[np.ix_(r, c)], acc_ref.astype(np.int32), what + " acc")
+    Yb = P.bf16_bits(Y)[np.ix_(r, c)]
+    P.assert_equal(Yb, Y_ref, what + " Y")
+    P.assert_bf16_within(Yb, y_ref, 0.0, what)
+
+
+def _rand(m, k, dtype, seed, std=1.0):
+    X = workloads.random_matrix(m, k, dtype, seed, std)
+    return X, P.host_f32(X)
+
+
+# ------------------------------------------------------------------ INT8 W8A8, full size
+
+def test_decode_q_proj_full():
+    X, W, info, x32, w32 = P.workload("decode_q_proj")
+    _int8_case(x32, w32, "asym", "u8", X.to(DEV), W.to(DEV), what="decode_q_proj")
+
+
+def test_prefill_ffn_up_sampled():
+    X, W, info, x32, w32 = P.workload("prefill_ffn_up")
+    rows = P.sample_indices(X.shape[0], 96, 1)
+    cols = P.sample_indices(W.shape[0], 1536, 2)
+    _int8_case(x32, w32, "sym", "s8", X.to(DEV), W.to(DEV), rows=rows, cols=cols,
+               what="prefill_ffn_up")
+
+
+# ------------------------------------------------------------------ INT8 W8A8, shapes
+
+@pytest.mark.parametrize("m,n,k", [
+    (1, 128, 256),          # single token, decode kernel
+    (16, 4096, 4096),       # decode shape, s8 weights
+    (17, 272, 160),         # decode kernel NT=32, N % 32 == 16, ragged K block
+    (64, 512, 1024),        # decode kernel NT=64
+    (65, 384, 512),         # tile kernel, one partial M tile
+    (300, 640, 1024),       # tile kernel, several tiles, ragged M
+    (384, 2304, 384),       # tile kernel BN=256 path (tiles >= SMs)
+    (130, 48, 32),          # K = 32: one K block mostly out of bounds; N = 48
+])
+@pytest.mark.parametrize("scheme,codes", [("asym", "s8"), ("asym", "u8"), ("sym", "s8")])
+def test_int8_shapes(m, n, k, scheme, codes):
+    X, x32 = _rand(m, k, torch.bfloat16, seed=m + n + k)
+    W, w32 = _rand(n, k, torch.bfloat16, seed=m * n + k, std=0.02)
+    _int8_case(x32, w32, scheme, codes, X.to(DEV), W.to(DEV), what=f"{m}x{n}x{k} {scheme}/{codes}")
+
+
+@pytest.mark.parametrize("m", [8, 256])
+def test_int8_bias(m):
+    X, x32 = _rand(m, 512, torch.bfloat16, seed=41)
+    W, w32 = _rand(320, 512, torch.bfloat16, seed=42, std=0.02)
+    bias = np.linspace(-3, 3, 320).astype(np.float32)
+    _int8_case(x32, w32, "asym", "s8", X.to(DEV), W.to(DEV), bias=bias, what=f"bias m={m}")
+
+
+def test_int8_empty_m():
+    W = workloads.random_matrix(64, 64, torch.bfloat16, 1, 0.02).to(DEV)
+    qw = q8.q8_quantize_weight(W, "asym", "s8")
+    qa = q8.q8_quantize_act(torch.empty((0, 64), dtype=torch.bfloat16, device=DEV), "int8")
+    Y = q8.q8_linear_w8a8(qa, qw)
+    torch.cuda.synchronize()
+    assert Y.shape == (0, 64)
+
+
+def test_int8_strided_output():
+    X, x32 = _rand(20, 256, torch.bfloat16, seed=43)
+    W, w32 = _rand(64, 256, torch.bfloat16, seed=44, std=0.02)
+    qa = q8.q8_quantize_act(X.to(DEV), "int8")
+    qw = q8.q8_quantize_weight(W.to(DEV), "sym", "s8")
+    big = torch.full((20, 96), 7.0, dtype=torch.bfloat16, device=DEV)
+    q8.q8_linear_w8a8(qa, qw, out=big[:, 16:80])
+    torch.cuda.synchronize()
+    xq, Sx, rs = O.quant_act_int8(x32)
+    wq, Sw, _ = O.quant_weight(w32, "sym")
+    _, _, Y_ref = O.linear_w8a8_int8(xq, Sx, rs, wq, Sw)
+    P.assert_equal(P.bf16_bits(big[:, 16:80]), Y_ref, "strided Y")
+    assert (big[:, :16] == 7).all() and (big[:, 80:] == 7).all(), "write outside the output view"
+
+
+# ------------------------------------------------------------------ FP8
+
+def _fp8_case(x32, w32, X_dev, W_dev, ub, bias=None, rows=None, cols=None, what=""):
+    qa = q8.q8_quantize_act(X_dev, "fp8", clip_ub=ub)
+    qw = q8.q8_quantize_weight(W_dev, "fp8", "e4m3")
+    m, n = X_dev.shape[0], W_dev.shape[0]
+    b_dev = None if bias is None else torch.from_numpy(bias).to(DEV)
+    acc = torch.empty((m, n), dtype=torch.float32, device=DEV)
+    Y = q8.q8_linear_w8a8(qa, qw, bias=b_dev, acc_debug=acc)
+    torch.cuda.synchronize()
+    xq, Sx = O.quant_act_fp8(x32, ub)
+    wq, Sw, _ = O.quant_weight(w32, "fp8")
+    r = np.arange(m) if rows is None else rows
+    c = np.arange(n) if cols is None else cols
+    acc_ref, y_ref, _ = O.linear_w8a8_fp8(xq, Sx, wq, Sw, bias, r, c)
+    a_abs = np.abs(O.widen_e4m3(xq[r])).astype(np.float64)
+    b_abs = np.abs(O.widen_e4m3(wq[c])).astype(np.float64)
+    mag = a_abs @ b_abs.T
+    k = x32.shape[1]
+    acc_bound = k * 2.0**-22 * mag
+    got_acc = acc.cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+    assert np.all(np.abs(got_acc - acc_ref) <= acc_bound + 2.0**-24 * np.abs(acc_ref)), what + " acc"
+    extra = acc_bound * Sx[r][:, None].astype(np.float64) * Sw[c][None, :].astype(np.float64)
+    return P.assert_bf16_within(P.bf16_bits(Y)[np.ix_(r, c)], y_ref, extra, what)
+
+
+def test_fp8_rowwise_sampled():
+    X, W, info, x32, w32 = P.workload("fp8_rowwise")
+    rows = P.sample_indices(X.shape[0], 64, 3)
+    cols = P.sample_indices(W.shape[0], 1024, 4)
+    _fp8_case(x32, w32, X.to(DEV), W.to(DEV), 1200.0, rows=rows, cols=cols, what="fp8_rowwise")
+
+
+@pytest.mark.parametrize("m,n,k", [(5, 256, 512), (16, 1024, 2048), (200, 528, 1024),
+                                   (256, 2560, 512)])
+def test_fp8_shapes(m, n, k):
+    X, x32 = _rand(m, k, torch.bfloat16, seed=m + 7 * k)
+    X[0, 0] = 3000.0                        # beyond the upper bound: saturates
+    x32 = P.host_f32(X)
+    W, w32 = _rand(n, k, torch.bfloat16, seed=n + k, std=0.02)
+    bias = np.linspace(-1, 1, n).astype(np.float32)
+    _fp8_case(x32, w32, X.to(DEV), W.to(DEV), 1200.0, bias=bias, what=f"fp8 {m}x{n}x{k}")
+
+
+# ------------------------------------------------------------------ LLM.int8 mixed
+
+def _mixed_case(X, W, threshold, codes="s8", has_fp16_weight=False, bias=None, rows=None,
+                cols=None, what=""):
+    x32, w32 = P.host_f32(X), P.host_f32(W)
+    Wd = W.to(DEV)
+    qw = q8.q8_quantize_weight(Wd, "asym", codes)
+    b_dev = None if bias is None else torch.from_numpy(bias).to(DEV)
+    Y, dbg = q8.q8_linear_int8_mixed(X.to(DEV), qw, threshold,
+                                     W16=Wd if has_fp16_weight else None, bias=b_dev, debug=True)
+    torch.cuda.synchronize()
+    wq, Sw, Zw = O.quant_weight(w32, "asym", codes)
+    m, n = X.shape[0], W.shape[0]
+    r = np.arange(m) if rows is None else rows
+    c = np.arange(n) if cols is None else cols
+    ref = O.linear_int8_mixed(x32, wq, Sw, Zw, threshold, w16_full=w32 if has_fp16_weight else None,
+                              bias=bias, rows=r, cols=c)
+    P.assert_equal(dbg["mask"].cpu().numpy(), ref["mask"], what + " mask")
+    assert int(dbg["count"].item()) == ref["count"], what + " count"
+    P.assert_equal(dbg["acc"].cpu().numpy()[np.ix_(r, c)], ref["acc"].astype(np.int32), what + " acc")
+    # outlier stream: fp32 accumulation of fp16 products over count columns
+    y16 = dbg["y16"].cpu().numpy()[np.ix_(r, c)].astype(np.float64)
+    mag16 = np.abs(x32[np.ix_(r, ref["idx"])]).astype(np.float64) @ np.abs(ref["w16"][c]).T.astype(np.float64)
+    kb = max(ref["count"], 1) * 2.0**-22 * mag16
+    assert np.all(np.abs(y16 - ref["y16"]) <= kb + 2.0**-24 * np.abs(ref["y16"])), what + " y16"
+    if ref["count"] > 0:
+        fro = np.linalg.norm(y16 - ref["y16"]) / max(np.linalg.norm(ref["y16"]), 1e-30)
+        assert fro <= 1e-3, what + f" y16 relative Frobenius {fro}"
+    return P.assert_bf16_within(P.bf16_bits(Y)[np.ix_(r, c)], ref["y"], kb, what), ref["count"]
+
+
+def test_tiny_mixed_full():
+    X, W, info, x32, w32 = P.workload("tiny_mixed")
+    _, count = _mixed_case(X, W, 6.0, what="tiny_mixed")
+    assert count == 2
+
+
+def test_mixed_512_sampled():
+    X, W, info, x32, w32 = P.workload("mixed_512")
+    cols = P.sample_indices(W.shape[0], 1024, 5)
+    _mixed_case(X, W, 6.0, cols=cols, what="mixed_512")
+
+
+@pytest.mark.parametrize("threshold", [0.0, float("inf"), 1e-30, 2.5])
+def test_mixed_thresholds(threshold):
+    X = workloads.random_matrix(40, 320, torch.float16, seed=51)
+    X[:, 17] *= 20
+    W = workloads.random_matrix(96, 320, torch.float16, seed=52, std=0.02)
+    _mixed_case(X, W, threshold, what=f"T={threshold}")
+
+
+def test_mixed_off_equals_w8a8_bit_exact():
+    X = workloads.random_matrix(48, 256, torch.float16, seed=53)
+    X[:, 9] *= 15
+    W = workloads.random_matrix(128, 256, torch.float16, seed=54, std=0.02)
+    Wd = W.to(DEV)
+    qw = q8.q8_quantize_weight(Wd, "asym", "s8")
+    Ym = q8.q8_linear_int8_mixed(X.to(DEV), qw, 0.0)
+    Yp = q8.q8_linear_w8a8(q8.q8_quantize_act(X.to(DEV), "int8"), qw)
+    torch.cuda.synchronize()
+    P.assert_equal(P.bf16_bits(Ym), P.bf16_bits(Yp), "threshold 0 vs W8A8")
+
+
+@pytest.mark.parametrize("codes,fp16w", [("u8", False), ("s8", True)])
+def test_mixed_variants(codes, fp16w):
+    X = workloads.random_matrix(130, 512, torch.float16, seed=55)
+    X[:, [1, 300, 301]] *= 12
+    W = workloads.random_matrix(272, 512, torch.float16, seed=56, std=0.02)
+    bias = np.linspace(-1, 1, 272).astype(np.float32)
+    _mixed_case(X, W, 6.0, codes=codes, has_fp16_weight=fp16w, bias=bias,
+                what=f"mixed {codes} fp16w={fp16w}")
+
+
+def test_mixed_many_outliers():
+    # 100 outlier columns: two fp16 K blocks of 64 in the outlier GEMM
+    X = workloads.random_matrix(64, 1024, torch.float16, seed=57)
+    X[:, ::10] *= 10
+    W = workloads.random_matrix(128, 1024, torch.float16, seed=58, std=0.02)
+    _, count = _mixed_case(X, W, 6.0, what="many outliers")
+    assert count > 64
+
+
+def test_device_status_clean():
+    assert q8.q8_get_device_status() == 0

@@ -178,3 +178,19 @@ def test_mixed_bias_added_after_merge():
     r = O.linear_int8_mixed(x, wq, Sw, Zw, 6.0, bias=bias)
     r0 = O.linear_int8_mixed(x, wq, Sw, Zw, 6.0)
     assert np.array_equal(r["y"], (r0["y"] + bias).astype(np.float32))
+
+
+@pytest.mark.parametrize("kind", ["s8", "u8", "e4m3"])
+def test_dequant_weight_codes(kind):
+    w = workloads.random_matrix(16, 64, torch.bfloat16, 12, 0.02).float().numpy()
+    scheme = {"s8": "asym", "u8": "asym", "e4m3": "fp8"}[kind]
+    q, S, Z = O.quant_weight(w, scheme, {"s8": "s8", "u8": "u8", "e4m3": "e4m3"}[kind])
+    d = O.dequant_weight_codes(q, kind, S, Z)
+    if kind == "e4m3":
+        vals = torch.from_numpy(q.view(np.int8)).view(torch.float8_e4m3fn).double().numpy()
+        exact = S[:, None].astype(np.float64) * vals
+    else:
+        exact = S[:, None].astype(np.float64) * (q.astype(np.float64) - Z[:, None])
+    assert np.all(np.abs(d - exact) <= 2.0**-24 * np.abs(exact))
+    # dequantized weights sit within the quantization error of the originals
+    assert np.all(np.abs(d - w) <= np.maximum(S[:, None] * 0.51, np.abs(w) * 2.0**-3))
