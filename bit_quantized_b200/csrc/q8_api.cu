@@ -68,10 +68,11 @@ q8_status launch_status(cudaError_t e) {
 }
 
 q8_status check_weight(const q8_weight* w) {
-    if (!w || !w->codes || !w->scale) return Q8_ERR_NULL;
+    if (!w) return Q8_ERR_NULL;
     if (w->n < 0 || w->k <= 0 || w->n > kMaxDim || w->k > kMaxDim || w->k % 32 != 0 ||
         w->n % 16 != 0 || w->ld < w->k)
         return Q8_ERR_SHAPE;
+    if (w->n > 0 && (!w->codes || !w->scale)) return Q8_ERR_NULL;
     if (w->code_dtype != Q8_S8 && w->code_dtype != Q8_U8 && w->code_dtype != Q8_E4M3)
         return Q8_ERR_DTYPE;
     if (w->code_dtype == Q8_E4M3 && w->zero_point) return Q8_ERR_SCHEME;
@@ -144,8 +145,6 @@ size_t q8_workspace_size(int op, int64_t m, int64_t n, int64_t k) {
 q8_status q8_quantize_weight(const void* W, q8_dtype w_dtype, int64_t n, int64_t k, int64_t ldw,
                              q8_scheme scheme, q8_dtype code_dtype, void* codes, float* scale,
                              float* zero_point, q8_stream_t stream) {
-    if (!W || !codes || !scale) return Q8_ERR_NULL;
-    if (scheme == Q8_ASYM_INT8 && !zero_point) return Q8_ERR_NULL;
     if (n < 0 || k <= 0 || n > kMaxDim || k > kMaxDim || k % 32 != 0) return Q8_ERR_SHAPE;
     if (!float_input(w_dtype)) return Q8_ERR_DTYPE;
     if (!(ldw >= k)) return Q8_ERR_SHAPE;
@@ -155,6 +154,9 @@ q8_status q8_quantize_weight(const void* W, q8_dtype w_dtype, int64_t n, int64_t
         case Q8_FP8_E4M3: if (code_dtype != Q8_E4M3) return Q8_ERR_SCHEME; break;
         default: return Q8_ERR_SCHEME;
     }
+    if (n == 0) return Q8_OK;   // empty call
+    if (!W || !codes || !scale) return Q8_ERR_NULL;
+    if (scheme == Q8_ASYM_INT8 && !zero_point) return Q8_ERR_NULL;
     if (!aligned16(W) || !aligned16(codes) || !ld_ok(ldw, k, w_dtype)) return Q8_ERR_ALIGN;
     q8_status st = check_device();
     if (st != Q8_OK) return st;
@@ -181,10 +183,11 @@ q8_status q8_dequantize_weight(const q8_weight* w, q8_dtype out_dtype, void* out
 q8_status q8_quantize_act(const void* X, q8_dtype x_dtype, int64_t m, int64_t k, int64_t ldx,
                           q8_scheme scheme, float clip_ub, void* codes, float* scale,
                           int32_t* rowsum, q8_stream_t stream) {
-    if (!X || !codes || !scale) return Q8_ERR_NULL;
     if (m < 0 || k <= 0 || m > kMaxDim || k > kMaxDim || k % 32 != 0 || ldx < k) return Q8_ERR_SHAPE;
     if (!float_input(x_dtype)) return Q8_ERR_DTYPE;
     if (scheme != Q8_SYM_INT8 && scheme != Q8_FP8_E4M3) return Q8_ERR_SCHEME;
+    if (m == 0) return Q8_OK;   // empty call: pointers may be NULL, nothing is launched
+    if (!X || !codes || !scale) return Q8_ERR_NULL;
     if (!aligned16(X) || !aligned16(codes) || !ld_ok(ldx, k, x_dtype)) return Q8_ERR_ALIGN;
     q8_status st = check_device();
     if (st != Q8_OK) return st;
@@ -201,8 +204,9 @@ static q8_status validate_outlier_act(const void* X, q8_dtype x_dtype, int64_t m
                                       int64_t ldx, void* codes, float* scale, int32_t* rowsum,
                                       uint8_t* mask, int32_t* idx, int32_t* count,
                                       void* x_outlier, int64_t ldo) {
-    if (!X || !codes || !scale || !rowsum || !mask || !idx || !count) return Q8_ERR_NULL;
+    if (!mask || !idx || !count) return Q8_ERR_NULL;
     if (m < 0 || k <= 0 || m > kMaxDim || k > kMaxKInt8 || k % 32 != 0 || ldx < k) return Q8_ERR_SHAPE;
+    if (m > 0 && (!X || !codes || !scale || !rowsum)) return Q8_ERR_NULL;
     if (x_outlier && (ldo < (k + 63) / 64 * 64)) return Q8_ERR_SHAPE;
     if (x_dtype != Q8_F16) return Q8_ERR_DTYPE;
     if (!aligned16(X) || !aligned16(codes) || !ld_ok(ldx, k, x_dtype)) return Q8_ERR_ALIGN;
@@ -247,11 +251,13 @@ q8_status q8_linear_w8a8(const q8_act* x, const q8_weight* w, const float* bias,
     (void)ws_bytes;
     q8_status st = check_weight(w);
     if (st != Q8_OK) return st;
-    if (!x || !x->codes || !x->scale || !Y) return Q8_ERR_NULL;
+    if (!x) return Q8_ERR_NULL;
     if (x->m < 0 || x->m > kMaxDim || x->k != w->k || x->ld < x->k || ldy < w->n) return Q8_ERR_SHAPE;
     const bool fp8 = x->code_dtype == Q8_E4M3;
     if (fp8 != (w->code_dtype == Q8_E4M3) || (x->code_dtype != Q8_S8 && !fp8)) return Q8_ERR_DTYPE;
     if (!fp8 && w->k > kMaxKInt8) return Q8_ERR_SHAPE;
+    if (x->m == 0 || w->n == 0) return Q8_OK;   // empty call
+    if (!x->codes || !x->scale || !Y) return Q8_ERR_NULL;
     if (!fp8 && w->zero_point && !x->rowsum) return Q8_ERR_NULL;
     if (!aligned16(x->codes) || !aligned16(x->scale) || x->ld % 16 != 0 || !aligned16(Y) ||
         ldy % 8 != 0 || (bias && !aligned16(bias)) || (acc_debug && !aligned16(acc_debug)))
@@ -278,10 +284,11 @@ q8_status q8_linear_int8_mixed(const void* X, q8_dtype x_dtype, int64_t m, int64
                                void* workspace, size_t ws_bytes, q8_stream_t stream) {
     q8_status st = check_weight(w);
     if (st != Q8_OK) return st;
-    if (!X || !Y) return Q8_ERR_NULL;
     if (w->code_dtype == Q8_E4M3) return Q8_ERR_DTYPE;
     if (x_dtype != Q8_F16) return Q8_ERR_DTYPE;
     if (m < 0 || m > kMaxDim || k != w->k || k > kMaxKInt8 || ldx < k || ldy < w->n) return Q8_ERR_SHAPE;
+    if (m == 0 || w->n == 0) return Q8_OK;   // empty call
+    if (!X || !Y) return Q8_ERR_NULL;
     if (!aligned16(X) || !ld_ok(ldx, k, x_dtype) || !aligned16(Y) || ldy % 8 != 0 ||
         (W16 && !aligned16(W16)) || (bias && !aligned16(bias)) ||
         (acc_debug && !aligned16(acc_debug)) || (y16_debug && !aligned16(y16_debug)))
@@ -305,7 +312,6 @@ q8_status q8_linear_int8_mixed(const void* X, q8_dtype x_dtype, int64_t m, int64
     __half* wo = reinterpret_cast<__half*>(p);
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (m == 0) return Q8_OK;
     st = run_outlier_act(X, m, k, ldx, threshold, codes, sx, rowsum, mask, idx, count, xo, kp, s);
     if (st != Q8_OK) return st;
     st = launch_status(launch_gather_weight_outliers(*w, static_cast<const __half*>(W16), idx,
