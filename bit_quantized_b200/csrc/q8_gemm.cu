@@ -36,6 +36,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <climits>
 #include <cstring>
 #include <mutex>
 
@@ -157,7 +158,10 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const uint32_t tmem_base = tmem_base_sh;
 
     int n16_kb = 0;
-    if constexpr (MIXED) n16_kb = (*p.outlier_count + 63) / 64;
+    if constexpr (MIXED) {
+        pdl_wait();   // the outlier count comes from the previous kernels
+        n16_kb = (*p.outlier_count + 63) / 64;
+    }
     const int total_kb = num_kb + n16_kb;
     const int num_tiles = tiles_m * tiles_n;
 
@@ -170,6 +174,7 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 tma_prefetch_desc(&tmA16);
                 tma_prefetch_desc(&tmB16);
             }
+            pdl_wait();   // operands may come from the previous kernel
             uint32_t issued = 0;             // stages that ever received a load
             uint32_t last_par = 0;           // parity of each stage's last load
             int stage = 0;
@@ -268,6 +273,7 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue
+        pdl_wait();   // scales and row sums may come from the previous kernel
         const int q = warp & 3;  // this warp's TMEM lane quarter
         const bool has_zp = p.zw != nullptr;
         int buf = 0;
@@ -379,7 +385,9 @@ struct DecodeCfg {
     static constexpr int A_BYTES = kBM * kBKB;   // 128 weight rows
     static constexpr int B_BYTES = NT * kBKB;    // NT token rows
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int RED_BYTES = NT * kBM * 4;
+    // Partials pushed by every rank: [rank][tokens owned][128 channels], at most
+    // 8 ranks each owning ceil(NT / ranks) tokens.
+    static constexpr int RED_BYTES = (NT + 8) * kBM * 4;
     static constexpr int STAGES_RAW = (kSmemBudget - RED_BYTES) / STAGE;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static constexpr int TMEM_COLS = NT < 32 ? 32 : NT;
@@ -389,11 +397,11 @@ struct DecodeCfg {
 template <int NT, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                   const EpiParams p, int num_kb, int kb_per_split, int splits) {
+                   const EpiParams p, int num_kb, int kb_per_split, int splits, int nstages) {
     using C = DecodeCfg<NT, KIND>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint32_t* red = reinterpret_cast<uint32_t*>(smem + C::STAGES * C::STAGE);  // [NT][128]
+    uint32_t* red = reinterpret_cast<uint32_t*>(smem + nstages * C::STAGE);  // [NT][128]
     __shared__ __align__(8) uint64_t full_bar[C::STAGES];
     __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
     __shared__ __align__(8) uint64_t tfull_bar;
@@ -410,7 +418,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     const int my_kb = kb1 > kb0 ? kb1 - kb0 : 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
+        for (int s = 0; s < nstages; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
         }
@@ -432,11 +440,23 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         if (elect_one()) {
             tma_prefetch_desc(&tmW);
             tma_prefetch_desc(&tmX);
-            uint32_t issued = 0, last_par = 0;
-            int stage = 0;
-            uint32_t phase = 0;
+            // The weights do not depend on the previous kernel: their first
+            // ring of loads goes out before the programmatic-launch wait, the
+            // activation codes of the same stages right after it.
+            const int first = my_kb < nstages ? my_kb : nstages;
+            for (int i = 0; i < first; ++i) {
+                uint8_t* sa = smem + i * C::STAGE;
+                mbar_arrive_expect_tx(&full_bar[i], C::STAGE);
+                tma_load_2d(sa, &tmW, &full_bar[i], (kb0 + i) * kBKB, tn * kBM);
+            }
+            pdl_wait();
+            for (int i = 0; i < first; ++i)
+                tma_load_2d(smem + i * C::STAGE + C::A_BYTES, &tmX, &full_bar[i], (kb0 + i) * kBKB, 0);
+            uint32_t issued = (1u << first) - 1u, last_par = 0;
+            int stage = first == nstages ? 0 : first;
+            uint32_t phase = first == nstages ? 1u : 0u;
             bool ok = true;
-            for (int kb = kb0; kb < kb1; ++kb) {
+            for (int kb = kb0 + first; kb < kb1; ++kb) {
                 if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
                     ok = false;
                     break;
@@ -447,13 +467,13 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                 tma_load_2d(sa + C::A_BYTES, &tmX, &full_bar[stage], kb * kBKB, 0);
                 issued |= 1u << stage;
                 last_par = (last_par & ~(1u << stage)) | (phase << stage);
-                if (++stage == C::STAGES) {
+                if (++stage == nstages) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
             if (!ok)
-                for (int s = 0; s < C::STAGES; ++s)
+                for (int s = 0; s < nstages; ++s)
                     if (issued & (1u << s)) mbar_wait(&full_bar[s], (last_par >> s) & 1, nullptr, nullptr);
         }
         __syncwarp();
@@ -482,7 +502,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                         mma_issue<kKindI8>(tmem_base, ad + 2 * ks, bd + 2 * ks, idesc, (i | ks) != 0);
                 }
                 tc_commit(&empty_bar[stage]);
-                if (++stage == C::STAGES) {
+                if (++stage == nstages) {
                     stage = 0;
                     phase ^= 1;
                 }
@@ -492,33 +512,45 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         }
         __syncwarp();
     } else {
-        // Epilogue warps: TMEM partial -> own shared memory, laid out [token][channel].
+        // Epilogue warps: push this rank's TMEM partial for token t into the
+        // shared memory of the rank that finishes t (t % splits), at slot
+        // [rank][t / splits][channel].
         const int q = warp & 3;
         const int ch = q * 32 + lane;
+        const int tpo = (NT + splits - 1) / splits;     // tokens owned per rank
         bool have = my_kb > 0 && mbar_wait(&tfull_bar, 0, &abort_sh, p.status);
         if (have) tc_fence_after();
         __syncwarp();
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+        const uint32_t red_base = smem_addr(red);
 #pragma unroll
         for (int c = 0; c < NT; c += 16) {
             uint32_t r[16];
             tmem_ld16(tb + c, r);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) red[(c + i) * kBM + ch] = have ? r[i] : 0u;
+            for (int i = 0; i < 16; ++i) {
+                const int t = c + i;
+                const uint32_t owner = static_cast<uint32_t>(t % splits);
+                const uint32_t off = ((rank * tpo + t / splits) * kBM + ch) * 4u;
+                st_shared_cluster_u32(map_shared_rank(red_base + off, owner), have ? r[i] : 0u);
+            }
         }
         __syncwarp();
     }
 
-    // Partials of the whole cluster are visible after this barrier.
+    // Every rank's pushed partials are visible after this barrier; after it no
+    // CTA touches another CTA's shared memory, so each may exit when done.
     __syncthreads();
     cluster_sync();
 
     if (warp >= 2) {
-        // Rank r finishes the tokens t with t % splits == r, summing the ranks'
+        pdl_wait();   // token scales and row sums come from the previous kernel
+        // Rank r finishes the tokens t with t % splits == r, summing the
         // partials in rank order.
         const int q = warp & 3;
         const int ch = q * 32 + lane;
+        const int tpo = (NT + splits - 1) / splits;
         const int n = tn * kBM + ch;
         const bool has_zp = p.zw != nullptr;
         const bool col_ok = n < p.n;
@@ -526,19 +558,19 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         const float zw = (col_ok && has_zp) ? p.zw[n] : 0.f;
         const float bias = (col_ok && p.bias) ? p.bias[n] : 0.f;
         for (int t = static_cast<int>(rank); t < NT && t < p.m; t += splits) {
-            const uint32_t local = smem_addr(&red[t * kBM + ch]);
+            const int tl = t / splits;
             uint32_t acc_bits;
             float v;
             if constexpr (KIND == kE4M3) {
                 float s = 0.f;
                 for (int r = 0; r < splits; ++r)
-                    s = __fadd_rn(s, __uint_as_float(ld_shared_cluster_u32(map_shared_rank(local, r))));
+                    s = __fadd_rn(s, __uint_as_float(red[(r * tpo + tl) * kBM + ch]));
                 acc_bits = __float_as_uint(s);
                 v = __fmul_rn(__fmul_rn(s, p.sx[t]), sw);
             } else {
                 int32_t s = 0;
                 for (int r = 0; r < splits; ++r)
-                    s += static_cast<int32_t>(ld_shared_cluster_u32(map_shared_rank(local, r)));
+                    s += static_cast<int32_t>(red[(r * tpo + tl) * kBM + ch]);
                 acc_bits = static_cast<uint32_t>(s);
                 v = dequant_int(s, zw, has_zp ? p.rowsum[t] : 0, p.sx[t], sw, has_zp);
             }
@@ -551,9 +583,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         }
     }
 
-    // Keep this CTA's shared memory alive until every rank has read it.
     __syncthreads();
-    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
@@ -631,8 +661,21 @@ q8_status run_tile(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     const int tiles = tiles_m * tiles_n;
     const int num_kb = static_cast<int>((a.k + kBKB - 1) / kBKB);
     const int grid = tiles < sm_count() ? tiles : sm_count();
-    kern<<<grid, kThreads, C::SMEM, s>>>(tA, tB, tA16, tB16, ep, num_kb, tiles_m, tiles_n);
-    return cudaGetLastError() == cudaSuccess ? Q8_OK : Q8_ERR_LAUNCH;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tA16, tB16, ep, num_kb, tiles_m, tiles_n) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    return Q8_OK;
 }
 
 template <int NT, int KIND>
@@ -646,29 +689,36 @@ q8_status run_decode(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
     const int tiles_n = static_cast<int>((a.n + kBM - 1) / kBM);
     const int num_kb = static_cast<int>((a.k + kBKB - 1) / kBKB);
-    // Split K so that the grid covers the SMs once, at most 8 CTAs per cluster,
-    // with every split non-empty.
-    int want = sm_count() / tiles_n;
+    // Split K across the CTAs of a cluster (at most 8, every split non-empty)
+    // so that the grid fills the SMs at two CTAs per SM, which the short stage
+    // ring of a split allows.
+    int want = 2 * sm_count() / tiles_n;
     if (want < 1) want = 1;
     if (want > 8) want = 8;
     if (want > num_kb) want = num_kb;
     const int per = (num_kb + want - 1) / want;
     const int splits = (num_kb + per - 1) / per;
+    const int nstages = per < C::STAGES ? per : C::STAGES;
+    const int smem = nstages * C::STAGE + C::RED_BYTES + 1024;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles_n), static_cast<unsigned>(splits), 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = static_cast<unsigned>(splits);
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tW, tX, ep, num_kb, per, splits) != cudaSuccess)
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tW, tX, ep, num_kb, per, splits, nstages) != cudaSuccess) {
+        cudaGetLastError();
         return Q8_ERR_LAUNCH;
+    }
     return Q8_OK;
 }
 
@@ -677,9 +727,23 @@ q8_status dispatch_kind(const LinearArgs& a, const EpiParams& ep, cudaStream_t s
     if (a.m <= 16) return run_decode<16, KIND>(a, ep, s);
     if (a.m <= 32) return run_decode<32, KIND>(a, ep, s);
     if (a.m <= 64) return run_decode<64, KIND>(a, ep, s);
-    // Output tiles of 128 x 256 unless that leaves most SMs idle.
-    const int64_t tiles256 = ((a.m + 127) / 128) * ((a.n + 255) / 256);
-    if (tiles256 >= sm_count()) return run_tile<256, KIND, false>(a, ep, s);
+    // Output tile width: the persistent grid's makespan is
+    // ceil(tiles / SMs) tiles of time proportional to BN, so pick the BN with
+    // the smallest waves x BN (the wider tile on ties).
+    const int64_t sms = sm_count();
+    const int cand[3] = {256, 224, 128};
+    int best = 256;
+    int64_t best_cost = INT64_MAX;
+    for (int bn : cand) {
+        const int64_t tiles = ((a.m + 127) / 128) * ((a.n + bn - 1) / bn);
+        const int64_t cost = ((tiles + sms - 1) / sms) * bn;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    if (best == 256) return run_tile<256, KIND, false>(a, ep, s);
+    if (best == 224) return run_tile<224, KIND, false>(a, ep, s);
     return run_tile<128, KIND, false>(a, ep, s);
 }
 

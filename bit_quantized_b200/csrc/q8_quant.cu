@@ -38,17 +38,18 @@ template <> struct VecOf<__half> { static constexpr int N = 8; };
 template <> struct VecOf<__nv_bfloat16> { static constexpr int N = 8; };
 template <> struct VecOf<float> { static constexpr int N = 4; };
 
+// Read-only streaming load (not volatile, so the compiler can issue all of a
+// thread's loads before the first use and keep them in flight together).
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
     uint4 u;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
-                 : "l"(p));
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(u.x), "=r"(u.y), "=r"(u.z), "=r"(u.w)
+        : "l"(p));
     return u;
 }
 
 template <typename T>
-__device__ __forceinline__ void load_vec(const T* p, float (&v)[VecOf<T>::N]) {
-    const uint4 u = ld_stream16(p);
+__device__ __forceinline__ void unpack_vec(const uint4 u, float (&v)[VecOf<T>::N]) {
     if constexpr (VecOf<T>::N == 4) {
         v[0] = __uint_as_float(u.x); v[1] = __uint_as_float(u.y);
         v[2] = __uint_as_float(u.z); v[3] = __uint_as_float(u.w);
@@ -67,6 +68,11 @@ __device__ __forceinline__ void load_vec(const T* p, float (&v)[VecOf<T>::N]) {
             }
         }
     }
+}
+
+template <typename T>
+__device__ __forceinline__ void load_vec(const T* p, float (&v)[VecOf<T>::N]) {
+    unpack_vec<T>(ld_stream16(p), v);
 }
 
 struct RowStats {
@@ -133,7 +139,7 @@ __device__ __forceinline__ uint32_t e4m3_code(float v) {
 // One group of TPR threads per row; MAXV 16-byte vectors per thread stay in
 // registers between the two passes (longer rows are read twice).
 template <typename T, int OP, int TPR, int MAXV>
-__global__ void __launch_bounds__(kBlock) row_quant_kernel(RowQuantArgs a) {
+__global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
     constexpr int V = VecOf<T>::N;
     constexpr int RPB = kBlock / TPR;
     __shared__ float red[3 * (kBlock / 32)];
@@ -143,6 +149,9 @@ __global__ void __launch_bounds__(kBlock) row_quant_kernel(RowQuantArgs a) {
     const int t = threadIdx.x % TPR;
     const int64_t nvec = a.k / V;
     const bool cached = nvec <= static_cast<int64_t>(TPR) * MAXV;
+    // A GEMM launched next may start its prologue and weight loads now; it
+    // waits for this grid to finish before it reads the codes written here.
+    pdl_launch_dependents();
 
     for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * RPB; row0 < a.rows;
          row0 += static_cast<int64_t>(gridDim.x) * RPB) {
@@ -150,7 +159,7 @@ __global__ void __launch_bounds__(kBlock) row_quant_kernel(RowQuantArgs a) {
         const bool active = row < a.rows;
         const T* src = static_cast<const T*>(a.src) + (active ? row : 0) * a.ld;
 
-        float cache[MAXV][V];
+        uint4 raw[MAXV];  // the row's 16-byte vectors, kept packed between the passes
         RowStats st{0.f, FLT_MAX, -FLT_MAX};
         auto skipped = [&](int64_t col) -> bool { return a.skip != nullptr && a.skip[col] != 0; };
         auto accumulate = [&](const float (&v)[V], int64_t j) {
@@ -166,12 +175,19 @@ __global__ void __launch_bounds__(kBlock) row_quant_kernel(RowQuantArgs a) {
         };
         if (active) {
             if (cached) {
+                // All loads first, so they are in flight together.
+#pragma unroll
+                for (int i = 0; i < MAXV; ++i) {
+                    const int64_t j = t + static_cast<int64_t>(i) * TPR;
+                    if (j < nvec) raw[i] = ld_stream16(src + j * V);
+                }
 #pragma unroll
                 for (int i = 0; i < MAXV; ++i) {
                     const int64_t j = t + static_cast<int64_t>(i) * TPR;
                     if (j < nvec) {
-                        load_vec<T>(src + j * V, cache[i]);
-                        accumulate(cache[i], j);
+                        float v[V];
+                        unpack_vec<T>(raw[i], v);
+                        accumulate(v, j);
                     }
                 }
             } else {
@@ -235,7 +251,11 @@ __global__ void __launch_bounds__(kBlock) row_quant_kernel(RowQuantArgs a) {
 #pragma unroll
                 for (int i = 0; i < MAXV; ++i) {
                     const int64_t j = t + static_cast<int64_t>(i) * TPR;
-                    if (j < nvec) quantize(cache[i], j);
+                    if (j < nvec) {
+                        float v[V];
+                        unpack_vec<T>(raw[i], v);
+                        quantize(v, j);
+                    }
                 }
             } else {
                 for (int64_t j = t; j < nvec; j += TPR) {
@@ -293,9 +313,11 @@ cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
         row_quant_kernel<T, OP, TPR, 8><<<static_cast<unsigned>(blocks), kBlock, 0, s>>>(a);
         return cudaGetLastError();
     };
-    if (nvec <= 32 * 8) return go(std::integral_constant<int, 32>{});
-    if (nvec <= 64 * 8) return go(std::integral_constant<int, 64>{});
-    if (nvec <= 128 * 8) return go(std::integral_constant<int, 128>{});
+    // With few rows, spread each row over more threads so more loads are in flight.
+    const bool few_rows = a.rows < 4 * 148;
+    if (nvec <= 32 * 8 && !few_rows) return go(std::integral_constant<int, 32>{});
+    if (nvec <= 64 * 8 && !(few_rows && nvec > 64 * 2)) return go(std::integral_constant<int, 64>{});
+    if (nvec <= 128 * 8 && !(few_rows && nvec > 128 * 2)) return go(std::integral_constant<int, 128>{});
     return go(std::integral_constant<int, 256>{});
 }
 

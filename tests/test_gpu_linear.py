@@ -73,6 +73,7 @@ def test_prefill_ffn_up_sampled():
     (300, 640, 1024),       # tile kernel, several tiles, ragged M
     (384, 2304, 384),       # tile kernel BN=256 path (tiles >= SMs)
     (130, 48, 32),          # K = 32: one K block mostly out of bounds; N = 48
+    (512, 8288, 256),       # tile kernel BN=224 path (37 x 224-wide tiles, ragged N)
 ])
 @pytest.mark.parametrize("scheme,codes", [("asym", "s8"), ("asym", "u8"), ("sym", "s8")])
 def test_int8_shapes(m, n, k, scheme, codes):
