@@ -33,10 +33,12 @@ Q8_ERR_UNSUPPORTED_ARCH, Q8_ERR_LAUNCH, Q8_ERR_DEVICE_TIMEOUT, Q8_ERR_WORKSPACE,
 Q8_S8, Q8_U8, Q8_E4M3, Q8_F16, Q8_BF16, Q8_F32, Q8_S32 = range(7)
 Q8_ASYM_INT8, Q8_SYM_INT8, Q8_FP8_E4M3 = range(3)
 Q8_OP_LINEAR_W8A8, Q8_OP_LINEAR_INT8_MIXED = 0, 1
+Q8_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 EXPORTED = [
     "q8_quantize_weight", "q8_dequantize_weight", "q8_quantize_act", "q8_outlier_quantize_act",
-    "q8_linear_w8a8", "q8_linear_int8_mixed", "q8_workspace_size", "q8_status_string",
+    "q8_linear_w8a8", "q8_linear_int8_mixed", "q8_linear_int8_mixed_noalloc",
+    "q8_workspace_size", "q8_status_string",
     "q8_get_device_status", "q8_clear_device_status", "q8_device_check", "q8_version",
 ]
 
@@ -64,6 +66,8 @@ _SIG = {
                         _sz, _vp], _int),
     "q8_linear_int8_mixed": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeight), _vp, _f, _vp,
                               _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
+    "q8_linear_int8_mixed_noalloc": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeight), _vp,
+                                      _f, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp], _int),
     "q8_workspace_size": ([_int, _i64, _i64, _i64], _sz),
     "q8_status_string": ([_int], ctypes.c_char_p),
     "q8_get_device_status": ([_vp, _vp], _int),

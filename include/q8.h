@@ -250,6 +250,38 @@ q8_status q8_linear_int8_mixed(const void *X, q8_dtype x_dtype, int64_t m, int64
                                int32_t *acc_debug, float *y16_debug, void *workspace,
                                size_t ws_bytes, q8_stream_t stream);
 
+/*
+ * q8_linear_int8_mixed without a caller workspace, for callers that cannot
+ * allocate device memory: an engine that plans all of its device memory up
+ * front and forbids allocation while serving, a plain C caller with no device
+ * allocator, or code running where cudaMalloc may not be called.  (The pages
+ * have no counterpart: this is an interface convenience of this library.)
+ *
+ * Same arguments and results as q8_linear_int8_mixed, minus workspace and
+ * ws_bytes.  The scratch is one static device array inside the library, of
+ * Q8_NOALLOC_SCRATCH_BYTES (64 MiB); every GPU that loads the library's module
+ * holds it until the process exits.  This call allocates nothing and calls no
+ * allocating routine.
+ *   Limit     q8_workspace_size(Q8_OP_LINEAR_INT8_MIXED, m, w->n, k) must not
+ *             exceed Q8_NOALLOC_SCRATCH_BYTES (e.g. m <= 512 at n = k = 4096);
+ *             larger sizes return Q8_ERR_SHAPE before anything is launched.
+ *   Set-up    the first call on each device looks up the array's device
+ *             address (cudaGetSymbolAddress, with that device current) and
+ *             caches it; make that first call before any stream capture.
+ *   Sharing   every call on a device uses the same scratch, which keeps the
+ *             last call's contents (nothing in it needs to start at zero).
+ *             Calls whose executions overlap on the GPU (other streams, other
+ *             threads) race on it: serialize them.
+ */
+#define Q8_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+q8_status q8_linear_int8_mixed_noalloc(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
+                                       int64_t ldx, const q8_weight *w, const void *W16,
+                                       float threshold, const float *bias, void *Y, int64_t ldy,
+                                       uint8_t *outlier_mask, int32_t *outlier_count,
+                                       int32_t *acc_debug, float *y16_debug,
+                                       q8_stream_t stream);
+
 enum { Q8_OP_LINEAR_W8A8 = 0, Q8_OP_LINEAR_INT8_MIXED = 1 };
 
 /* Bytes of device workspace an operation needs for these sizes (host function,
