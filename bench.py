@@ -2,20 +2,22 @@
 """Benchmark of the 8-bit quantized linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl q8|reference]
-                    [--workload NAME] [--no-extras]
+                    [--workload NAME] [--no-extras] [--no-cpu-baseline]
 
 A step is one forward of the quantized linear layer on one batch of synthetic
 input: dynamic per-token activation quantization followed by the W8A8 GEMM
 with its dequant epilogue (weights are quantized once, offline, before the
 timed region, as the pages do on load).  The default workload is the
 q_proj-shaped decode layer: 16 tokens x 4096 -> 4096, bf16 in, asymmetric
-uint8 weights, INT32 accumulation, bf16 out.
+uint8 weights, INT32 accumulation, bf16 out; --workload picks another of the
+seeded workloads in workloads.py (prefill FFN-up INT8, FP8 rowwise, LLM.int8).
 
 Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs,
 bracketed by a barrier and a device synchronize, timed with CUDA events on the
-launching stream, max over ranks.  Steps rotate over 16 independent weight
-sets (268 MB of codes, more than the 126 MB L2), so every step reads its
-weights from HBM.  Prints one JSON line on rank 0.
+launching stream, max over ranks.  Steps rotate over independent layers
+whose working set is more than twice the 126 MB L2 (16 layers, 268 MB of
+weight codes, for the decode layer), so every step reads its weights from
+HBM.  Prints one JSON line on rank 0.
 
 --impl reference times the CPU oracle (oracle/) on the host cores instead,
 each step a bounded sample of the same workload.
@@ -42,7 +44,6 @@ import workloads  # noqa: E402
 
 METRIC = "W8A8 linear TOPS & % of B200 INT8/FP8 tensor peak; act-quant GB/s vs HBM"
 UNIT = "TOPS"
-ROTATE = 16           # independent layers cycled through by the timed steps
 NOMINAL_INT8_OVER_BF16 = 2.0   # dense INT8/FP8 4.5 P vs bf16 2.25 P per GPU
 
 
@@ -60,7 +61,9 @@ def peaks():
 
 # ---------------------------------------------------------------- distributed
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """One process per GPU: reads RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* from
+    the environment (torchrun) and joins the process group (NCCL on GPUs)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -68,7 +71,8 @@ def dist_setup(n_gpus: int):
         import datetime
         import torch.distributed as dist
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend is None:
+            backend = "nccl" if torch.cuda.is_available() else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local)
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
@@ -81,6 +85,12 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def aggregate_tops(steps: int, world: int, ops_per_step: float, ms_max: float) -> float:
+    """Whole-job throughput: the operations of every rank's K steps over the
+    slowest rank's time (weak scaling: per-GPU work fixed as N grows)."""
+    return steps * world * ops_per_step / (ms_max * 1e-3) / 1e12
 
 
 def max_over_ranks(value: float, world: int) -> float:
@@ -154,36 +164,103 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-# ---------------------------------------------------------------- inputs
+# ---------------------------------------------------------------- workloads
 
-def decode_layers(q8, dev, rotate: int, seed0: int):
-    """Rotating decode layers drawn with the decode recipe on the device:
-    W ~ N(0, 0.02) with 1% of entries redrawn from N(0, 0.2), X ~ N(0, 1)."""
-    w = workloads.WORKLOADS["decode_q_proj"]
-    g = torch.Generator(device=dev)
+# Default timed steps per workload (about a second or two of device time each).
+DEFAULT_STEPS = {"decode_q_proj": 100000, "tiny_mixed": 50000, "mixed_512": 20000,
+                 "prefill_ffn_up": 4000, "fp8_rowwise": 2000}
+DEFAULT_E2E_STEPS = {"decode_q_proj": 20000, "tiny_mixed": 20000, "mixed_512": 2000,
+                     "prefill_ffn_up": 100, "fp8_rowwise": 50}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def step_hbm_bytes(w) -> int:
+    """Bytes one step must move: weight codes, bf16/fp16 input, activation codes, bf16 output."""
+    return w.n * w.k + 2 * w.m * w.k + w.m * w.k + 2 * w.m * w.n
+
+
+def rotation(w) -> int:
+    """Independent layers cycled through so the working set exceeds twice the L2."""
+    r = -(-2 * L2_BYTES // step_hbm_bytes(w))
+    return int(min(16, max(2, r)))
+
+
+def make_layers(q8, dev, name: str, rotate: int, seed0: int):
+    """`rotate` independent layers of the workload, drawn with its seeded recipe
+    (workloads.make_inputs, one seed per layer), weights quantized once."""
+    w = workloads.WORKLOADS[name]
     layers = []
     for i in range(rotate):
-        g.manual_seed(seed0 + i)
-        X = torch.randn(w.m, w.k, generator=g, device=dev).to(torch.bfloat16)
-        W = torch.randn(w.n, w.k, generator=g, device=dev) * 0.02
-        heavy = torch.rand(w.n, w.k, generator=g, device=dev) < 0.01
-        W = torch.where(heavy, torch.randn(w.n, w.k, generator=g, device=dev) * 0.2, W)
-        W = W.to(torch.bfloat16)
-        qw = q8.q8_quantize_weight(W, "asym", "u8")
-        del W
-        qa = q8.QAct(torch.empty((w.m, w.k), dtype=torch.int8, device=dev),
-                     torch.empty(w.m, dtype=torch.float32, device=dev),
-                     torch.empty(w.m, dtype=torch.int32, device=dev), q8.Q8_S8)
-        Y = torch.empty((w.m, w.n), dtype=torch.bfloat16, device=dev)
-        layers.append({"X": X, "qw": qw, "qa": qa, "Y": Y})
+        X, W, _ = workloads.make_inputs(name, seed=seed0 + i)
+        X, Wd = X.to(dev), W.to(dev)
+        qw = q8.q8_quantize_weight(Wd, w.weight_scheme, w.weight_codes)
+        del Wd
+        L = {"X": X, "qw": qw, "Y": torch.empty((w.m, w.n), dtype=torch.bfloat16, device=dev)}
+        if w.kind == "w8a8_int8":
+            L["qa"] = q8.QAct(torch.empty((w.m, w.k), dtype=torch.int8, device=dev),
+                              torch.empty(w.m, dtype=torch.float32, device=dev),
+                              torch.empty(w.m, dtype=torch.int32, device=dev), q8.Q8_S8)
+        elif w.kind == "w8a8_fp8":
+            L["qa"] = q8.QAct(torch.empty((w.m, w.k), dtype=torch.float8_e4m3fn, device=dev),
+                              torch.empty(w.m, dtype=torch.float32, device=dev), None, q8.Q8_E4M3)
+        else:
+            L["ws"] = torch.empty(q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, w.m, w.n, w.k),
+                                  dtype=torch.uint8, device=dev)
+        layers.append(L)
     torch.cuda.synchronize()
     return layers
 
 
-def decode_gemm_bytes(w):
-    """Algorithmic HBM bytes of one decode GEMM launch: weight codes, activation
-    codes, bf16 output, per-channel scale/zero point, per-token scale/row sum."""
-    return w.n * w.k + w.m * w.k + 2 * w.m * w.n + 8 * w.n + 8 * w.m
+def step_functions(q8, w):
+    """(step, dominant kernel alone, kernel launches per step) for a workload."""
+    if w.kind == "int8_mixed":
+        def step(L, X=None):
+            q8.q8_linear_int8_mixed(L["X"] if X is None else X, L["qw"], w.threshold,
+                                    out=L["Y"], workspace=L["ws"])
+        return step, step, 5
+    scheme = "int8" if w.kind == "w8a8_int8" else "fp8"
+
+    def step(L, X=None):
+        q8.q8_quantize_act(L["X"] if X is None else X, scheme, clip_ub=w.clip_ub, out=L["qa"])
+        q8.q8_linear_w8a8(L["qa"], L["qw"], out=L["Y"])
+
+    def gemm(L, X=None):
+        q8.q8_linear_w8a8(L["qa"], L["qw"], out=L["Y"])
+    return step, gemm, 2
+
+
+def dominant_kernel(w, gemm_ms: float, pk: dict):
+    """Roofline entry of the step's dominant kernel (the GEMM)."""
+    ops = 2.0 * w.m * w.n * w.k
+    algo_bytes = w.n * w.k + w.m * w.k + 2 * w.m * w.n + 8 * w.n + 8 * w.m
+    t = gemm_ms * 1e-3
+    if w.name == "decode_q_proj" or w.m <= 64:
+        achieved = algo_bytes / t / 1e9
+        return {"bound": "hbm", "kernel": "gemm_decode_kernel (split-K cluster)",
+                "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "algorithmic_bytes": algo_bytes,
+                "peak_source": pk["source"] + " hbm_gbs (MEASURED_PEAKS.json, copy)"}
+    peak = pk["bf16_tflops_sustained"] * NOMINAL_INT8_OVER_BF16
+    achieved = ops / t / 1e12
+    return {"bound": "tensor", "kernel": "gemm_tile_kernel" + (" (LLM.int8)" if w.kind == "int8_mixed" else ""),
+            "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "algorithmic_ops": ops,
+            "peak_source": f"{pk['source']} bf16 sustained {pk['bf16_tflops_sustained']} x 2 "
+                           "(nominal dense INT8/FP8 : bf16 = 4.5 : 2.25); kernel timed in a long loop"}
+
+
+def describe(w):
+    if w.kind == "w8a8_fp8":
+        return {"x_dtype": "bf16", "weight": "per-channel FP8 e4m3 + fp32 scale",
+                "activation": f"per-token FP8 e4m3, clip {w.clip_ub}", "accumulate": "fp32",
+                "out": "bf16"}
+    wt = {"asym": "per-channel asymmetric " + ("uint8" if w.weight_codes == "u8" else "int8")
+          + " + fp32 S/Z", "sym": "per-channel symmetric int8 + fp32 S"}[w.weight_scheme]
+    d = {"x_dtype": "fp16" if w.x_dtype == torch.float16 else "bf16", "weight": wt,
+         "activation": "per-token symmetric int8", "accumulate": "int32", "out": "bf16"}
+    if w.kind == "int8_mixed":
+        d["outliers"] = f"LLM.int8 threshold {w.threshold}, fp16 outlier GEMM merged"
+    return d
 
 
 # ---------------------------------------------------------------- q8 arm
@@ -191,48 +268,41 @@ def decode_gemm_bytes(w):
 def run_q8(args, world, rank, local):
     from bit_quantized_b200 import q8
     dev = torch.device("cuda", local)
-    wl = workloads.WORKLOADS["decode_q_proj"]
+    wl = workloads.WORKLOADS[args.workload]
     pk = peaks()
     ops_per_step = 2.0 * wl.m * wl.n * wl.k
-    layers = decode_layers(q8, dev, ROTATE, seed0=1000 * (rank + 1))
-
-    def step(i):
-        L = layers[i % ROTATE]
-        q8.q8_quantize_act(L["X"], "int8", out=L["qa"])
-        q8.q8_linear_w8a8(L["qa"], L["qw"], out=L["Y"])
-
-    def gemm_only(i):
-        L = layers[i % ROTATE]
-        q8.q8_linear_w8a8(L["qa"], L["qw"], out=L["Y"])
+    R = rotation(wl)
+    layers = make_layers(q8, dev, args.workload, R, seed0=1000 * rank)
+    step_fn, kernel_fn, launches = step_functions(q8, wl)
 
     # warm-up (eager, through the public API)
     for i in range(args.warmup):
-        step(i)
+        step_fn(layers[i % R])
     torch.cuda.synchronize()
 
-    # One CUDA graph per rotation of the 16 layers (no event nodes inside: an
+    # One CUDA graph per rotation of the R layers (no event nodes inside: an
     # event record node costs several microseconds, more than a decode kernel).
     def make_graphs(fn):
         s = torch.cuda.Stream(device=dev)
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            for i in range(ROTATE):
-                fn(i)
+            for i in range(R):
+                fn(layers[i])
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         out = {}
-        for n_steps in sorted({ROTATE, args.steps % ROTATE} - {0}):
+        for n_steps in sorted({R, args.steps % R} - {0}):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 for i in range(n_steps):
-                    fn(i)
+                    fn(layers[i])
             out[n_steps] = g
         return out
 
     def timed(gmap, sampler=None):
-        full, rem = divmod(args.steps, ROTATE)
-        for _ in range(max(1, args.warmup // ROTATE)):
-            gmap[ROTATE].replay()
+        full, rem = divmod(args.steps, R)
+        for _ in range(max(1, args.warmup // R)):
+            gmap[R].replay()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize()
@@ -241,7 +311,7 @@ def run_q8(args, world, rank, local):
             time.sleep(0.25)
         t0.record()
         for _ in range(full):
-            gmap[ROTATE].replay()
+            gmap[R].replay()
         if rem:
             gmap[rem].replay()
         t1.record()
@@ -250,47 +320,44 @@ def run_q8(args, world, rank, local):
         barrier(world)
         return max_over_ranks(t0.elapsed_time(t1), world), clk
 
-    step_graphs = make_graphs(step)
-    sampler = ClockSampler(local)
-    ms_max, clocks = timed(step_graphs, sampler)
-    value = args.steps * world * ops_per_step / (ms_max * 1e-3) / 1e12
+    step_graphs = make_graphs(step_fn)
+    ms_max, clocks = timed(step_graphs, ClockSampler(local))
+    value = aggregate_tops(args.steps, world, ops_per_step, ms_max)
+    del step_graphs
     # The dominant kernel's average launch duration: the same K launches of the
-    # GEMM alone, replayed the same way right after, CUDA events on this stream.
-    gemm_graphs = make_graphs(gemm_only)
-    gemm_ms, _ = timed(gemm_graphs)
-    gemm_avg_ms = gemm_ms / args.steps
-    del step_graphs, gemm_graphs
+    # GEMM alone (for LLM.int8, the whole call), replayed the same way right
+    # after the timed steps, CUDA events on this stream.
+    kernel_graphs = make_graphs(kernel_fn)
+    kernel_ms, _ = timed(kernel_graphs)
+    kernel_avg_ms = kernel_ms / args.steps
+    del kernel_graphs
 
-    # e2e: pinned host input -> C ABI calls -> pinned host output, every step
-    e2e = run_e2e(q8, layers, args, world, ops_per_step)
-
-    algo_bytes = decode_gemm_bytes(wl)
-    achieved = algo_bytes / (gemm_avg_ms * 1e-3) / 1e9
-    traffic = load_profile_traffic("decode_gemm")
+    e2e = run_e2e(q8, layers, R, step_fn, args, world, ops_per_step, wl)
+    roof = dominant_kernel(wl, kernel_avg_ms, pk)
+    roof["traffic"] = load_profile_traffic(args.workload)
+    roof["avg_launch_us"] = round(kernel_avg_ms * 1e3, 3)
+    roof["duration_from"] = ("K launches of the kernel replayed alone right after the timed steps"
+                             if launches == 2 else "K whole calls replayed right after the timed steps")
+    ws_bytes = R * step_hbm_bytes(wl)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8",
-        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights with 1% N(0,0.2) tail)",
-        "config": {"workload": "decode_q_proj", "m_tokens": wl.m, "n_out": wl.n, "k_in": wl.k,
-                   "x_dtype": "bf16", "weight": "per-channel asymmetric uint8 + fp32 S/Z",
-                   "activation": "per-token symmetric int8", "accumulate": "int32",
-                   "out": "bf16", "parallelism": f"dp{world} (independent batches per GPU)",
-                   "l2": f"steps rotate over {ROTATE} weight sets "
-                         f"({ROTATE * wl.n * wl.k / 1e6:.0f} MB of codes > 126 MB L2)",
-                   "timing": "CUDA graphs of 16 steps, CUDA events, max over ranks"},
-        "roofline": {"bound": "hbm", "kernel": "gemm_decode_kernel<16, s8xu8>",
-                     "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
-                     "algorithmic_bytes": algo_bytes, "avg_launch_us": round(gemm_avg_ms * 1e3, 3),
-                     "duration_from": "K GEMM launches replayed alone right after the timed steps",
-                     "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if wl.kind == "w8a8_fp8" else "s8",
+        "data": "synthetic (seeded recipe of workloads.py, one seed per rotated layer)",
+        "config": {"workload": args.workload, "m_tokens": wl.m, "n_out": wl.n, "k_in": wl.k,
+                   **describe(wl), "parallelism": f"dp{world} (independent batches per GPU)",
+                   "l2": (f"steps rotate over {R} layers ({ws_bytes / 1e6:.0f} MB > 126 MB L2)"
+                          if ws_bytes > L2_BYTES else
+                          f"{R} layers ({ws_bytes / 1e6:.1f} MB) stay L2-resident"),
+                   "timing": f"CUDA graphs of {R} steps, CUDA events, max over ranks"},
+        "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": clocks,
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(args.workload, seconds=args.cpu_seconds)
     if world == 1 and rank == 0 and not args.no_extras:
         line["per_config"] = extras(q8, dev, pk)
     if world > 1:
@@ -300,18 +367,22 @@ def run_q8(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def run_e2e(q8, layers, args, world, ops_per_step):
-    w = workloads.WORKLOADS["decode_q_proj"]
+def run_e2e(q8, layers, R, step_fn, args, world, ops_per_step, w):
+    """Same step through the public API with the input copied from pinned host
+    memory and the bf16 output copied back to pinned host memory every step."""
     steps = min(args.steps, args.e2e_steps)
     hx = [L["X"].cpu().pin_memory() for L in layers]
     hy = [torch.empty((w.m, w.n), dtype=torch.bfloat16).pin_memory() for _ in layers]
     dx = torch.empty_like(layers[0]["X"])
+
+    def one(i):
+        L = layers[i % R]
+        dx.copy_(hx[i % R], non_blocking=True)
+        step_fn(L, dx)
+        hy[i % R].copy_(L["Y"], non_blocking=True)
+
     for i in range(min(args.warmup, 8)):
-        L = layers[i % ROTATE]
-        dx.copy_(hx[i % ROTATE], non_blocking=True)
-        q8.q8_quantize_act(dx, "int8", out=L["qa"])
-        q8.q8_linear_w8a8(L["qa"], L["qw"], out=L["Y"])
-        hy[i % ROTATE].copy_(L["Y"], non_blocking=True)
+        one(i)
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -319,11 +390,7 @@ def run_e2e(q8, layers, args, world, ops_per_step):
     wall0 = time.perf_counter()
     t0.record()
     for i in range(steps):
-        L = layers[i % ROTATE]
-        dx.copy_(hx[i % ROTATE], non_blocking=True)
-        q8.q8_quantize_act(dx, "int8", out=L["qa"])
-        q8.q8_linear_w8a8(L["qa"], L["qw"], out=L["Y"])
-        hy[i % ROTATE].copy_(L["Y"], non_blocking=True)
+        one(i)
     t1.record()
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
@@ -333,7 +400,7 @@ def run_e2e(q8, layers, args, world, ops_per_step):
             "h2d_bytes_per_step": int(hx[0].numel() * hx[0].element_size()),
             "d2h_bytes_per_step": int(hy[0].numel() * hy[0].element_size()),
             "steps": steps, "ms_per_step": ms / steps, "wall_s": round(wall, 4),
-            "path": "pinned host X -> q8_quantize_act -> q8_linear_w8a8 -> pinned host Y, eager"}
+            "path": "pinned host X -> quantize + linear through the q8 C ABI -> pinned host Y, eager"}
 
 
 def load_profile_traffic(kernel_tag: str):
@@ -432,53 +499,73 @@ def extras(q8, dev, pk):
 
 # ---------------------------------------------------------------- CPU oracle
 
-def oracle_decode_inputs():
+def oracle_inputs(name: str):
     from oracle import oracle as O
-    X, W, _ = workloads.make_inputs("decode_q_proj")
-    x32 = O.widen16(workloads.bits16(X), "bf16")
-    w32 = O.widen16(workloads.bits16(W), "bf16")
-    wq, Sw, Zw = O.quant_weight(w32, "asym", "u8")
-    return O, x32, wq, Sw, Zw
+    w = workloads.WORKLOADS[name]
+    X, W, _ = workloads.make_inputs(name)
+    fmt = "f16" if w.x_dtype == torch.float16 else "bf16"
+    x32 = O.widen16(workloads.bits16(X), fmt)
+    w32 = O.widen16(workloads.bits16(W), fmt)
+    q = O.quant_weight(w32, w.weight_scheme, w.weight_codes)
+    return O, w, x32, q
 
 
-def cpu_baseline(seconds: float = 10.0):
-    """The oracle, as it stands, on full decode steps for about `seconds`."""
-    O, x32, wq, Sw, Zw = oracle_decode_inputs()
-    w = workloads.WORKLOADS["decode_q_proj"]
-    ops = 2.0 * w.m * w.n * w.k
+def oracle_step(O, w, x32, q, rows, cols):
+    """One oracle forward of the workload on the given token rows and output columns."""
+    wq, Sw, Zw = q
+    xs = x32[rows]
+    r = np.arange(len(rows))
+    if w.kind == "w8a8_int8":
+        xq, Sx, rs = O.quant_act_int8(xs)
+        O.linear_w8a8_int8(xq, Sx, rs, wq, Sw, Zw, None, r, cols)
+    elif w.kind == "w8a8_fp8":
+        xq, Sx = O.quant_act_fp8(xs, w.clip_ub)
+        O.linear_w8a8_fp8(xq, Sx, wq, Sw, None, r, cols)
+    else:
+        O.linear_int8_mixed(x32, wq, Sw, Zw, w.threshold, rows=rows, cols=cols)
+
+
+def cpu_baseline(name: str, seconds: float = 10.0):
+    """The oracle, as it stands, on the workload's step for about `seconds`:
+    full steps when one takes under a second, else steps on a row sample."""
+    O, w, x32, q = oracle_inputs(name)
+    cols = np.arange(w.n)
+    t0 = time.perf_counter()
+    oracle_step(O, w, x32, q, np.arange(1), cols)
+    per_row = time.perf_counter() - t0
+    rows_n = int(max(1, min(w.m, 1.0 / max(per_row, 1e-9))))
+    rows = np.arange(rows_n)
+    ops = 2.0 * rows_n * w.n * w.k
     done, t0 = 0, time.perf_counter()
     while True:
-        xq, Sx, rs = O.quant_act_int8(x32)
-        O.linear_w8a8_int8(xq, Sx, rs, wq, Sw, Zw)
+        oracle_step(O, w, x32, q, rows, cols)
         done += 1
         if time.perf_counter() - t0 >= seconds:
             break
     dt = time.perf_counter() - t0
+    what = "full steps" if rows_n == w.m else f"steps on {rows_n} of {w.m} token rows"
     return {"value": round(done * ops / dt / 1e12, 6), "unit": UNIT, "cores": O.threads(),
             "kind": "oracle",
-            "sample": f"{done} full decode steps (16x4096 act quant + 16x4096x4096 int8 GEMM "
-                      f"+ epilogue) in {dt:.1f} s; weight quantization excluded as on the GPU"}
+            "sample": f"{done} {what} of {name} ({w.m}x{w.n}x{w.k}: activation quantization + "
+                      f"GEMM + epilogue) in {dt:.1f} s; weight quantization excluded as on the GPU"}
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    O, x32, wq, Sw, Zw = oracle_decode_inputs()
-    w = workloads.WORKLOADS["decode_q_proj"]
-    # Size each step's sample so that warm-up + K steps take about a minute.
+    O, w, x32, q = oracle_inputs(args.workload)
+    cols_all = np.arange(w.n)
+    # Size each step's sample (one token row x some output columns) so that
+    # warm-up + K steps take about a minute.
     t0 = time.perf_counter()
-    xq, Sx, rs = O.quant_act_int8(x32[:1])
-    O.linear_w8a8_int8(xq, Sx, rs, wq, Sw, Zw, None, np.array([0]), np.arange(w.n))
+    oracle_step(O, w, x32, q, np.arange(1), cols_all)
     per_col = (time.perf_counter() - t0) / w.n
     budget = 60.0 / max(1, args.steps + args.warmup)
-    cols = int(max(16, min(w.n, budget / max(per_col, 1e-9))))
-    colsel = np.arange(cols)
-    rows = np.array([0])
+    ncols = int(max(16, min(w.n, budget / max(per_col, 1e-9))))
+    cols = cols_all[:ncols]
 
     def step(i):
-        r = np.array([i % w.m])
-        xq, Sx, rs = O.quant_act_int8(x32[r])
-        O.linear_w8a8_int8(xq, Sx, rs, wq, Sw, Zw, None, np.array([0]), colsel)
+        oracle_step(O, w, x32, q, np.array([i % w.m]), cols)
 
     for i in range(args.warmup):
         step(i)
@@ -486,15 +573,15 @@ def run_reference(args, world, rank):
     for i in range(args.steps):
         step(i)
     dt = time.perf_counter() - t0
-    ops = 2.0 * rows.size * cols * w.k * args.steps
-    value = ops / dt / 1e12
-    sample = (f"each step: 1 token row of the 16x4096 decode input (act quant) x {cols} of 4096 "
-              "output columns (int8 GEMM + epilogue)")
+    value = 2.0 * ncols * w.k * args.steps / dt / 1e12
+    sample = (f"each step: 1 token row of the {w.m}x{w.k} {args.workload} input (activation "
+              f"quantization) x {ncols} of {w.n} output columns (GEMM + epilogue)")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "s8", "data": "synthetic",
-            "config": {"workload": "decode_q_proj", "m_tokens": w.m, "n_out": w.n, "k_in": w.k},
+            "vs_baseline": None, "dtype": "e4m3" if w.kind == "w8a8_fp8" else "s8",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "m_tokens": w.m, "n_out": w.n, "k_in": w.k},
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": O.threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -505,14 +592,19 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=32)
     ap.add_argument("--impl", choices=["q8", "reference"], default="q8")
-    ap.add_argument("--e2e-steps", type=int, default=20000)
+    ap.add_argument("--workload", choices=workloads.ORDER, default="decode_q_proj")
+    ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = DEFAULT_STEPS[args.workload]
+    if args.e2e_steps is None:
+        args.e2e_steps = DEFAULT_E2E_STEPS[args.workload]
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":
