@@ -149,9 +149,13 @@ __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
     const int t = threadIdx.x % TPR;
     const int64_t nvec = a.k / V;
     const bool cached = nvec <= static_cast<int64_t>(TPR) * MAXV;
-    // A GEMM launched next may start its prologue and weight loads now; it
-    // waits for this grid to finish before it reads the codes written here.
-    pdl_launch_dependents();
+    // Activation quantizers let a GEMM launched next start its prologue and
+    // weight loads now (it waits for this grid before reading the codes written
+    // here).  This grid was launched without programmatic dependency, so every
+    // earlier kernel, the one that wrote the weights included, has completed.
+    // Weight quantizers do not trigger: a GEMM right after one must not load
+    // the weight before it is fully written.
+    if constexpr (OP == kOpActInt8 || OP == kOpActFp8) pdl_launch_dependents();
 
     for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * RPB; row0 < a.rows;
          row0 += static_cast<int64_t>(gridDim.x) * RPB) {
