@@ -277,6 +277,51 @@ q8_status q8_linear_w8a8(const q8_act* x, const q8_weight* w, const float* bias,
     return launch_linear(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+q8_status q8_linear_w8a8_dynamic(const void* X, q8_dtype x_dtype, int64_t m, int64_t k,
+                                 int64_t ldx, q8_scheme act_scheme, float clip_ub,
+                                 const q8_weight* w, const float* bias, void* Y, int64_t ldy,
+                                 void* act_codes, float* act_scale, int32_t* act_rowsum,
+                                 void* acc_debug, q8_stream_t stream) {
+    q8_status st = check_weight(w);
+    if (st != Q8_OK) return st;
+    if (m < 0 || m > kMaxDim || k != w->k || ldx < k || ldy < w->n) return Q8_ERR_SHAPE;
+    if (!float_input(x_dtype)) return Q8_ERR_DTYPE;
+    const bool fp8 = act_scheme == Q8_FP8_E4M3;
+    if (act_scheme != Q8_SYM_INT8 && !fp8) return Q8_ERR_SCHEME;
+    if (fp8 != (w->code_dtype == Q8_E4M3)) return Q8_ERR_DTYPE;
+    if (!fp8 && w->k > kMaxKInt8) return Q8_ERR_SHAPE;
+    if (m == 0 || w->n == 0) return Q8_OK;   // empty call
+    if (!X || !Y || !act_codes || !act_scale || (!fp8 && !act_rowsum)) return Q8_ERR_NULL;
+    if (!aligned16(X) || !ld_ok(ldx, k, x_dtype) || !aligned16(Y) || ldy % 8 != 0 ||
+        !aligned16(act_codes) || !aligned16(act_scale) || (bias && !aligned16(bias)) ||
+        (acc_debug && !aligned16(acc_debug)))
+        return Q8_ERR_ALIGN;
+    st = check_device();
+    if (st != Q8_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    LinearArgs a = {};
+    a.m = m; a.n = w->n; a.k = k;
+    a.a_codes = act_codes; a.lda = k;
+    a.b_codes = w->codes; a.ldb = w->ld;
+    a.kind = fp8 ? 2 : (w->code_dtype == Q8_U8 ? 1 : 0);
+    a.sx = act_scale; a.rowsum = fp8 ? nullptr : act_rowsum;
+    a.sw = w->scale; a.zw = fp8 ? nullptr : w->zero_point;
+    a.bias = bias;
+    a.y = static_cast<__nv_bfloat16*>(Y); a.ldy = ldy;
+    a.acc_debug = acc_debug;
+    // The quantizer lets the GEMM start early (programmatic dependent launch):
+    // the GEMM's prologue and weight loads overlap the quantization.
+    RowQuantArgs r = {};
+    r.src = X; r.src_dtype = x_dtype; r.rows = m; r.k = k; r.ld = ldx;
+    r.op = fp8 ? kOpActFp8 : kOpActInt8;
+    r.clip_ub = clip_ub;
+    r.codes = act_codes; r.scale = act_scale;
+    r.rowsum = fp8 ? nullptr : act_rowsum;
+    st = launch_status(launch_row_quant(r, s));
+    if (st != Q8_OK) return st;
+    return launch_linear(a, s);
+}
+
 q8_status q8_linear_int8_mixed(const void* X, q8_dtype x_dtype, int64_t m, int64_t k, int64_t ldx,
                                const q8_weight* w, const void* W16, float threshold,
                                const float* bias, void* Y, int64_t ldy, uint8_t* outlier_mask,

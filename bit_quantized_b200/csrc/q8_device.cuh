@@ -226,14 +226,6 @@ __device__ __forceinline__ void cluster_sync() {
                      : "memory");
 }
 
-// Second barrier of a cluster exchange: only orders completion of the remote
-// shared-memory reads, so the arrive is relaxed (no wait for global stores).
-__device__ __forceinline__ void cluster_sync_relaxed() {
-    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\t"
-                 "barrier.cluster.wait.aligned;" ::
-                     : "memory");
-}
-
 // Programmatic dependent launch: the next kernel in the stream may start its
 // prologue once every CTA of this grid has executed launch_dependents; it
 // calls wait before touching anything this grid writes.
@@ -255,14 +247,6 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t ran
 __device__ __forceinline__ void st_shared_cluster_u32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
-
-__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred = 0;

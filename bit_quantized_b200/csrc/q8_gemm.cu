@@ -590,6 +590,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     }
 }
 
+
 // ============================================================================
 // Host side
 // ============================================================================
@@ -722,6 +723,7 @@ q8_status run_decode(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     return Q8_OK;
 }
 
+
 template <int KIND>
 q8_status dispatch_kind(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     if (a.m <= 16) return run_decode<16, KIND>(a, ep, s);
@@ -748,6 +750,7 @@ q8_status dispatch_kind(const LinearArgs& a, const EpiParams& ep, cudaStream_t s
 }
 
 }  // namespace
+
 
 q8_status launch_linear(const LinearArgs& a, cudaStream_t s) {
     if (a.m == 0 || a.n == 0) return Q8_OK;

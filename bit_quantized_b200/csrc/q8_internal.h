@@ -72,4 +72,5 @@ struct LinearArgs {
 
 q8_status launch_linear(const LinearArgs& a, cudaStream_t s);
 
+
 }  // namespace q8

@@ -37,7 +37,8 @@ Q8_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 EXPORTED = [
     "q8_quantize_weight", "q8_dequantize_weight", "q8_quantize_act", "q8_outlier_quantize_act",
-    "q8_linear_w8a8", "q8_linear_int8_mixed", "q8_linear_int8_mixed_noalloc",
+    "q8_linear_w8a8", "q8_linear_w8a8_dynamic", "q8_linear_int8_mixed",
+    "q8_linear_int8_mixed_noalloc",
     "q8_workspace_size", "q8_status_string",
     "q8_get_device_status", "q8_clear_device_status", "q8_device_check", "q8_version",
 ]
@@ -64,6 +65,8 @@ _SIG = {
                                  _vp, _i64, _vp], _int),
     "q8_linear_w8a8": ([ctypes.POINTER(CAct), ctypes.POINTER(CWeight), _vp, _vp, _i64, _vp, _vp,
                         _sz, _vp], _int),
+    "q8_linear_w8a8_dynamic": ([_vp, _int, _i64, _i64, _i64, _int, _f, ctypes.POINTER(CWeight),
+                                _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp], _int),
     "q8_linear_int8_mixed": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeight), _vp, _f, _vp,
                               _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "q8_linear_int8_mixed_noalloc": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeight), _vp,
@@ -250,6 +253,34 @@ def q8_linear_w8a8(x: QAct, w: QWeight, bias: Optional[torch.Tensor] = None,
                                out.stride(0), _ptr(acc_debug), None, 0, _stream(stream)),
            "q8_linear_w8a8")
     return out
+
+
+def q8_linear_w8a8_dynamic(X: torch.Tensor, w: QWeight, scheme: str = "int8",
+                           clip_ub: float = 0.0, bias: Optional[torch.Tensor] = None,
+                           out: Optional[torch.Tensor] = None, act: Optional[QAct] = None,
+                           acc_debug: Optional[torch.Tensor] = None, stream=None):
+    """Activation quantization + W8A8 linear in one call; returns (Y, QAct)."""
+    _cuda(X, "X")
+    m, k = X.shape
+    n = w.codes.shape[0]
+    dev = X.device
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    if act is None:
+        if scheme == "int8":
+            act = QAct(torch.empty((m, k), dtype=torch.int8, device=dev),
+                       torch.empty(m, dtype=torch.float32, device=dev),
+                       torch.empty(m, dtype=torch.int32, device=dev), Q8_S8)
+        else:
+            act = QAct(torch.empty((m, k), dtype=torch.float8_e4m3fn, device=dev),
+                       torch.empty(m, dtype=torch.float32, device=dev), None, Q8_E4M3)
+    cw = w.c()
+    _check(_lib.q8_linear_w8a8_dynamic(
+        _ptr(X), _FLOAT_DT[X.dtype], m, k, X.stride(0),
+        Q8_SYM_INT8 if scheme == "int8" else Q8_FP8_E4M3, float(clip_ub), ctypes.byref(cw),
+        _ptr(bias), _ptr(out), out.stride(0), _ptr(act.codes), _ptr(act.scale),
+        _ptr(act.rowsum), _ptr(acc_debug), _stream(stream)), "q8_linear_w8a8_dynamic")
+    return out, act
 
 
 def q8_linear_int8_mixed(X: torch.Tensor, w: QWeight, threshold: float = 6.0,

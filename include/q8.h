@@ -228,6 +228,30 @@ q8_status q8_linear_w8a8(const q8_act *x, const q8_weight *w, const float *bias,
                          q8_stream_t stream);
 
 /*
+ * Dynamic per-token activation quantization and the W8A8 linear in one call:
+ * the same results, bit for bit, as q8_quantize_act(X, act_scheme, clip_ub)
+ * followed by q8_linear_w8a8 ([Xilyfe] dynamic quantization: the activation
+ * scale is computed from each call's input; [FBGEMM] 5.2-5.3: quantize the
+ * input per row, then the rowwise GEMM, on every forward).
+ *
+ *   X            device, m x k, Q8_F16 / Q8_BF16 / Q8_F32, row stride ldx.
+ *   act_scheme   Q8_SYM_INT8 with an INT8 weight (Q8_S8 / Q8_U8), or
+ *                Q8_FP8_E4M3 with an E4M3 weight; clip_ub as q8_quantize_act.
+ *   act_codes    device m x k output codes (row stride k), act_scale [m] and,
+ *   act_scale,   for INT8, act_rowsum [m]: the quantized activation, written as
+ *   act_rowsum   q8_quantize_act writes it (required).
+ *   acc_debug    as q8_linear_w8a8.
+ * Two launches: the quantizer lets the GEMM start early (programmatic
+ * dependent launch), so the GEMM's prologue and weight loads overlap the
+ * quantization.  The launch-overlap rule of q8_linear_w8a8 applies.
+ */
+q8_status q8_linear_w8a8_dynamic(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
+                                 int64_t ldx, q8_scheme act_scheme, float clip_ub,
+                                 const q8_weight *w, const float *bias, void *Y, int64_t ldy,
+                                 void *act_codes, float *act_scale, int32_t *act_rowsum,
+                                 void *acc_debug, q8_stream_t stream);
+
+/*
  * LLM.int8 mixed-decomposition linear ([LLM.int8] 核心思想; BitsAndBytesConfig
  * llm_int8_threshold, llm_int8_has_fp16_weight).  One call runs
  * q8_outlier_quantize_act on X, the INT8 GEMM of the regular stream, and the

@@ -242,3 +242,69 @@ def test_mixed_many_outliers():
 
 def test_device_status_clean():
     assert q8.q8_get_device_status() == 0
+
+
+# ------------------------------------------------------------------ one-call activation quant + linear
+
+def _dynamic_vs_two_step(X, W, scheme, codes, wscheme, ub=0.0, bias=None, what=""):
+    Xd, Wd = X.to(DEV), W.to(DEV)
+    qw = q8.q8_quantize_weight(Wd, wscheme, codes)
+    m, n = X.shape[0], W.shape[0]
+    b = None if bias is None else torch.from_numpy(bias).to(DEV)
+    acc_dt = torch.float32 if scheme == "fp8" else torch.int32
+    acc1 = torch.empty((m, n), dtype=acc_dt, device=DEV)
+    acc2 = torch.empty((m, n), dtype=acc_dt, device=DEV)
+    Y1, act = q8.q8_linear_w8a8_dynamic(Xd, qw, scheme, clip_ub=ub, bias=b, acc_debug=acc1)
+    qa = q8.q8_quantize_act(Xd, scheme, clip_ub=ub)
+    Y2 = q8.q8_linear_w8a8(qa, qw, bias=b, acc_debug=acc2)
+    torch.cuda.synchronize()
+    P.assert_equal(P.codes_u8(act.codes), P.codes_u8(qa.codes), what + " codes")
+    P.assert_equal(act.scale.cpu().numpy().view(np.uint32), qa.scale.cpu().numpy().view(np.uint32),
+                   what + " scale")
+    if scheme == "int8":
+        P.assert_equal(act.rowsum.cpu().numpy(), qa.rowsum.cpu().numpy(), what + " rowsum")
+        P.assert_equal(acc1.cpu().numpy(), acc2.cpu().numpy(), what + " acc")
+        P.assert_equal(P.bf16_bits(Y1), P.bf16_bits(Y2), what + " Y")
+    else:
+        # split-K partial sums are added in a different order than one TMEM accumulator
+        y2 = P.bf16_values(P.bf16_bits(Y2))
+        xq = P.codes_u8(qa.codes)
+        mag = np.abs(O.widen_e4m3(xq)).astype(np.float64) @ np.abs(O.widen_e4m3(P.codes_u8(qw.codes))).T
+        sx, sw = qa.scale.cpu().numpy().astype(np.float64), qw.scale.cpu().numpy().astype(np.float64)
+        extra = X.shape[1] * 2.0**-22 * mag * sx[:, None] * sw[None, :]
+        P.assert_bf16_within(P.bf16_bits(Y1), y2, extra, what)
+    return Y1, qw, act
+
+
+@pytest.mark.parametrize("m,n,k,dtype", [
+    (16, 4096, 4096, torch.bfloat16),   # decode workload shape
+    (1, 128, 256, torch.float16),
+    (17, 272, 160, torch.bfloat16),     # NT=32, ragged last K block
+    (33, 512, 1024, torch.float16),     # NT=64
+    (64, 384, 4096, torch.bfloat16),
+    (65, 256, 256, torch.bfloat16),     # tile kernel
+    (8, 256, 512, torch.float32),       # fp32 input
+])
+@pytest.mark.parametrize("codes,wscheme", [("u8", "asym"), ("s8", "sym")])
+def test_dynamic_int8_matches_two_step(m, n, k, dtype, codes, wscheme):
+    X = workloads.random_matrix(m, k, dtype, seed=m * 7 + k)
+    W = workloads.random_matrix(n, k, dtype, seed=n + 3 * k, std=0.02)
+    bias = np.linspace(-1, 1, n).astype(np.float32) if m % 2 else None
+    _dynamic_vs_two_step(X, W, "int8", codes, wscheme, bias=bias, what=f"dyn {m}x{n}x{k} {codes}")
+
+
+@pytest.mark.parametrize("m,n,k", [(16, 1024, 2048), (5, 256, 512), (40, 512, 1024)])
+def test_dynamic_fp8_matches_two_step(m, n, k):
+    X = workloads.random_matrix(m, k, torch.bfloat16, seed=m + k) * 3
+    X[0, 1] = 5000.0                         # beyond the upper bound
+    W = workloads.random_matrix(n, k, torch.bfloat16, seed=n + k, std=0.02)
+    _dynamic_vs_two_step(X, W, "fp8", "e4m3", "fp8", ub=1200.0, what=f"dyn fp8 {m}x{n}x{k}")
+
+
+def test_dynamic_decode_workload_against_oracle():
+    X, W, info, x32, w32 = P.workload("decode_q_proj")
+    Y, qw, act = _dynamic_vs_two_step(X, W, "int8", "u8", "asym", what="decode workload")
+    xq, Sx, rs = O.quant_act_int8(x32)
+    wq, Sw, Zw = O.quant_weight(w32, "asym", "u8")
+    _, _, Y_ref = O.linear_w8a8_int8(xq, Sx, rs, wq, Sw, Zw)
+    P.assert_equal(P.bf16_bits(Y), Y_ref, "decode workload Y vs oracle")
