@@ -209,7 +209,8 @@ static q8_status validate_outlier_act(const void* X, q8_dtype x_dtype, int64_t m
     if (m > 0 && (!X || !codes || !scale || !rowsum)) return Q8_ERR_NULL;
     if (x_outlier && (ldo < (k + 63) / 64 * 64)) return Q8_ERR_SHAPE;
     if (x_dtype != Q8_F16) return Q8_ERR_DTYPE;
-    if (!aligned16(X) || !aligned16(codes) || !ld_ok(ldx, k, x_dtype)) return Q8_ERR_ALIGN;
+    if (!aligned16(X) || !aligned16(codes) || !ld_ok(ldx, k, x_dtype) || !aligned16(mask))
+        return Q8_ERR_ALIGN;
     if (x_outlier && (!aligned16(x_outlier) || ldo % 8 != 0)) return Q8_ERR_ALIGN;
     return Q8_OK;
 }

@@ -156,6 +156,9 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
+    // The next kernel (typically the next layer's activation quantizer, which
+    // waits for this grid before touching memory) may launch now.
+    pdl_launch_dependents();
 
     int n16_kb = 0;
     if constexpr (MIXED) {
@@ -435,6 +438,9 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
+    // The next kernel (typically the next layer's activation quantizer, which
+    // waits for this grid before touching memory) may launch now.
+    pdl_launch_dependents();
 
     if (warp == 0) {
         if (elect_one()) {

@@ -32,6 +32,7 @@ namespace {
 
 constexpr float kEps = 1e-8f;
 constexpr int kBlock = 256;
+constexpr int kMaxVec = 16;   // 16-byte vectors a thread keeps in registers
 
 template <typename T> struct VecOf;
 template <> struct VecOf<__half> { static constexpr int N = 8; };
@@ -80,13 +81,16 @@ struct RowStats {
 };
 
 // Reduction of per-thread stats over the TPR threads that share a row.
-template <int TPR>
+template <int TPR, bool MINMAX>
 __device__ __forceinline__ RowStats group_reduce(RowStats s, float* red) {
 #pragma unroll
     for (int o = (TPR < 32 ? TPR : 32) / 2; o > 0; o >>= 1) {
-        s.amax = fmaxf(s.amax, __shfl_xor_sync(0xffffffffu, s.amax, o));
-        s.lo = fminf(s.lo, __shfl_xor_sync(0xffffffffu, s.lo, o));
-        s.hi = fmaxf(s.hi, __shfl_xor_sync(0xffffffffu, s.hi, o));
+        if constexpr (MINMAX) {
+            s.lo = fminf(s.lo, __shfl_xor_sync(0xffffffffu, s.lo, o));
+            s.hi = fmaxf(s.hi, __shfl_xor_sync(0xffffffffu, s.hi, o));
+        } else {
+            s.amax = fmaxf(s.amax, __shfl_xor_sync(0xffffffffu, s.amax, o));
+        }
     }
     if constexpr (TPR > 32) {
         constexpr int W = TPR / 32;
@@ -132,12 +136,164 @@ __device__ __forceinline__ float clampf(float v, float lo, float hi) {
     return fminf(fmaxf(v, lo), hi);
 }
 
-__device__ __forceinline__ uint32_t e4m3_code(float v) {
-    return static_cast<uint32_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+
+// Codes of one 16-byte vector (V elements) from the IEEE quotient fl32(x / S),
+// without a division per element.
+//
+// With R = RN(1/S) (one reciprocal per row) the product t = RN(x * R) has a
+// relative error below 2^-23 against x / S, and fl32(x / S) adds 2^-24, so
+// |t - fl32(x / S)| <= 1.5 * 2^-23 |t|.
+//   Integer codes: |t| <= 1024 (wider inputs are clamped; their codes saturate
+//   anyway).  Adding 1.5 * 2^23 rounds t to an integer half to even (the sum lies
+//   in [2^23, 2^24), where floats are integers, and the constant is even); the
+//   low byte of the sum is the code's two's-complement byte (the constant's low
+//   byte is 0), and d = t - rne(t) is exact.  An ulp of t is at most 2^-13, so
+//   when |d| < 0.499 no half-integer lies between t and fl32(x / S): both round
+//   to the same integer.
+//   E4M3 codes: rounding to E4M3 (half to even, saturating) is monotonic, and
+//   t (1 - 2^-20) and t (1 + 2^-20) bracket fl32(x / S); when both convert to
+//   the same code, so does fl32(x / S).  (Values too small for the bracket to
+//   widen round to zero either way.)
+// A vector with any element near a rounding boundary is redone with exact
+// divisions, out of line (it is rare).
+constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
-// One group of TPR threads per row; MAXV 16-byte vectors per thread stay in
-// registers between the two passes (longer rows are read twice).
+// Exact out-of-line paths; they take the packed input vector and return the
+// packed codes by value so the fast paths keep everything in registers.
+template <typename T>
+__device__ __noinline__ uint2 int_codes_exact(const uint4 u, float S, float Z, float lo_clamp,
+                                              float hi_clamp, float bias) {
+    constexpr int V = VecOf<T>::N;
+    float v[V];
+    unpack_vec<T>(u, v);
+    uint32_t words[2] = {0u, 0u};
+    for (int w = 0; w < V / 4; ++w) {
+        uint32_t b[4];
+        for (int e = 0; e < 4; ++e) {
+            float q = rintf(__fdiv_rn(v[4 * w + e], S));
+            q = fminf(fmaxf(__fadd_rn(q, Z), lo_clamp), hi_clamp);
+            b[e] = __float_as_uint(__fadd_rn(__fadd_rn(q, bias), kMagic));
+        }
+        words[w] = pack_low_bytes(b[0], b[1], b[2], b[3]);
+    }
+    return make_uint2(words[0], words[1]);
+}
+
+template <typename T>
+__device__ __noinline__ uint2 e4m3_codes_exact(const uint4 u, float S) {
+    constexpr int V = VecOf<T>::N;
+    float v[V];
+    unpack_vec<T>(u, v);
+    uint32_t words[2] = {0u, 0u};
+    for (int w = 0; w < V / 4; ++w) {
+        uint32_t b[4];
+        for (int e = 0; e < 4; ++e)
+            b[e] = static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(v[4 * w + e], S), __NV_SATFINITE, __NV_E4M3));
+        words[w] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    }
+    return make_uint2(words[0], words[1]);
+}
+
+__device__ __forceinline__ float2 splat2(float a) { return make_float2(a, a); }
+
+// The fast paths below work on pairs with the sm_100 packed fp32 instructions
+// (two IEEE round-to-nearest operations per instruction, so each lane's result
+// is the scalar one).
+
+// Symmetric integer codes clamp(rne(x / S), -127, 127): |x / S| <= 127 up to
+// rounding for every element of the row (the caller masks skipped columns).
+template <typename T, int V>
+__device__ __forceinline__ void int_codes_sym(const uint4 u, const float (&v)[V], float S, float R,
+                                              uint32_t* words) {
+    const float2 R2 = splat2(R), M2 = splat2(kMagic), nM2 = splat2(-kMagic), n1 = splat2(-1.0f);
+    float dmax = 0.f;
+#pragma unroll
+    for (int w = 0; w < V / 4; ++w) {
+        uint32_t b[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float2 t2 = __fmul2_rn(make_float2(v[4 * w + 2 * h], v[4 * w + 2 * h + 1]), R2);
+            const float2 y2 = __fadd2_rn(t2, M2);
+            const float2 d2 = __ffma2_rn(__fadd2_rn(y2, nM2), n1, t2);   // t - rne(t), exact
+            dmax = fmaxf(dmax, fmaxf(fabsf(d2.x), fabsf(d2.y)));
+            b[2 * h] = __float_as_uint(y2.x);
+            b[2 * h + 1] = __float_as_uint(y2.y);
+        }
+        words[w] = pack_low_bytes(b[0], b[1], b[2], b[3]);
+    }
+    if (!(dmax < 0.499f)) {
+        const uint2 r = int_codes_exact<T>(u, S, 0.0f, -127.0f, 127.0f, 0.0f);
+        words[0] = r.x;
+        if constexpr (V == 8) words[1] = r.y;
+    }
+}
+
+// Asymmetric integer codes clamp(rne(x / S) + Z, -128, 127), + 128 for uint8.
+template <typename T, int V>
+__device__ __forceinline__ void int_codes_asym(const uint4 u, const float (&v)[V], float S, float R,
+                                               float Z, float bias, uint32_t* words) {
+    const float2 R2 = splat2(R), M2 = splat2(kMagic), nM2 = splat2(-kMagic), n1 = splat2(-1.0f);
+    const float2 Z2 = splat2(Z), BM2 = splat2(bias + kMagic);
+    float dmax = 0.f;
+#pragma unroll
+    for (int w = 0; w < V / 4; ++w) {
+        uint32_t b[4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float2 t2 = __fmul2_rn(make_float2(v[4 * w + 2 * h], v[4 * w + 2 * h + 1]), R2);
+            t2.x = fminf(fmaxf(t2.x, -1024.0f), 1024.0f);
+            t2.y = fminf(fmaxf(t2.y, -1024.0f), 1024.0f);
+            const float2 q2 = __fadd2_rn(__fadd2_rn(t2, M2), nM2);
+            const float2 d2 = __ffma2_rn(q2, n1, t2);
+            dmax = fmaxf(dmax, fmaxf(fabsf(d2.x), fabsf(d2.y)));
+            float2 c2 = __fadd2_rn(q2, Z2);
+            c2.x = fminf(fmaxf(c2.x, -128.0f), 127.0f);
+            c2.y = fminf(fmaxf(c2.y, -128.0f), 127.0f);
+            const float2 e2 = __fadd2_rn(c2, BM2);   // integers below 2^23 + 2^8: exact
+            b[2 * h] = __float_as_uint(e2.x);
+            b[2 * h + 1] = __float_as_uint(e2.y);
+        }
+        words[w] = pack_low_bytes(b[0], b[1], b[2], b[3]);
+    }
+    if (!(dmax < 0.499f)) {
+        const uint2 r = int_codes_exact<T>(u, S, Z, -128.0f, 127.0f, bias);
+        words[0] = r.x;
+        if constexpr (V == 8) words[1] = r.y;
+    }
+}
+
+template <typename T, int V>
+__device__ __forceinline__ void e4m3_codes(const uint4 u, const float (&v)[V], float S, float R,
+                                           uint32_t* words) {
+    const float2 R2 = splat2(R), lo2 = splat2(1.0f - 0x1p-20f), hi2 = splat2(1.0f + 0x1p-20f);
+    bool bad = false;
+#pragma unroll
+    for (int w = 0; w < V / 4; ++w) {
+        uint32_t hw[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float2 t2 = __fmul2_rn(make_float2(v[4 * w + 2 * h], v[4 * w + 2 * h + 1]), R2);
+            const uint32_t cl = __nv_cvt_float2_to_fp8x2(__fmul2_rn(t2, lo2), __NV_SATFINITE, __NV_E4M3);
+            const uint32_t ch = __nv_cvt_float2_to_fp8x2(__fmul2_rn(t2, hi2), __NV_SATFINITE, __NV_E4M3);
+            bad |= cl != ch;
+            hw[h] = cl;   // element 2h in the low byte, 2h + 1 in the high byte
+        }
+        words[w] = hw[0] | (hw[1] << 16);
+    }
+    if (bad) {
+        const uint2 r = e4m3_codes_exact<T>(u, S);
+        words[0] = r.x;
+        if constexpr (V == 8) words[1] = r.y;
+    }
+}
+
+// One group of TPR threads per row; up to MAXV 16-byte vectors per thread stay
+// in registers between the two passes (longer rows are read twice, the second
+// time from L2).
 template <typename T, int OP, int TPR, int MAXV>
 __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
     constexpr int V = VecOf<T>::N;
@@ -149,13 +305,14 @@ __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
     const int t = threadIdx.x % TPR;
     const int64_t nvec = a.k / V;
     const bool cached = nvec <= static_cast<int64_t>(TPR) * MAXV;
-    // Activation quantizers let a GEMM launched next start its prologue and
-    // weight loads now (it waits for this grid before reading the codes written
-    // here).  This grid was launched without programmatic dependency, so every
-    // earlier kernel, the one that wrote the weights included, has completed.
-    // Weight quantizers do not trigger: a GEMM right after one must not load
-    // the weight before it is fully written.
+    // Launched with programmatic dependent launch: this grid may start while
+    // the previous kernel runs, so it waits for it before touching memory.
+    // Activation quantizers then let the GEMM that follows start its prologue
+    // and weight loads (it waits for this grid before reading the codes).
+    // Weight quantizers do not: a GEMM right after one must not load the
+    // weight before it is fully written.
     if constexpr (OP == kOpActInt8 || OP == kOpActFp8) pdl_launch_dependents();
+    pdl_wait();
 
     for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * RPB; row0 < a.rows;
          row0 += static_cast<int64_t>(gridDim.x) * RPB) {
@@ -165,16 +322,44 @@ __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
 
         uint4 raw[MAXV];  // the row's 16-byte vectors, kept packed between the passes
         RowStats st{0.f, FLT_MAX, -FLT_MAX};
-        auto skipped = [&](int64_t col) -> bool { return a.skip != nullptr && a.skip[col] != 0; };
-        auto accumulate = [&](const float (&v)[V], int64_t j) {
+        const bool use_skip = (OP == kOpActInt8) && a.skip != nullptr;
+        // Pass 1: row absmax (or min and max for the asymmetric scheme).  16-bit
+        // inputs use packed pair min / max / abs, which are exact.
+        auto accumulate = [&](const uint4 u, int64_t j) {
+            if (use_skip) {
+                float v[V];
+                unpack_vec<T>(u, v);
 #pragma unroll
-            for (int e = 0; e < V; ++e) {
-                if constexpr (OP == kOpActInt8) {
-                    if (skipped(j * V + e)) continue;
+                for (int e = 0; e < V; ++e)
+                    if (a.skip[j * V + e] == 0) st.amax = fmaxf(st.amax, fabsf(v[e]));
+            } else if constexpr (sizeof(T) == 2) {
+                using T2 = typename std::conditional<std::is_same<T, __half>::value, __half2, __nv_bfloat162>::type;
+                const T2* p2 = reinterpret_cast<const T2*>(&u);
+                T2 m2 = p2[0];
+                if constexpr (OP == kOpWeightAsym) {
+                    T2 l2 = p2[0];
+#pragma unroll
+                    for (int q = 1; q < 4; ++q) {
+                        m2 = __hmax2(m2, p2[q]);
+                        l2 = __hmin2(l2, p2[q]);
+                    }
+                    st.hi = fmaxf(st.hi, fmaxf(static_cast<float>(m2.x), static_cast<float>(m2.y)));
+                    st.lo = fminf(st.lo, fminf(static_cast<float>(l2.x), static_cast<float>(l2.y)));
+                } else {
+                    m2 = __habs2(m2);
+#pragma unroll
+                    for (int q = 1; q < 4; ++q) m2 = __hmax2(m2, __habs2(p2[q]));
+                    st.amax = fmaxf(st.amax, fmaxf(static_cast<float>(m2.x), static_cast<float>(m2.y)));
                 }
-                st.amax = fmaxf(st.amax, fabsf(v[e]));
-                st.lo = fminf(st.lo, v[e]);
-                st.hi = fmaxf(st.hi, v[e]);
+            } else {
+                float v[V];
+                unpack_vec<T>(u, v);
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    st.amax = fmaxf(st.amax, fabsf(v[e]));
+                    st.lo = fminf(st.lo, v[e]);
+                    st.hi = fmaxf(st.hi, v[e]);
+                }
             }
         };
         if (active) {
@@ -188,21 +373,13 @@ __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
 #pragma unroll
                 for (int i = 0; i < MAXV; ++i) {
                     const int64_t j = t + static_cast<int64_t>(i) * TPR;
-                    if (j < nvec) {
-                        float v[V];
-                        unpack_vec<T>(raw[i], v);
-                        accumulate(v, j);
-                    }
+                    if (j < nvec) accumulate(raw[i], j);
                 }
             } else {
-                for (int64_t j = t; j < nvec; j += TPR) {
-                    float v[V];
-                    load_vec<T>(src + j * V, v);
-                    accumulate(v, j);
-                }
+                for (int64_t j = t; j < nvec; j += TPR) accumulate(ld_stream16(src + j * V), j);
             }
         }
-        st = group_reduce<TPR>(st, red);
+        st = group_reduce<TPR, OP == kOpWeightAsym>(st, red);
 
         float S = 1.f, Z = 0.f;
         if constexpr (OP == kOpActInt8 || OP == kOpWeightSym) {
@@ -219,35 +396,36 @@ __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
             Z = clampf(__fsub_rn(rintf(__fdiv_rn(-st.lo, S)), 128.0f), -128.0f, 127.0f);
         }
 
+        const float R = __frcp_rn(S);   // RN(1/S), shared by the row
         int rsum = 0;
         uint8_t* dst = static_cast<uint8_t*>(a.codes) + (active ? row : 0) * a.k;
-        auto quantize = [&](const float (&v)[V], int64_t j) {
-            uint32_t packed[V / 4];
+        // Pass 2: codes (see int_codes_sym / int_codes_asym / e4m3_codes).
+        auto quantize = [&](const uint4 u, int64_t j) {
+            float v[V];
+            unpack_vec<T>(u, v);
+            uint32_t words[V / 4];
+            if constexpr (OP == kOpActInt8 || OP == kOpWeightSym) {
+                int_codes_sym<T, V>(u, v, S, R, words);
+                if (use_skip) {
+                    // LLM.int8: outlier columns carry code 0 (mask bytes are 0 or 1,
+                    // so mask * 0xFF selects whole bytes).
 #pragma unroll
-            for (int w = 0; w < V / 4; ++w) packed[w] = 0;
-#pragma unroll
-            for (int e = 0; e < V; ++e) {
-                const float qv = __fdiv_rn(v[e], S);
-                uint32_t byte;
-                if constexpr (OP == kOpActInt8 || OP == kOpWeightSym) {
-                    int c = static_cast<int>(clampf(rintf(qv), -127.0f, 127.0f));
-                    if constexpr (OP == kOpActInt8) {
-                        if (skipped(j * V + e)) c = 0;
-                    }
-                    rsum += c;
-                    byte = static_cast<uint32_t>(c) & 0xFFu;
-                } else if constexpr (OP == kOpWeightAsym) {
-                    const int c = static_cast<int>(clampf(__fadd_rn(rintf(qv), Z), -128.0f, 127.0f));
-                    byte = a.codes_u8 ? static_cast<uint32_t>(c + 128) : (static_cast<uint32_t>(c) & 0xFFu);
-                } else {
-                    byte = e4m3_code(qv);
+                    for (int w = 0; w < V / 4; ++w)
+                        words[w] &= ~(*reinterpret_cast<const uint32_t*>(a.skip + j * V + 4 * w) * 0xFFu);
                 }
-                packed[e / 4] |= byte << (8 * (e % 4));
+                if constexpr (OP == kOpActInt8) {
+#pragma unroll
+                    for (int w = 0; w < V / 4; ++w) rsum = __dp4a(static_cast<int>(words[w]), 0x01010101, rsum);
+                }
+            } else if constexpr (OP == kOpWeightAsym) {
+                int_codes_asym<T, V>(u, v, S, R, Z, a.codes_u8 ? 128.0f : 0.0f, words);
+            } else {
+                e4m3_codes<T, V>(u, v, S, R, words);
             }
             if constexpr (V == 8) {
-                *reinterpret_cast<uint2*>(dst + j * V) = make_uint2(packed[0], packed[1]);
+                *reinterpret_cast<uint2*>(dst + j * V) = make_uint2(words[0], words[1]);
             } else {
-                *reinterpret_cast<uint32_t*>(dst + j * V) = packed[0];
+                *reinterpret_cast<uint32_t*>(dst + j * V) = words[0];
             }
         };
         if (active) {
@@ -255,18 +433,10 @@ __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
 #pragma unroll
                 for (int i = 0; i < MAXV; ++i) {
                     const int64_t j = t + static_cast<int64_t>(i) * TPR;
-                    if (j < nvec) {
-                        float v[V];
-                        unpack_vec<T>(raw[i], v);
-                        quantize(v, j);
-                    }
+                    if (j < nvec) quantize(raw[i], j);
                 }
             } else {
-                for (int64_t j = t; j < nvec; j += TPR) {
-                    float v[V];
-                    load_vec<T>(src + j * V, v);
-                    quantize(v, j);
-                }
+                for (int64_t j = t; j < nvec; j += TPR) quantize(ld_stream16(src + j * V), j);
             }
         }
         if constexpr (OP == kOpActInt8) rsum = group_sum<TPR>(rsum, redi);
@@ -314,14 +484,28 @@ cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
         constexpr int RPB = kBlock / TPR;
         int64_t blocks = (a.rows + RPB - 1) / RPB;
         if (blocks > 65535 * 4) blocks = 65535 * 4;
-        row_quant_kernel<T, OP, TPR, 8><<<static_cast<unsigned>(blocks), kBlock, 0, s>>>(a);
-        return cudaGetLastError();
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+        cfg.blockDim = dim3(kBlock, 1, 1);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, row_quant_kernel<T, OP, TPR, kMaxVec>, a);
     };
-    // With few rows, spread each row over more threads so more loads are in flight.
-    const bool few_rows = a.rows < 4 * 148;
-    if (nvec <= 32 * 8 && !few_rows) return go(std::integral_constant<int, 32>{});
-    if (nvec <= 64 * 8 && !(few_rows && nvec > 64 * 2)) return go(std::integral_constant<int, 64>{});
-    if (nvec <= 128 * 8 && !(few_rows && nvec > 128 * 2)) return go(std::integral_constant<int, 128>{});
+    // Threads per row: enough to hold the row in registers (16 vectors a
+    // thread), and, for short matrices, enough to spread the rows over the SMs;
+    // otherwise as few as possible, so the per-row reductions (warp shuffles
+    // for one warp) stay a small part of the work.
+    int64_t need = (nvec + kMaxVec - 1) / kMaxVec;
+    int64_t spread = (static_cast<int64_t>(kBlock) * 148 + a.rows - 1) / (a.rows > 0 ? a.rows : 1);
+    const int64_t tpr = need > spread ? need : spread;
+    if (tpr <= 32) return go(std::integral_constant<int, 32>{});
+    if (tpr <= 64) return go(std::integral_constant<int, 64>{});
+    if (tpr <= 128) return go(std::integral_constant<int, 128>{});
     return go(std::integral_constant<int, 256>{});
 }
 

@@ -214,14 +214,16 @@ q8_status q8_outlier_quantize_act(const void *X, q8_dtype x_dtype, int64_t m, in
  *              output (row stride n), or NULL.
  *   workspace  unused by this call today; pass q8_workspace_size(Q8_OP_LINEAR_W8A8, ...)
  *              bytes (currently 0; NULL accepted).
- * Launch overlap: the GEMM is launched with programmatic dependent launch.
- * When the kernel right before it in the stream is this library's activation
- * quantizer, the GEMM starts loading the weight while that kernel runs and
- * waits for it before reading x.  Every kernel before the quantizer has
- * finished by then, so the weight only has to be complete before the
- * quantizer is launched, which stream order already guarantees.  (A kernel of
- * the caller's own that runs right before this call and triggers programmatic
- * launch early must not be the one writing the weight.)
+ * Launch overlap: the quantize and GEMM kernels are launched with
+ * programmatic dependent launch, and each waits for the kernel before it
+ * before reading anything that kernel may write.  The one exception is the
+ * weight: when the kernel right before the GEMM is this library's activation
+ * quantizer, the GEMM starts loading the weight early, while that quantizer
+ * and the kernel before it may still run.  The weight must therefore not be
+ * written by a kernel that triggers programmatic launch early
+ * (griddepcontrol.launch_dependents) and runs just before the quantizer.  This
+ * library's weight quantizer does not trigger, so quantize_weight followed by
+ * any sequence of these calls is safe.
  */
 q8_status q8_linear_w8a8(const q8_act *x, const q8_weight *w, const float *bias, void *Y,
                          int64_t ldy, void *acc_debug, void *workspace, size_t ws_bytes,

@@ -192,3 +192,28 @@ def test_outlier_act_one_row():
     X = workloads.random_matrix(1, 64, torch.float16, seed=32)
     X[0, 63] = 7.0
     assert _outlier_check(X, 6.0, "one row") == 1
+
+
+def test_quotient_rounding_at_exact_midpoints():
+    """Rows whose scale is exactly 1 put x / S on integer and E4M3 rounding
+    midpoints, where the kernel must fall back to the exact quotient."""
+    ints = [127.0, 62.5, 63.5, -62.5, -63.5, 0.5, 1.5, -0.5, 2.5, -2.5, 100.5, -126.5]
+    Xi = torch.zeros(2, 64, dtype=torch.bfloat16)
+    Xi[0, :len(ints)] = torch.tensor(ints)
+    Xi[1, :len(ints)] = -torch.tensor(ints)
+    _act_int8_check(Xi, P.host_f32(Xi), "integer midpoints")
+    # E4M3 midpoints: 1.0625 (1 | 1.125), 3.125 (3 | 3.25), 0.0029296875 (subnormal 3*2^-10),
+    # 240 (224 | 256), 432 (416 | 448)
+    mids = [448.0, 1.0625, 3.125, 0.0029296875, 240.0, 432.0, -1.0625, -240.0, 1.1875, 13.0]
+    Xf = torch.zeros(2, 64, dtype=torch.bfloat16)
+    Xf[0, :len(mids)] = torch.tensor(mids)
+    Xf[1, :len(mids)] = -torch.tensor(mids)
+    _act_fp8_check(Xf, P.host_f32(Xf), 0.0, "e4m3 midpoints")
+    W = torch.zeros(16, 64, dtype=torch.bfloat16)
+    W[0, :len(mids)] = torch.tensor(mids)
+    _weight_check(W, P.host_f32(W), "fp8", "e4m3", "weight e4m3 midpoints")
+    Wa = torch.zeros(16, 64, dtype=torch.float32)
+    Wa[:, 0] = 0.0
+    Wa[:, 1] = 255.0            # S = 1 exactly, Z = -128
+    Wa[:, 2:14] = torch.tensor([0.5, 1.5, 2.5, 100.5, 127.5, 128.5, 200.5, 254.5, 3.5, 4.5, 5.5, 6.5])
+    _weight_check(Wa, P.host_f32(Wa), "asym", "s8", "asym integer midpoints")
