@@ -80,6 +80,17 @@ struct RowStats {
     float amax, lo, hi;
 };
 
+// Barrier over the TPR threads of one row group (named barrier 1 + group;
+// the whole block when one group fills it).
+template <int TPR>
+__device__ __forceinline__ void group_sync() {
+    if constexpr (TPR >= kBlock) {
+        __syncthreads();
+    } else {
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + static_cast<int>(threadIdx.x) / TPR), "n"(TPR) : "memory");
+    }
+}
+
 // Reduction of per-thread stats over the TPR threads that share a row.
 template <int TPR, bool MINMAX>
 __device__ __forceinline__ RowStats group_reduce(RowStats s, float* red) {
@@ -98,7 +109,7 @@ __device__ __forceinline__ RowStats group_reduce(RowStats s, float* red) {
         if (lane == 0) {
             red[3 * warp] = s.amax; red[3 * warp + 1] = s.lo; red[3 * warp + 2] = s.hi;
         }
-        __syncthreads();
+        group_sync<TPR>();
         const int base = (warp / W) * W;
         RowStats r{0.f, FLT_MAX, -FLT_MAX};
 #pragma unroll
@@ -107,7 +118,7 @@ __device__ __forceinline__ RowStats group_reduce(RowStats s, float* red) {
             r.lo = fminf(r.lo, red[3 * (base + i) + 1]);
             r.hi = fmaxf(r.hi, red[3 * (base + i) + 2]);
         }
-        __syncthreads();
+        group_sync<TPR>();
         return r;
     }
     return s;
@@ -121,12 +132,12 @@ __device__ __forceinline__ int group_sum(int v, int* red) {
         constexpr int W = TPR / 32;
         const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
         if (lane == 0) red[warp] = v;
-        __syncthreads();
+        group_sync<TPR>();
         const int base = (warp / W) * W;
         int r = 0;
 #pragma unroll
         for (int i = 0; i < W; ++i) r += red[base + i];
-        __syncthreads();
+        group_sync<TPR>();
         return r;
     }
     return v;
@@ -137,317 +148,432 @@ __device__ __forceinline__ float clampf(float v, float lo, float hi) {
 }
 
 
-// Codes of one 16-byte vector (V elements) from the IEEE quotient fl32(x / S),
-// without a division per element.
+// Codes of one 16-byte vector (V elements) without a division per element.
 //
-// With R = RN(1/S) (one reciprocal per row) the product t = RN(x * R) has a
-// relative error below 2^-23 against x / S, and fl32(x / S) adds 2^-24, so
-// |t - fl32(x / S)| <= 1.5 * 2^-23 |t|.
-//   Integer codes: |t| <= 1024 (wider inputs are clamped; their codes saturate
-//   anyway).  Adding 1.5 * 2^23 rounds t to an integer half to even (the sum lies
-//   in [2^23, 2^24), where floats are integers, and the constant is even); the
-//   low byte of the sum is the code's two's-complement byte (the constant's low
-//   byte is 0), and d = t - rne(t) is exact.  An ulp of t is at most 2^-13, so
-//   when |d| < 0.499 no half-integer lies between t and fl32(x / S): both round
-//   to the same integer.
-//   E4M3 codes: rounding to E4M3 (half to even, saturating) is monotonic, and
-//   t (1 - 2^-20) and t (1 + 2^-20) bracket fl32(x / S); when both convert to
-//   the same code, so does fl32(x / S).  (Values too small for the bracket to
-//   widen round to zero either way.)
-// A vector with any element near a rounding boundary is redone with exact
-// divisions, out of line (it is rare).
-constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+// The target is a rounding of the IEEE quotient fl32(x / S): rne for integer
+// codes, E4M3 (half to even, saturating) for FP8.  Each row gets two
+// multipliers rlo <= 1/S <= rhi, made with directed roundings and widened so
+// that x * rlo and x * rhi (after the fast path's own rounding) enclose
+// fl32(x / S), with fl32(x / S) strictly inside for integer codes.  Both
+// roundings are monotonic, so where the two ends of the bracket give the same
+// code, that is the code of fl32(x / S).  Elements where they differ lie within
+// a few ulps of a rounding boundary; their codes are recomputed with an exact
+// division.  That is not as rare as the bracket width suggests: with 16-bit
+// inputs, x / S often falls exactly on a boundary (127 x / absmax is a ratio of
+// two short mantissas), about 2 elements in 1000.
+//   Integer codes: one fused multiply-add per end, y = RN(x * r + c), with
+//   c = 1.5 * 2^23 (+ Z + bias for asymmetric codes).  The exact product plus
+//   c lies in [2^23, 2^24), where floats are the integers, so y - c is x * r
+//   rounded to an integer and the low byte of y is the code byte.  With Z
+//   folded into c an exact tie would round to the parity of c, but a tie
+//   strictly inside the bracket makes the two ends differ, so folded ties are
+//   always recomputed.  Rows where |x * r| could leave that range, or whose
+//   codes would need the [-128, 127] clamp, are coded exactly throughout
+//   (constant rows, rows that do not cross zero).
+//   E4M3 codes: t = RN(x * r) per end, then the hardware conversion.
+constexpr float kMagic = 12582912.0f;    // 1.5 * 2^23
+constexpr float kFastLimit = 2097152.0f; // 2^21: bound on |x * r| for the integer fast path
+
+// Internal op for the LLM.int8 regular stream: int8 activations with the
+// outlier columns (mask bytes of 1) left out of the absmax and coded as 0.
+constexpr int kOpActInt8Skip = 5;
 
 __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
     return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
-// Exact out-of-line paths; they take the packed input vector and return the
-// packed codes by value so the fast paths keep everything in registers.
-template <typename T>
-__device__ __noinline__ uint2 int_codes_exact(const uint4 u, float S, float Z, float lo_clamp,
-                                              float hi_clamp, float bias) {
-    constexpr int V = VecOf<T>::N;
-    float v[V];
-    unpack_vec<T>(u, v);
-    uint32_t words[2] = {0u, 0u};
-    for (int w = 0; w < V / 4; ++w) {
-        uint32_t b[4];
-        for (int e = 0; e < 4; ++e) {
-            float q = rintf(__fdiv_rn(v[4 * w + e], S));
-            q = fminf(fmaxf(__fadd_rn(q, Z), lo_clamp), hi_clamp);
-            b[e] = __float_as_uint(__fadd_rn(__fadd_rn(q, bias), kMagic));
-        }
-        words[w] = pack_low_bytes(b[0], b[1], b[2], b[3]);
-    }
-    return make_uint2(words[0], words[1]);
-}
-
-template <typename T>
-__device__ __noinline__ uint2 e4m3_codes_exact(const uint4 u, float S) {
-    constexpr int V = VecOf<T>::N;
-    float v[V];
-    unpack_vec<T>(u, v);
-    uint32_t words[2] = {0u, 0u};
-    for (int w = 0; w < V / 4; ++w) {
-        uint32_t b[4];
-        for (int e = 0; e < 4; ++e)
-            b[e] = static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(v[4 * w + e], S), __NV_SATFINITE, __NV_E4M3));
-        words[w] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-    }
-    return make_uint2(words[0], words[1]);
-}
-
 __device__ __forceinline__ float2 splat2(float a) { return make_float2(a, a); }
 
-// The fast paths below work on pairs with the sm_100 packed fp32 instructions
-// (two IEEE round-to-nearest operations per instruction, so each lane's result
-// is the scalar one).
+// Per-row constants.
+struct RowConsts {
+    float S, Z, bias;
+    float rlo, rhi;   // bracket multipliers
+    float add;        // integer codes: 1.5 * 2^23 + Z + bias
+    bool fast;        // the row may use the bracket path
+};
 
-// Symmetric integer codes clamp(rne(x / S), -127, 127): |x / S| <= 127 up to
-// rounding for every element of the row (the caller masks skipped columns).
-template <typename T, int V>
-__device__ __forceinline__ void int_codes_sym(const uint4 u, const float (&v)[V], float S, float R,
-                                              uint32_t* words) {
-    const float2 R2 = splat2(R), M2 = splat2(kMagic), nM2 = splat2(-kMagic), n1 = splat2(-1.0f);
-    float dmax = 0.f;
-#pragma unroll
-    for (int w = 0; w < V / 4; ++w) {
-        uint32_t b[4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const float2 t2 = __fmul2_rn(make_float2(v[4 * w + 2 * h], v[4 * w + 2 * h + 1]), R2);
-            const float2 y2 = __fadd2_rn(t2, M2);
-            const float2 d2 = __ffma2_rn(__fadd2_rn(y2, nM2), n1, t2);   // t - rne(t), exact
-            dmax = fmaxf(dmax, fmaxf(fabsf(d2.x), fabsf(d2.y)));
-            b[2 * h] = __float_as_uint(y2.x);
-            b[2 * h + 1] = __float_as_uint(y2.y);
-        }
-        words[w] = pack_low_bytes(b[0], b[1], b[2], b[3]);
+template <int OP>
+__device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, float clip_ub, float bias) {
+    RowConsts c;
+    c.Z = 0.f;
+    c.bias = bias;
+    if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpWeightSym) {
+        c.S = __fdiv_rn(amax, 127.0f);
+    } else if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
+        if (OP == kOpActFp8 && clip_ub > 0.f) amax = fminf(amax, clip_ub);
+        c.S = __fdiv_rn(amax, 448.0f);
+    } else {
+        c.S = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
     }
-    if (!(dmax < 0.499f)) {
-        const uint2 r = int_codes_exact<T>(u, S, 0.0f, -127.0f, 127.0f, 0.0f);
-        words[0] = r.x;
-        if constexpr (V == 8) words[1] = r.y;
+    if (!(c.S >= kEps)) c.S = kEps;
+    // When S is a power of two, 1/S is exact and so is x * (1/S) = x / S (the
+    // product keeps x's significand): no bracket is needed, except for
+    // asymmetric codes with an odd Z + bias folded into the rounding constant.
+    const float rd = __frcp_rd(c.S), ru = __frcp_ru(c.S);
+    const bool exact_rcp = rd == ru;
+    if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
+        // t = RN(x * r) adds one more rounding (2^-24) on top of the ends.
+        c.rlo = exact_rcp ? rd : __fmul_rd(rd, 1.0f - 0x1p-22f);
+        c.rhi = exact_rcp ? ru : __fmul_ru(ru, 1.0f + 0x1p-22f);
+        c.add = 0.f;
+        c.fast = true;
+    } else {
+        // fl32(x / S) is within 2^-24 of x / S; the (1 -+ 2^-23) factors put it
+        // strictly inside [x * rlo, x * rhi] (the products are exact in the FMA).
+        c.rlo = __fmul_rd(rd, 1.0f - 0x1p-23f);
+        c.rhi = __fmul_ru(ru, 1.0f + 0x1p-23f);
+        if constexpr (OP == kOpWeightAsym) {
+            c.Z = clampf(__fsub_rn(rintf(__fdiv_rn(-lo, c.S)), 128.0f), -128.0f, 127.0f);
+            // Codes are monotonic in w: the ends of the row bound all of them.
+            const float qlo = __fadd_rn(rintf(__fdiv_rn(lo, c.S)), c.Z);
+            const float qhi = __fadd_rn(rintf(__fdiv_rn(hi, c.S)), c.Z);
+            c.fast = fmaxf(fabsf(lo), fabsf(hi)) * c.rhi <= kFastLimit && qlo >= -128.0f && qhi <= 127.0f;
+            if (exact_rcp && (static_cast<int>(c.Z + bias) & 1) == 0) c.rlo = c.rhi = rd;
+        } else {
+            c.fast = amax * c.rhi <= kFastLimit;
+            if (exact_rcp) c.rlo = c.rhi = rd;
+        }
+        c.add = kMagic + c.Z + bias;   // an integer below 2^24: exact
+    }
+    return c;
+}
+
+// Fast codes of one vector from the lower end of the bracket, and per word the
+// code bytes where the upper end disagrees.  keep clears the bytes of left-out
+// columns (all ones otherwise); their disagreements do not count.
+template <typename T, int OP>
+__device__ __forceinline__ void fast_codes(const uint4 u, const RowConsts& c, const uint2 keep,
+                                           uint32_t (&words)[2], uint32_t (&diff)[2]) {
+    constexpr int V = VecOf<T>::N;
+    const uint32_t kp[2] = {keep.x, keep.y};
+    float v[V];
+    unpack_vec<T>(u, v);
+    words[1] = diff[1] = 0u;
+    if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
+        const float2 L = splat2(c.rlo), H = splat2(c.rhi);
+#pragma unroll
+        for (int w = 0; w < V / 4; ++w) {
+            uint32_t cl[2], cd[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float2 x2 = make_float2(v[4 * w + 2 * h], v[4 * w + 2 * h + 1]);
+                cl[h] = __nv_cvt_float2_to_fp8x2(__fmul2_rn(x2, L), __NV_SATFINITE, __NV_E4M3);
+                cd[h] = cl[h] ^ __nv_cvt_float2_to_fp8x2(__fmul2_rn(x2, H), __NV_SATFINITE, __NV_E4M3);
+            }
+            // element 2h in the low byte of each half, 2h + 1 in the high byte
+            words[w] = __byte_perm(cl[0], cl[1], 0x5410);
+            diff[w] = __byte_perm(cd[0], cd[1], 0x5410);
+        }
+    } else {
+        const float2 L = splat2(c.rlo), H = splat2(c.rhi), A = splat2(c.add);
+#pragma unroll
+        for (int w = 0; w < V / 4; ++w) {
+            const float2 x0 = make_float2(v[4 * w], v[4 * w + 1]);
+            const float2 x1 = make_float2(v[4 * w + 2], v[4 * w + 3]);
+            const float2 l0 = __ffma2_rn(x0, L, A), l1 = __ffma2_rn(x1, L, A);
+            const float2 h0 = __ffma2_rn(x0, H, A), h1 = __ffma2_rn(x1, H, A);
+            const uint32_t lw = pack_low_bytes(__float_as_uint(l0.x), __float_as_uint(l0.y),
+                                               __float_as_uint(l1.x), __float_as_uint(l1.y)) & kp[w];
+            const uint32_t hw = pack_low_bytes(__float_as_uint(h0.x), __float_as_uint(h0.y),
+                                               __float_as_uint(h1.x), __float_as_uint(h1.y)) & kp[w];
+            words[w] = lw;
+            diff[w] = lw ^ hw;
+        }
     }
 }
 
-// Asymmetric integer codes clamp(rne(x / S) + Z, -128, 127), + 128 for uint8.
-template <typename T, int V>
-__device__ __forceinline__ void int_codes_asym(const uint4 u, const float (&v)[V], float S, float R,
-                                               float Z, float bias, uint32_t* words) {
-    const float2 R2 = splat2(R), M2 = splat2(kMagic), nM2 = splat2(-kMagic), n1 = splat2(-1.0f);
-    const float2 Z2 = splat2(Z), BM2 = splat2(bias + kMagic);
-    float dmax = 0.f;
-#pragma unroll
-    for (int w = 0; w < V / 4; ++w) {
-        uint32_t b[4];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float2 t2 = __fmul2_rn(make_float2(v[4 * w + 2 * h], v[4 * w + 2 * h + 1]), R2);
-            t2.x = fminf(fmaxf(t2.x, -1024.0f), 1024.0f);
-            t2.y = fminf(fmaxf(t2.y, -1024.0f), 1024.0f);
-            const float2 q2 = __fadd2_rn(__fadd2_rn(t2, M2), nM2);
-            const float2 d2 = __ffma2_rn(q2, n1, t2);
-            dmax = fmaxf(dmax, fmaxf(fabsf(d2.x), fabsf(d2.y)));
-            float2 c2 = __fadd2_rn(q2, Z2);
-            c2.x = fminf(fmaxf(c2.x, -128.0f), 127.0f);
-            c2.y = fminf(fmaxf(c2.y, -128.0f), 127.0f);
-            const float2 e2 = __fadd2_rn(c2, BM2);   // integers below 2^23 + 2^8: exact
-            b[2 * h] = __float_as_uint(e2.x);
-            b[2 * h + 1] = __float_as_uint(e2.y);
+// Exact codes, with an IEEE division, for the elements of a vector whose byte
+// in `redo` is nonzero; the other bytes of `words` are kept.  Out of line: it
+// runs for a few elements in a thousand.
+template <typename T, int OP>
+__device__ __noinline__ uint2 exact_codes(const uint4 u, float S, float Z, float bias, uint2 redo,
+                                          uint2 words) {
+    constexpr int V = VecOf<T>::N;
+    float v[V];
+    unpack_vec<T>(u, v);
+    uint32_t w[2] = {words.x, words.y};
+    const uint32_t r[2] = {redo.x, redo.y};
+    for (int e = 0; e < V; ++e) {
+        const int sh = 8 * (e % 4);
+        if (((r[e / 4] >> sh) & 0xFFu) == 0u) continue;
+        uint32_t b;
+        if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
+            b = static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(v[e], S), __NV_SATFINITE, __NV_E4M3));
+        } else {
+            const float lo = OP == kOpWeightAsym ? -128.0f : -127.0f;
+            const float q = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(v[e], S)), Z), lo), 127.0f);
+            b = static_cast<uint32_t>(static_cast<int>(__fadd_rn(q, bias))) & 0xFFu;
         }
-        words[w] = pack_low_bytes(b[0], b[1], b[2], b[3]);
+        w[e / 4] = (w[e / 4] & ~(0xFFu << sh)) | (b << sh);
     }
-    if (!(dmax < 0.499f)) {
-        const uint2 r = int_codes_exact<T>(u, S, Z, -128.0f, 127.0f, bias);
-        words[0] = r.x;
-        if constexpr (V == 8) words[1] = r.y;
+    return make_uint2(w[0], w[1]);
+}
+
+// Exact code byte of one element.
+template <int OP>
+__device__ __forceinline__ uint32_t exact_code(float x, float S, float Z, float bias) {
+    if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
+        return static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(x, S), __NV_SATFINITE, __NV_E4M3));
+    } else {
+        const float lo = OP == kOpWeightAsym ? -128.0f : -127.0f;
+        const float q = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(x, S)), Z), lo), 127.0f);
+        return static_cast<uint32_t>(static_cast<int>(__fadd_rn(q, bias))) & 0xFFu;
     }
 }
 
-template <typename T, int V>
-__device__ __forceinline__ void e4m3_codes(const uint4 u, const float (&v)[V], float S, float R,
-                                           uint32_t* words) {
-    const float2 R2 = splat2(R), lo2 = splat2(1.0f - 0x1p-20f), hi2 = splat2(1.0f + 0x1p-20f);
-    bool bad = false;
+// Per-warp queue of elements whose bracket ends disagree: their value, their
+// byte position in the row and the fast code written for them.
+constexpr int kQueueCap = 320;
+constexpr int kDrainAt = 64;   // drained once this full: one step adds at most 32 x 8
+struct FixQueue {
+    float x[kQueueCap];
+    int pos[kQueueCap];
+    int fast[kQueueCap];
+    int n;
+};
+
+// Pushes the flagged elements of one vector (bytes of d that are nonzero).
+// Out of line, so the unrolled pass keeps a small instruction footprint.
+template <typename T>
+__device__ __noinline__ void push_flagged(const uint4 u, uint2 d, uint2 w, int pos0, FixQueue* q) {
+    constexpr int V = VecOf<T>::N;
+    float v[V];
+    unpack_vec<T>(u, v);
+    const uint32_t dd[2] = {d.x, d.y}, ww[2] = {w.x, w.y};
 #pragma unroll
-    for (int w = 0; w < V / 4; ++w) {
-        uint32_t hw[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const float2 t2 = __fmul2_rn(make_float2(v[4 * w + 2 * h], v[4 * w + 2 * h + 1]), R2);
-            const uint32_t cl = __nv_cvt_float2_to_fp8x2(__fmul2_rn(t2, lo2), __NV_SATFINITE, __NV_E4M3);
-            const uint32_t ch = __nv_cvt_float2_to_fp8x2(__fmul2_rn(t2, hi2), __NV_SATFINITE, __NV_E4M3);
-            bad |= cl != ch;
-            hw[h] = cl;   // element 2h in the low byte, 2h + 1 in the high byte
+    for (int e = 0; e < V; ++e) {
+        const int sh = 8 * (e % 4);
+        if (((dd[e / 4] >> sh) & 0xFFu) != 0u) {
+            const int slot = atomicAdd(&q->n, 1);
+            if (slot < kQueueCap) {
+                q->x[slot] = v[e];
+                q->pos[slot] = pos0 + e;
+                q->fast[slot] = static_cast<int>(static_cast<int8_t>((ww[e / 4] >> sh) & 0xFFu));
+            }
         }
-        words[w] = hw[0] | (hw[1] << 16);
-    }
-    if (bad) {
-        const uint2 r = e4m3_codes_exact<T>(u, S);
-        words[0] = r.x;
-        if constexpr (V == 8) words[1] = r.y;
     }
 }
 
-// One group of TPR threads per row; up to MAXV 16-byte vectors per thread stay
-// in registers between the two passes (longer rows are read twice, the second
-// time from L2).
+// Recodes the queued elements, 32 at a time, and empties the queue; returns
+// the change of this lane's share of the row sum (int8 codes).  Called by the
+// whole warp, after the fast codes of the queued elements are stored: the
+// barrier orders those stores before the corrections, which another lane of
+// the warp may write.
+template <int OP>
+__device__ __noinline__ int drain_queue(FixQueue* q, uint8_t* dst_row, float S, float Z, float bias) {
+    __syncwarp();
+    const int n = q->n;
+    int delta = 0;
+    for (int e = threadIdx.x & 31; e < n; e += 32) {
+        const uint32_t b = exact_code<OP>(q->x[e], S, Z, bias);
+        dst_row[q->pos[e]] = static_cast<uint8_t>(b);
+        delta += static_cast<int>(static_cast<int8_t>(b)) - q->fast[e];
+    }
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) q->n = 0;
+    __syncwarp();
+    return delta;
+}
+
+// Zeroes the 16-bit elements of a vector that are left out; mb holds 0xFF per
+// left-out element.
+__device__ __forceinline__ uint4 zero_skipped16(uint4 u, const uint2 mb) {
+    // widen each mask byte to its 16-bit lane
+    const uint32_t k0 = __byte_perm(mb.x, 0u, 0x1100), k1 = __byte_perm(mb.x, 0u, 0x3322);
+    const uint32_t k2 = __byte_perm(mb.y, 0u, 0x1100), k3 = __byte_perm(mb.y, 0u, 0x3322);
+    u.x &= ~k0; u.y &= ~k1; u.z &= ~k2; u.w &= ~k3;
+    return u;
+}
+
+template <typename T, int OP>
+__device__ __forceinline__ void accumulate_stats(const uint4 u, RowStats& st) {
+    constexpr int V = VecOf<T>::N;
+    if constexpr (sizeof(T) == 2) {
+        using T2 = typename std::conditional<std::is_same<T, __half>::value, __half2, __nv_bfloat162>::type;
+        const T2* p2 = reinterpret_cast<const T2*>(&u);
+        T2 m2 = __hmax2(p2[0], p2[1]), l2 = __hmin2(p2[0], p2[1]);
+        m2 = __hmax2(m2, __hmax2(p2[2], p2[3]));
+        l2 = __hmin2(l2, __hmin2(p2[2], p2[3]));
+        st.hi = fmaxf(st.hi, fmaxf(static_cast<float>(m2.x), static_cast<float>(m2.y)));
+        st.lo = fminf(st.lo, fminf(static_cast<float>(l2.x), static_cast<float>(l2.y)));
+    } else {
+        float v[V];
+        unpack_vec<T>(u, v);
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            st.lo = fminf(st.lo, v[e]);
+            st.hi = fmaxf(st.hi, v[e]);
+        }
+    }
+}
+
+// One group of TPR (a multiple of 32) threads per row.  Thread t of a group
+// handles the row's 16-byte vectors t, t + TPR, t + 2 TPR, ...; up to MAXV of
+// them stay in registers between the two passes (longer rows are read twice,
+// the second time from L2).
 template <typename T, int OP, int TPR, int MAXV>
 __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
+    static_assert(TPR % 32 == 0, "a warp works on one row");
     constexpr int V = VecOf<T>::N;
     constexpr int RPB = kBlock / TPR;
+    constexpr bool kSkip = OP == kOpActInt8Skip;
+    constexpr bool kRowsum = OP == kOpActInt8 || OP == kOpActInt8Skip;
     __shared__ float red[3 * (kBlock / 32)];
     __shared__ int redi[kBlock / 32];
+    __shared__ FixQueue fixq[kBlock / 32];
+    FixQueue* q = &fixq[threadIdx.x / 32];
 
     const int g = threadIdx.x / TPR;
     const int t = threadIdx.x % TPR;
     const int64_t nvec = a.k / V;
     const bool cached = nvec <= static_cast<int64_t>(TPR) * MAXV;
+    // Vectors this thread holds when the row is cached, and the most any
+    // thread of its warp holds (the first one).
+    const int nvl = cached ? static_cast<int>((nvec - t + TPR - 1) / TPR) : 0;
+    const int nvw = cached ? static_cast<int>((nvec - (t & ~31) + TPR - 1) / TPR) : 0;
+    const float bias = (OP == kOpWeightAsym && a.codes_u8) ? 128.0f : 0.0f;
     // Launched with programmatic dependent launch: this grid may start while
     // the previous kernel runs, so it waits for it before touching memory.
     // Activation quantizers then let the GEMM that follows start its prologue
     // and weight loads (it waits for this grid before reading the codes).
     // Weight quantizers do not: a GEMM right after one must not load the
     // weight before it is fully written.
-    if constexpr (OP == kOpActInt8 || OP == kOpActFp8) pdl_launch_dependents();
+    if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActFp8) pdl_launch_dependents();
     pdl_wait();
 
     for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * RPB; row0 < a.rows;
          row0 += static_cast<int64_t>(gridDim.x) * RPB) {
         const int64_t row = row0 + g;
-        const bool active = row < a.rows;
-        const T* src = static_cast<const T*>(a.src) + (active ? row : 0) * a.ld;
+        const bool active = row < a.rows;   // the same for a whole warp
+        const T* src_row = static_cast<const T*>(a.src) + (active ? row : 0) * a.ld;
+        uint8_t* dst_row = static_cast<uint8_t*>(a.codes) + (active ? row : 0) * a.k;
+        const T* src = src_row + static_cast<int64_t>(t) * V;
+        uint8_t* dst = dst_row + static_cast<int64_t>(t) * V;
+        const int nv = active ? nvl : 0;
+        const int nvmax = active ? nvw : 0;
+        // Every thread of the block holds MAXV vectors: no per-vector guards.
+        // (Uniform over the block, as the reductions below synchronize it.)
+        const bool full = nvec == static_cast<int64_t>(TPR) * MAXV && row0 + RPB <= a.rows;
+        auto keep_of = [&](int64_t j) -> uint2 {
+            if constexpr (kSkip) {
+                const uint2 m = *reinterpret_cast<const uint2*>(a.skip + j * V);
+                return make_uint2(~(m.x * 0xFFu), ~(m.y * 0xFFu));
+            } else {
+                return make_uint2(~0u, ~0u);
+            }
+        };
 
-        uint4 raw[MAXV];  // the row's 16-byte vectors, kept packed between the passes
+        // Pass 1: row min and max (absmax = max(max, -min)).  Vectors past the
+        // end of the row are zero, which leaves absmax unchanged; asymmetric
+        // rows only count loaded vectors.  Left-out columns are zeroed.
+        uint4 raw[MAXV];
         RowStats st{0.f, FLT_MAX, -FLT_MAX};
-        const bool use_skip = (OP == kOpActInt8) && a.skip != nullptr;
-        // Pass 1: row absmax (or min and max for the asymmetric scheme).  16-bit
-        // inputs use packed pair min / max / abs, which are exact.
-        auto accumulate = [&](const uint4 u, int64_t j) {
-            if (use_skip) {
-                float v[V];
-                unpack_vec<T>(u, v);
+        auto pass1 = [&](auto full_tag) {
+            constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
-                for (int e = 0; e < V; ++e)
-                    if (a.skip[j * V + e] == 0) st.amax = fmaxf(st.amax, fabsf(v[e]));
-            } else if constexpr (sizeof(T) == 2) {
-                using T2 = typename std::conditional<std::is_same<T, __half>::value, __half2, __nv_bfloat162>::type;
-                const T2* p2 = reinterpret_cast<const T2*>(&u);
-                T2 m2 = p2[0];
-                if constexpr (OP == kOpWeightAsym) {
-                    T2 l2 = p2[0];
+            for (int i = 0; i < MAXV; ++i)
+                raw[i] = (FULL || i < nv) ? ld_stream16(src + i * TPR * V) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-                    for (int q = 1; q < 4; ++q) {
-                        m2 = __hmax2(m2, p2[q]);
-                        l2 = __hmin2(l2, p2[q]);
+            for (int i = 0; i < MAXV; ++i) {
+                if (FULL || i < nv) {
+                    if constexpr (kSkip) {
+                        const uint2 kp = keep_of(t + static_cast<int64_t>(i) * TPR);
+                        raw[i] = zero_skipped16(raw[i], make_uint2(~kp.x, ~kp.y));
                     }
-                    st.hi = fmaxf(st.hi, fmaxf(static_cast<float>(m2.x), static_cast<float>(m2.y)));
-                    st.lo = fminf(st.lo, fminf(static_cast<float>(l2.x), static_cast<float>(l2.y)));
-                } else {
-                    m2 = __habs2(m2);
-#pragma unroll
-                    for (int q = 1; q < 4; ++q) m2 = __hmax2(m2, __habs2(p2[q]));
-                    st.amax = fmaxf(st.amax, fmaxf(static_cast<float>(m2.x), static_cast<float>(m2.y)));
-                }
-            } else {
-                float v[V];
-                unpack_vec<T>(u, v);
-#pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    st.amax = fmaxf(st.amax, fabsf(v[e]));
-                    st.lo = fminf(st.lo, v[e]);
-                    st.hi = fmaxf(st.hi, v[e]);
+                    accumulate_stats<T, OP>(raw[i], st);
                 }
             }
         };
-        if (active) {
-            if (cached) {
-                // All loads first, so they are in flight together.
-#pragma unroll
-                for (int i = 0; i < MAXV; ++i) {
-                    const int64_t j = t + static_cast<int64_t>(i) * TPR;
-                    if (j < nvec) raw[i] = ld_stream16(src + j * V);
+        if (cached) {
+            if (full) pass1(std::true_type{}); else pass1(std::false_type{});
+        } else if (active) {
+            for (int64_t j = t; j < nvec; j += TPR) {
+                uint4 u = ld_stream16(src_row + j * V);
+                if constexpr (kSkip) {
+                    const uint2 kp = keep_of(j);
+                    u = zero_skipped16(u, make_uint2(~kp.x, ~kp.y));
                 }
-#pragma unroll
-                for (int i = 0; i < MAXV; ++i) {
-                    const int64_t j = t + static_cast<int64_t>(i) * TPR;
-                    if (j < nvec) accumulate(raw[i], j);
-                }
-            } else {
-                for (int64_t j = t; j < nvec; j += TPR) accumulate(ld_stream16(src + j * V), j);
+                accumulate_stats<T, OP>(u, st);
             }
         }
+        st.amax = fmaxf(st.hi, -st.lo);
         st = group_reduce<TPR, OP == kOpWeightAsym>(st, red);
+        if constexpr (OP != kOpWeightAsym) st.amax = fmaxf(st.amax, 0.0f);
 
-        float S = 1.f, Z = 0.f;
-        if constexpr (OP == kOpActInt8 || OP == kOpWeightSym) {
-            S = __fdiv_rn(st.amax, 127.0f);
-        } else if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
-            float amax = st.amax;
-            if (OP == kOpActFp8 && a.clip_ub > 0.f) amax = fminf(amax, a.clip_ub);
-            S = __fdiv_rn(amax, 448.0f);
-        } else {
-            S = __fdiv_rn(__fsub_rn(st.hi, st.lo), 255.0f);
-        }
-        if (!(S >= kEps)) S = kEps;
-        if constexpr (OP == kOpWeightAsym) {
-            Z = clampf(__fsub_rn(rintf(__fdiv_rn(-st.lo, S)), 128.0f), -128.0f, 127.0f);
-        }
+        const RowConsts c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias);
 
-        const float R = __frcp_rn(S);   // RN(1/S), shared by the row
+        // Pass 2: codes.  c.fast and `cached` are the same for the whole warp.
+        // Elements whose bracket ends disagree go to the warp's queue, which is
+        // drained (32 elements at a time, with exact divisions) whenever it is
+        // half full and at the end of the pass.
         int rsum = 0;
-        uint8_t* dst = static_cast<uint8_t*>(a.codes) + (active ? row : 0) * a.k;
-        // Pass 2: codes (see int_codes_sym / int_codes_asym / e4m3_codes).
-        auto quantize = [&](const uint4 u, int64_t j) {
-            float v[V];
-            unpack_vec<T>(u, v);
-            uint32_t words[V / 4];
-            if constexpr (OP == kOpActInt8 || OP == kOpWeightSym) {
-                int_codes_sym<T, V>(u, v, S, R, words);
-                if (use_skip) {
-                    // LLM.int8: outlier columns carry code 0 (mask bytes are 0 or 1,
-                    // so mask * 0xFF selects whole bytes).
-#pragma unroll
-                    for (int w = 0; w < V / 4; ++w)
-                        words[w] &= ~(*reinterpret_cast<const uint32_t*>(a.skip + j * V + 4 * w) * 0xFFu);
-                }
-                if constexpr (OP == kOpActInt8) {
-#pragma unroll
-                    for (int w = 0; w < V / 4; ++w) rsum = __dp4a(static_cast<int>(words[w]), 0x01010101, rsum);
-                }
-            } else if constexpr (OP == kOpWeightAsym) {
-                int_codes_asym<T, V>(u, v, S, R, Z, a.codes_u8 ? 128.0f : 0.0f, words);
-            } else {
-                e4m3_codes<T, V>(u, v, S, R, words);
-            }
+        __syncwarp();   // the previous row's queue is drained
+        if ((threadIdx.x & 31) == 0) q->n = 0;
+        __syncwarp();
+        auto drain = [&]() { rsum += drain_queue<OP>(q, dst_row, c.S, c.Z, c.bias); };
+        auto finish = [&](uint32_t w0, uint32_t w1, uint8_t* p) {
             if constexpr (V == 8) {
-                *reinterpret_cast<uint2*>(dst + j * V) = make_uint2(words[0], words[1]);
+                *reinterpret_cast<uint2*>(p) = make_uint2(w0, w1);
             } else {
-                *reinterpret_cast<uint32_t*>(dst + j * V) = words[0];
+                *reinterpret_cast<uint32_t*>(p) = w0;
+            }
+            if constexpr (kRowsum) {
+                rsum = __dp4a(static_cast<int>(w0), 0x01010101, rsum);
+                if constexpr (V == 8) rsum = __dp4a(static_cast<int>(w1), 0x01010101, rsum);
             }
         };
-        if (active) {
-            if (cached) {
+        auto pass2 = [&](auto full_tag) {
+            constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
-                for (int i = 0; i < MAXV; ++i) {
-                    const int64_t j = t + static_cast<int64_t>(i) * TPR;
-                    if (j < nvec) quantize(raw[i], j);
+            for (int i = 0; i < MAXV; ++i) {
+                if (FULL || i < nvmax) {   // uniform over the warp
+                    const bool valid = FULL || i < nv;
+                    const uint2 kp = valid ? keep_of(t + static_cast<int64_t>(i) * TPR) : make_uint2(~0u, ~0u);
+                    uint32_t words[2], d[2];
+                    fast_codes<T, OP>(raw[i], c, kp, words, d);   // zero vectors: d = 0
+                    if (valid) finish(words[0], words[1], dst + i * TPR * V);
+                    if (__any_sync(0xffffffffu, (d[0] | d[1]) != 0u)) {
+                        if ((d[0] | d[1]) != 0u)
+                            push_flagged<T>(raw[i], make_uint2(d[0], d[1]), make_uint2(words[0], words[1]),
+                                            (t + i * TPR) * V, q);
+                        __syncwarp();
+                        if (q->n >= kDrainAt) drain();
+                    }
                 }
-            } else {
-                for (int64_t j = t; j < nvec; j += TPR) quantize(ld_stream16(src + j * V), j);
+            }
+        };
+        const bool redo = !(cached && c.fast);
+        if (cached && c.fast) {
+            if (full) pass2(std::true_type{}); else pass2(std::false_type{});
+            drain();
+        }
+        if (active && redo) {
+            // Rows longer than the register cache (read again, from L2), rows
+            // the fast path does not cover (every code exact).
+            rsum = 0;
+            for (int64_t j = t; j < nvec; j += TPR) {
+                const uint4 u = ld_stream16(src_row + j * V);
+                const uint2 kp = keep_of(j);
+                uint32_t words[2] = {0u, 0u}, d[2] = {~0u, ~0u};
+                if (c.fast) fast_codes<T, OP>(u, c, kp, words, d);
+                if ((d[0] | d[1]) != 0u) {
+                    const uint2 e = exact_codes<T, OP>(u, c.S, c.Z, c.bias, make_uint2(d[0], d[1]),
+                                                       make_uint2(words[0], words[1]));
+                    words[0] = e.x & kp.x;
+                    words[1] = e.y & kp.y;
+                }
+                finish(words[0], words[1], dst_row + j * V);
             }
         }
-        if constexpr (OP == kOpActInt8) rsum = group_sum<TPR>(rsum, redi);
+        if constexpr (kRowsum) rsum = group_sum<TPR>(rsum, redi);
 
         if (active && t == 0) {
-            a.scale[row] = S;
-            if constexpr (OP == kOpActInt8) {
+            a.scale[row] = c.S;
+            if constexpr (kRowsum) {
                 if (a.rowsum) a.rowsum[row] = rsum;
             }
             if constexpr (OP == kOpWeightAsym) {
-                a.zero_point[row] = a.codes_u8 ? __fadd_rn(Z, 128.0f) : Z;
+                a.zero_point[row] = a.codes_u8 ? __fadd_rn(c.Z, 128.0f) : c.Z;
             }
             if constexpr (OP == kOpWeightSym) {
                 if (a.zero_point) a.zero_point[row] = 0.0f;
@@ -455,18 +581,14 @@ __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
         }
         // LLM.int8: gather the outlier columns of this row into fp16, zero-padded
         // to a multiple of 64 columns for the tensor-core outlier GEMM.
-        if constexpr (OP == kOpActInt8 && sizeof(T) == 2) {
+        if constexpr (kSkip) {
             if (active && a.x_outlier != nullptr) {
                 const int cnt = *a.outlier_count;
                 const int cpad = (cnt + 63) / 64 * 64;
                 __half* xo = a.x_outlier + row * a.ldo;
                 for (int j = t; j < cpad; j += TPR) {
                     __half h = __float2half_rn(0.0f);
-                    if (j < cnt) {
-                        const T x = src[a.outlier_idx[j]];
-                        if constexpr (std::is_same<T, __half>::value) h = x;
-                        else h = __float2half_rn(__bfloat162float(x));
-                    }
+                    if (j < cnt) h = src_row[a.outlier_idx[j]];
                     xo[j] = h;
                 }
             }
@@ -512,7 +634,12 @@ cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
 template <typename T>
 cudaError_t launch_rows_dtype(const RowQuantArgs& a, cudaStream_t s) {
     switch (a.op) {
-        case kOpActInt8: return launch_rows_t<T, kOpActInt8>(a, s);
+        case kOpActInt8:
+            if (a.skip != nullptr) {
+                if constexpr (std::is_same<T, __half>::value) return launch_rows_t<T, kOpActInt8Skip>(a, s);
+                return cudaErrorInvalidValue;   // the outlier path takes fp16 inputs only
+            }
+            return launch_rows_t<T, kOpActInt8>(a, s);
         case kOpActFp8: return launch_rows_t<T, kOpActFp8>(a, s);
         case kOpWeightAsym: return launch_rows_t<T, kOpWeightAsym>(a, s);
         case kOpWeightSym: return launch_rows_t<T, kOpWeightSym>(a, s);

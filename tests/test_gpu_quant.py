@@ -217,3 +217,30 @@ def test_quotient_rounding_at_exact_midpoints():
     Wa[:, 1] = 255.0            # S = 1 exactly, Z = -128
     Wa[:, 2:14] = torch.tensor([0.5, 1.5, 2.5, 100.5, 127.5, 128.5, 200.5, 254.5, 3.5, 4.5, 5.5, 6.5])
     _weight_check(Wa, P.host_f32(Wa), "asym", "s8", "asym integer midpoints")
+
+
+def test_ties_with_non_power_of_two_scale():
+    """absmax = 127 * 9/64 (fp16-exact) gives S = 9/64 exactly, so
+    x = (n + 1/2) * 9/128 lies exactly on a rounding midpoint of x / S.  Whole
+    16-byte vectors of such elements give a thread more boundary elements than
+    its queue holds, which sends it through the per-vector exact path; single
+    ones go through the queue."""
+    m, k = 6, 256
+    g = torch.Generator().manual_seed(41)
+    n = torch.randint(-100, 100, (m, k), generator=g).to(torch.float32)
+    X = ((2 * n + 1) * 9 / 128).to(torch.float16)
+    X[:, 0] = 127 * 9 / 64
+    X[3:, 1:] = (torch.randn(3, k - 1, generator=g) * 4).to(torch.float16)
+    X[3, 37] = 0.5 * 9 / 64                 # one midpoint among regular values
+    X[4, 200] = -2.5 * 9 / 64
+    _act_int8_check(X, P.host_f32(X), "int8 ties, S = 9/64")
+    # E4M3 midpoints times S = 63 / 448 = 9/64
+    mids = torch.tensor([1.0625, 3.125, 240.0, 432.0, -1.0625, -13.0, 1.1875, 0.0029296875])
+    Xf = (mids.repeat(m, k // 8) * 9 / 64).to(torch.float16)
+    Xf[:, 0] = 63.0
+    Xf[3:, 1:] = (torch.randn(3, k - 1, generator=g) * 4).to(torch.float16)
+    Xf[3, 9] = 3.125 * 9 / 64
+    _act_fp8_check(Xf, P.host_f32(Xf), 0.0, "e4m3 ties, S = 9/64")
+    W = Xf.clone()
+    _weight_check(W, P.host_f32(W), "fp8", "e4m3", "weight e4m3 ties")
+    _weight_check(X.clone(), P.host_f32(X), "sym", "s8", "weight sym ties")
