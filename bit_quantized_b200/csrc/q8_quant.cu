@@ -206,10 +206,16 @@ __device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, 
         c.S = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
     }
     if (!(c.S >= kEps)) c.S = kEps;
+    // 1/S rounded down and up: from R = RN(1/S) and the sign of the residual
+    // 1 - S R, which the FMA gives exactly (|1 - S R| <= 2^-24 fits in a float).
     // When S is a power of two, 1/S is exact and so is x * (1/S) = x / S (the
     // product keeps x's significand): no bracket is needed, except for
     // asymmetric codes with an odd Z + bias folded into the rounding constant.
-    const float rd = __frcp_rd(c.S), ru = __frcp_ru(c.S);
+    const float R = __frcp_rn(c.S);
+    const float res = __fmaf_rn(-c.S, R, 1.0f);
+    const uint32_t rb = __float_as_uint(R);
+    const float rd = res < 0.f ? __uint_as_float(rb - 1u) : R;   // R > 1/S: one ulp down
+    const float ru = res > 0.f ? __uint_as_float(rb + 1u) : R;   // R < 1/S: one ulp up
     const bool exact_rcp = rd == ru;
     if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
         // t = RN(x * r) adds one more rounding (2^-24) on top of the ends.
@@ -412,7 +418,7 @@ __device__ __forceinline__ void accumulate_stats(const uint4 u, RowStats& st) {
 // them stay in registers between the two passes (longer rows are read twice,
 // the second time from L2).
 template <typename T, int OP, int TPR, int MAXV>
-__global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
+__global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(RowQuantArgs a) {
     static_assert(TPR % 32 == 0, "a warp works on one row");
     constexpr int V = VecOf<T>::N;
     constexpr int RPB = kBlock / TPR;
@@ -421,6 +427,7 @@ __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
     __shared__ float red[3 * (kBlock / 32)];
     __shared__ int redi[kBlock / 32];
     __shared__ FixQueue fixq[kBlock / 32];
+    __shared__ float cshare[kBlock / TPR][8];
     FixQueue* q = &fixq[threadIdx.x / 32];
 
     const int g = threadIdx.x / TPR;
@@ -500,7 +507,23 @@ __global__ void __launch_bounds__(kBlock, 2) row_quant_kernel(RowQuantArgs a) {
         st = group_reduce<TPR, OP == kOpWeightAsym>(st, red);
         if constexpr (OP != kOpWeightAsym) st.amax = fmaxf(st.amax, 0.0f);
 
-        const RowConsts c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias);
+        RowConsts c;
+        if constexpr (TPR > 32) {
+            // One warp of the group works the row constants out for all.
+            float* cs = cshare[g];
+            if (t < 32) {
+                c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias);
+                if (t == 0) {
+                    cs[0] = c.S; cs[1] = c.Z; cs[2] = c.bias; cs[3] = c.rlo;
+                    cs[4] = c.rhi; cs[5] = c.add; cs[6] = c.fast ? 1.0f : 0.0f;
+                }
+            }
+            group_sync<TPR>();
+            c.S = cs[0]; c.Z = cs[1]; c.bias = cs[2]; c.rlo = cs[3];
+            c.rhi = cs[4]; c.add = cs[5]; c.fast = cs[6] != 0.0f;
+        } else {
+            c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias);
+        }
 
         // Pass 2: codes.  c.fast and `cached` are the same for the whole warp.
         // Elements whose bracket ends disagree go to the warp's queue, which is
@@ -600,9 +623,9 @@ template <typename T, int OP>
 cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
     constexpr int V = VecOf<T>::N;
     const int64_t nvec = a.k / V;
-    // Threads per row: enough that each thread holds at most 8 vectors.
-    auto go = [&](auto tpr_tag) -> cudaError_t {
+    auto go = [&](auto tpr_tag, auto maxv_tag) -> cudaError_t {
         constexpr int TPR = decltype(tpr_tag)::value;
+        constexpr int MAXV = decltype(maxv_tag)::value;
         constexpr int RPB = kBlock / TPR;
         int64_t blocks = (a.rows + RPB - 1) / RPB;
         if (blocks > 65535 * 4) blocks = 65535 * 4;
@@ -616,19 +639,39 @@ cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, row_quant_kernel<T, OP, TPR, kMaxVec>, a);
+        return cudaLaunchKernelEx(&cfg, row_quant_kernel<T, OP, TPR, MAXV>, a);
     };
+    using T128 = std::integral_constant<int, 128>;
+    using T256 = std::integral_constant<int, 256>;
+    using C2 = std::integral_constant<int, 2>;
+    using C4 = std::integral_constant<int, 4>;
+    using C16 = std::integral_constant<int, kMaxVec>;
     // Threads per row: enough to hold the row in registers (16 vectors a
     // thread), and, for short matrices, enough to spread the rows over the SMs;
     // otherwise as few as possible, so the per-row reductions (warp shuffles
     // for one warp) stay a small part of the work.
-    int64_t need = (nvec + kMaxVec - 1) / kMaxVec;
-    int64_t spread = (static_cast<int64_t>(kBlock) * 148 + a.rows - 1) / (a.rows > 0 ? a.rows : 1);
-    const int64_t tpr = need > spread ? need : spread;
-    if (tpr <= 32) return go(std::integral_constant<int, 32>{});
-    if (tpr <= 64) return go(std::integral_constant<int, 64>{});
-    if (tpr <= 128) return go(std::integral_constant<int, 128>{});
-    return go(std::integral_constant<int, 256>{});
+    const int64_t need = (nvec + kMaxVec - 1) / kMaxVec;
+    const int64_t spread = (static_cast<int64_t>(kBlock) * 148 + a.rows - 1) / (a.rows > 0 ? a.rows : 1);
+    int64_t tpr = need > spread ? need : spread;
+    tpr = tpr <= 32 ? 32 : tpr <= 64 ? 64 : tpr <= 128 ? 128 : 256;
+    // Matrices that take several waves of 16-vector rows run at 4 vectors a
+    // thread instead (rows of up to 1024 vectors): fewer registers, twice the
+    // resident warps, so loads of some rows overlap the arithmetic of others.
+    const int64_t warps16 = a.rows * (tpr / 32);
+    if (warps16 > 2 * 148 * (kBlock / 32) && nvec <= 256 * 4) {
+        if (nvec <= 128 * 4) return go(T128{}, C4{});
+        return go(T256{}, C4{});
+    }
+    // Rows spread over 128 or 256 threads hold a few vectors each: a kernel
+    // unrolled for just those keeps the code short, which matters when each
+    // SM runs it once (small batches: the instructions are fetched cold).
+    if (tpr == 256 && nvec <= 256 * 2) return go(T256{}, C2{});
+    if (tpr >= 128 && nvec <= 128 * 4) return go(T128{}, C4{});
+    if (tpr == 256 && nvec <= 256 * 4) return go(T256{}, C4{});
+    if (tpr == 32) return go(std::integral_constant<int, 32>{}, C16{});
+    if (tpr == 64) return go(std::integral_constant<int, 64>{}, C16{});
+    if (tpr == 128) return go(T128{}, C16{});
+    return go(T256{}, C16{});
 }
 
 template <typename T>
