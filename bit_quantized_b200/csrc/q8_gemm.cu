@@ -411,6 +411,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     __shared__ __align__(8) uint64_t drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_sh;
+    __shared__ float sx_sh[NT];       // token scales and row sums, loaded while the MMAs run
+    __shared__ int32_t rowsum_sh[NT];
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -419,6 +421,8 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     const int kb0 = static_cast<int>(rank) * kb_per_split;
     const int kb1 = min(num_kb, kb0 + kb_per_split);
     const int my_kb = kb1 > kb0 ? kb1 - kb0 : 0;
+    // Epilogue constants of this thread's output channel (epilogue warps).
+    float e_sw = 0.f, e_zw = 0.f, e_bias = 0.f;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nstages; ++s) {
@@ -524,6 +528,23 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         const int q = warp & 3;
         const int ch = q * 32 + lane;
         const int tpo = (NT + splits - 1) / splits;     // tokens owned per rank
+        // The dequant inputs go out now, not after the reduction: the weight
+        // scales and zero points do not depend on the previous kernel, the
+        // token scales and row sums (its outputs) are complete after the wait.
+        {
+            const int n = tn * kBM + ch;
+            if (n < p.n) {
+                e_sw = p.sw[n];
+                if (p.zw) e_zw = p.zw[n];
+                if (p.bias) e_bias = p.bias[n];
+            }
+            pdl_wait();
+            const int t = q * 32 + lane;
+            if (t < NT) {
+                sx_sh[t] = t < p.m ? p.sx[t] : 0.f;
+                rowsum_sh[t] = (t < p.m && p.zw) ? p.rowsum[t] : 0;
+            }
+        }
         bool have = my_kb > 0 && mbar_wait(&tfull_bar, 0, &abort_sh, p.status);
         if (have) tc_fence_after();
         __syncwarp();
@@ -551,7 +572,6 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
     cluster_sync();
 
     if (warp >= 2) {
-        pdl_wait();   // token scales and row sums come from the previous kernel
         // Rank r finishes the tokens t with t % splits == r, summing the
         // partials in rank order.
         const int q = warp & 3;
@@ -560,9 +580,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
         const int n = tn * kBM + ch;
         const bool has_zp = p.zw != nullptr;
         const bool col_ok = n < p.n;
-        const float sw = col_ok ? p.sw[n] : 0.f;
-        const float zw = (col_ok && has_zp) ? p.zw[n] : 0.f;
-        const float bias = (col_ok && p.bias) ? p.bias[n] : 0.f;
+        const float sw = e_sw, zw = e_zw, bias = e_bias;
         for (int t = static_cast<int>(rank); t < NT && t < p.m; t += splits) {
             const int tl = t / splits;
             uint32_t acc_bits;
@@ -572,13 +590,13 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
                 for (int r = 0; r < splits; ++r)
                     s = __fadd_rn(s, __uint_as_float(red[(r * tpo + tl) * kBM + ch]));
                 acc_bits = __float_as_uint(s);
-                v = __fmul_rn(__fmul_rn(s, p.sx[t]), sw);
+                v = __fmul_rn(__fmul_rn(s, sx_sh[t]), sw);
             } else {
                 int32_t s = 0;
                 for (int r = 0; r < splits; ++r)
                     s += static_cast<int32_t>(red[(r * tpo + tl) * kBM + ch]);
                 acc_bits = static_cast<uint32_t>(s);
-                v = dequant_int(s, zw, has_zp ? p.rowsum[t] : 0, p.sx[t], sw, has_zp);
+                v = dequant_int(s, zw, rowsum_sh[t], sx_sh[t], sw, has_zp);
             }
             if (p.bias) v = __fadd_rn(v, bias);
             if (col_ok) {

@@ -441,10 +441,10 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
     const float bias = (OP == kOpWeightAsym && a.codes_u8) ? 128.0f : 0.0f;
     // Launched with programmatic dependent launch: this grid may start while
     // the previous kernel runs, so it waits for it before touching memory.
-    // Activation quantizers then let the GEMM that follows start its prologue
-    // and weight loads (it waits for this grid before reading the codes).
-    // Weight quantizers do not: a GEMM right after one must not load the
-    // weight before it is fully written.
+    // Activation quantizers first let the GEMM that follows launch, so that
+    // its CTAs become resident and load their weights meanwhile (it waits for
+    // this grid before reading the codes).  Weight quantizers do not: a GEMM
+    // right after one must not load the weight before it is fully written.
     if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActFp8) pdl_launch_dependents();
     pdl_wait();
 
