@@ -26,11 +26,14 @@
 
 #include "q8_device.cuh"
 #include "q8_internal.h"
+#include "q8_qmath.cuh"
 
 namespace q8 {
 namespace {
 
-constexpr float kEps = 1e-8f;
+using qm::kEps;
+using qm::kFastLimit;
+using qm::kMagic;
 constexpr int kBlock = 256;
 constexpr int kMaxVec = 16;   // 16-byte vectors a thread keeps in registers
 
@@ -171,8 +174,6 @@ __device__ __forceinline__ float clampf(float v, float lo, float hi) {
 //   codes would need the [-128, 127] clamp, are coded exactly throughout
 //   (constant rows, rows that do not cross zero).
 //   E4M3 codes: t = RN(x * r) per end, then the hardware conversion.
-constexpr float kMagic = 12582912.0f;    // 1.5 * 2^23
-constexpr float kFastLimit = 2097152.0f; // 2^21: bound on |x * r| for the integer fast path
 
 // Internal op for the LLM.int8 regular stream: int8 activations with the
 // outlier columns (mask bytes of 1) left out of the absmax and coded as 0.
@@ -206,16 +207,11 @@ __device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, 
         c.S = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
     }
     if (!(c.S >= kEps)) c.S = kEps;
-    // 1/S rounded down and up: from R = RN(1/S) and the sign of the residual
-    // 1 - S R, which the FMA gives exactly (|1 - S R| <= 2^-24 fits in a float).
     // When S is a power of two, 1/S is exact and so is x * (1/S) = x / S (the
     // product keeps x's significand): no bracket is needed, except for
     // asymmetric codes with an odd Z + bias folded into the rounding constant.
-    const float R = __frcp_rn(c.S);
-    const float res = __fmaf_rn(-c.S, R, 1.0f);
-    const uint32_t rb = __float_as_uint(R);
-    const float rd = res < 0.f ? __uint_as_float(rb - 1u) : R;   // R > 1/S: one ulp down
-    const float ru = res > 0.f ? __uint_as_float(rb + 1u) : R;   // R < 1/S: one ulp up
+    float rd, ru;
+    qm::reciprocal_bounds(c.S, rd, ru);
     const bool exact_rcp = rd == ru;
     if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
         // t = RN(x * r) adds one more rounding (2^-24) on top of the ends.

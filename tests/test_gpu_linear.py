@@ -284,6 +284,8 @@ def _dynamic_vs_two_step(X, W, scheme, codes, wscheme, ub=0.0, bias=None, what="
     (64, 384, 4096, torch.bfloat16),
     (65, 256, 256, torch.bfloat16),     # tile kernel
     (8, 256, 512, torch.float32),       # fp32 input
+    (3, 208, 160, torch.bfloat16),      # ragged N and last K block
+    (12, 1008, 3008, torch.float16),    # fp16, 12 token rows
 ])
 @pytest.mark.parametrize("codes,wscheme", [("u8", "asym"), ("s8", "sym")])
 def test_dynamic_int8_matches_two_step(m, n, k, dtype, codes, wscheme):
