@@ -459,13 +459,20 @@ def load_profile_traffic(kernel_tag: str):
     return entry.get("dram_bytes_per_launch")
 
 
+# Sources the GEMM kernels are compiled from (a traffic entry stays valid
+# while these are unchanged).
+GEMM_SOURCES = ("q8_device.cuh", "q8_gemm.cu", "q8_internal.h")
+
+
 def source_hash() -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_quantized_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in GEMM_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
+    with open(os.path.join(ROOT, "include", "q8.h"), "rb") as fh:
+        h.update(b"q8.h" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -492,7 +499,9 @@ def extras(q8, dev, pk):
     out = {"int8_fp8_peak_tops": int8_peak,
            "peak_note": f"{pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s x 2 (nominal "
                         "dense INT8/FP8 : bf16 ratio 4.5 : 2.25)",
-           "hbm_peak_gbs": pk["hbm_gbs"]}
+           "hbm_peak_gbs": pk["hbm_gbs"],
+           "timing": "each figure: one launch between CUDA events right after an L2 flush (launch "
+                     "latency included; the graph-replayed step above is the sustained figure)"}
     for name in workloads.ORDER:
         w = workloads.WORKLOADS[name]
         X, W, _ = workloads.make_inputs(name)

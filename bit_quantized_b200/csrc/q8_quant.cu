@@ -529,7 +529,10 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
         __syncwarp();   // the previous row's queue is drained
         if ((threadIdx.x & 31) == 0) q->n = 0;
         __syncwarp();
-        auto drain = [&]() { rsum += drain_queue<OP>(q, dst_row, c.S, c.Z, c.bias); };
+        auto drain = [&]() {
+            __syncwarp();
+            if (q->n != 0) rsum += drain_queue<OP>(q, dst_row, c.S, c.Z, c.bias);   // uniform
+        };
         auto finish = [&](uint32_t w0, uint32_t w1, uint8_t* p) {
             if constexpr (V == 8) {
                 *reinterpret_cast<uint2*>(p) = make_uint2(w0, w1);
