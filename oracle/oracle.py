@@ -67,6 +67,8 @@ def lib():
             "or_quant_weight_fp8": [vp, i64, i64, vp, vp],
             "or_quant_act_int8": [vp, i64, i64, vp, vp, vp, vp],
             "or_quant_act_fp8": [vp, i64, i64, f, vp, vp],
+            "or_quant_act_static": [vp, i64, i64, f, vp, vp, vp],
+            "or_requant": [vp, i64, f, vp],
             "or_outlier_columns": [vp, i64, i64, f, vp, vp, vp],
             "or_gemm_int": [vp, i32, i64, vp, i32, i64, i64, vp, i64, vp, i64, vp],
             "or_epilogue_int": [vp, vp, i64, vp, i64, vp, vp, vp, vp, vp, vp],
@@ -174,6 +176,25 @@ def quant_act_int8(x: np.ndarray, skip: Optional[np.ndarray] = None):
     sk = None if skip is None else np.ascontiguousarray(skip, dtype=np.uint8)
     lib().or_quant_act_int8(_ptr(x), m, k, _ptr(sk), _ptr(q), _ptr(S), _ptr(rs))
     return q, S, rs
+
+
+def quant_act_static(x: np.ndarray, S: float):
+    """Static per-tensor symmetric INT8: (codes, per-row scale copies, row sums)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    m, k = x.shape
+    q = np.empty((m, k), np.int8)
+    Sr = np.empty(m, np.float32)
+    rs = np.empty(m, np.int32)
+    lib().or_quant_act_static(_ptr(x), m, k, float(np.float32(S)), _ptr(q), _ptr(Sr), _ptr(rs))
+    return q, Sr, rs
+
+
+def requant(y: np.ndarray, S: float) -> np.ndarray:
+    """INT8 codes of a layer's fp32 output with the next layer's input scale."""
+    y = np.ascontiguousarray(y, dtype=np.float32)
+    q = np.empty(y.shape, np.int8)
+    lib().or_requant(_ptr(y), y.size, float(np.float32(S)), _ptr(q))
+    return q
 
 
 def quant_act_fp8(x: np.ndarray, ub: float):

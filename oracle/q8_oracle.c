@@ -318,6 +318,50 @@ void or_quant_act_int8(const float *X, int64_t m, int64_t k, const uint8_t *skip
 }
 
 /*
+ * Static (calibrated) symmetric INT8 quantization with one scale for the
+ * whole tensor ("大模型量化" (Xilyfe), the paragraph on 静态量化: the scale is
+ * worked out once from a calibration pass and reused on every call instead of
+ * being recomputed from each input).  Reading: symmetric, per-tensor, the
+ * caller passes S > 0; q = clamp(rne(fl32(x / S)), -127, 127), so inputs
+ * beyond 127 S saturate, as the code range of every other quantizer here.
+ * S is copied to every row's scale so the result feeds the W8A8 linear like
+ * a dynamic activation; rowsum[r] = sum of the row's codes (for asymmetric
+ * weights).
+ */
+static int8_t static_code(float x, float S) {
+    const float t = x / S;
+    return (int8_t)clampd(rne((double)t), -127.0, 127.0);
+}
+
+void or_quant_act_static(const float *X, int64_t m, int64_t k, float S, int8_t *q, float *Sout,
+                         int32_t *rowsum) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < m; ++r) {
+        int64_t sum = 0;
+        for (int64_t j = 0; j < k; ++j) {
+            const int8_t c = static_code(X[r * k + j], S);
+            q[r * k + j] = c;
+            sum += c;
+        }
+        Sout[r] = S;
+        if (rowsum) rowsum[r] = (int32_t)sum;
+    }
+}
+
+/*
+ * Re-quantization of a layer's output for the next layer ("大模型量化"
+ * (Xilyfe), 量化对象 section, INT8 这么小的范围不会导致溢出吗: after the INT32
+ * accumulation the result is scaled back into INT8 before it is passed on).
+ * Reading: the fp32 output y of the dequant epilogue (bias included) is
+ * quantized with the next layer's static input scale S_out:
+ * q = clamp(rne(fl32(y / S_out)), -127, 127).
+ */
+void or_requant(const float *y, int64_t count, float S, int8_t *q) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i) q[i] = static_code(y[i], S);
+}
+
+/*
  * Dynamic per-token FP8 E4M3 with an upper bound on the row scale
  * ([FBGEMM] 5.2 and 6: quantize_fp8_per_row clips the input at
  * activation_scale_ub, default 1200.0).  alpha = min(max|x|, ub) when ub > 0;
