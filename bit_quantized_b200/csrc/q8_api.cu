@@ -3,6 +3,7 @@
 // memory or synchronizes, except q8_get_device_status.
 #include <cuda_runtime.h>
 
+#include <cfloat>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -200,6 +201,25 @@ q8_status q8_quantize_act(const void* X, q8_dtype x_dtype, int64_t m, int64_t k,
     return launch_status(launch_row_quant(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+q8_status q8_quantize_act_static(const void* X, q8_dtype x_dtype, int64_t m, int64_t k, int64_t ldx,
+                                 float static_scale, void* codes, float* scale, int32_t* rowsum,
+                                 q8_stream_t stream) {
+    if (m < 0 || k <= 0 || m > kMaxDim || k > kMaxDim || k % 32 != 0 || ldx < k) return Q8_ERR_SHAPE;
+    if (!float_input(x_dtype)) return Q8_ERR_DTYPE;
+    if (!(static_scale > 0.0f) || !(static_scale <= FLT_MAX)) return Q8_ERR_SCHEME;
+    if (m == 0) return Q8_OK;   // empty call
+    if (!X || !codes || !scale) return Q8_ERR_NULL;
+    if (!aligned16(X) || !aligned16(codes) || !ld_ok(ldx, k, x_dtype)) return Q8_ERR_ALIGN;
+    q8_status st = check_device();
+    if (st != Q8_OK) return st;
+    RowQuantArgs a = {};
+    a.src = X; a.src_dtype = x_dtype; a.rows = m; a.k = k; a.ld = ldx;
+    a.op = kOpActInt8Static;
+    a.static_scale = static_scale;
+    a.codes = codes; a.scale = scale; a.rowsum = rowsum;
+    return launch_status(launch_row_quant(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 static q8_status validate_outlier_act(const void* X, q8_dtype x_dtype, int64_t m, int64_t k,
                                       int64_t ldx, void* codes, float* scale, int32_t* rowsum,
                                       uint8_t* mask, int32_t* idx, int32_t* count,
@@ -274,6 +294,37 @@ q8_status q8_linear_w8a8(const q8_act* x, const q8_weight* w, const float* bias,
     a.sw = w->scale; a.zw = fp8 ? nullptr : w->zero_point;
     a.bias = bias;
     a.y = static_cast<__nv_bfloat16*>(Y); a.ldy = ldy;
+    a.acc_debug = acc_debug;
+    return launch_linear(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+q8_status q8_linear_w8a8_requant(const q8_act* x, const q8_weight* w, const float* bias,
+                                 float out_scale, void* Yq, int64_t ldy, void* acc_debug,
+                                 q8_stream_t stream) {
+    q8_status st = check_weight(w);
+    if (st != Q8_OK) return st;
+    if (!x) return Q8_ERR_NULL;
+    if (x->m < 0 || x->m > kMaxDim || x->k != w->k || x->ld < x->k || ldy < w->n) return Q8_ERR_SHAPE;
+    if (x->code_dtype != Q8_S8 || w->code_dtype == Q8_E4M3) return Q8_ERR_DTYPE;
+    if (w->k > kMaxKInt8) return Q8_ERR_SHAPE;
+    if (!(out_scale > 0.0f) || !(out_scale <= FLT_MAX)) return Q8_ERR_SCHEME;
+    if (x->m == 0 || w->n == 0) return Q8_OK;   // empty call
+    if (!x->codes || !x->scale || !Yq) return Q8_ERR_NULL;
+    if (w->zero_point && !x->rowsum) return Q8_ERR_NULL;
+    if (!aligned16(x->codes) || !aligned16(x->scale) || x->ld % 16 != 0 || !aligned16(Yq) ||
+        ldy % 16 != 0 || (bias && !aligned16(bias)) || (acc_debug && !aligned16(acc_debug)))
+        return Q8_ERR_ALIGN;
+    st = check_device();
+    if (st != Q8_OK) return st;
+    LinearArgs a = {};
+    a.m = x->m; a.n = w->n; a.k = w->k;
+    a.a_codes = x->codes; a.lda = x->ld;
+    a.b_codes = w->codes; a.ldb = w->ld;
+    a.kind = w->code_dtype == Q8_U8 ? 1 : 0;
+    a.sx = x->scale; a.rowsum = x->rowsum;
+    a.sw = w->scale; a.zw = w->zero_point;
+    a.bias = bias;
+    a.yq = static_cast<int8_t*>(Yq); a.out_scale = out_scale; a.ldy = ldy;
     a.acc_debug = acc_debug;
     return launch_linear(a, reinterpret_cast<cudaStream_t>(stream));
 }

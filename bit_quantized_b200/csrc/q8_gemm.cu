@@ -62,6 +62,8 @@ struct EpiParams {
     const float* bias;
     __nv_bfloat16* y;
     int64_t ldy;
+    int8_t* yq;         // non-null: int8 output codes, clamp(rne(fl32(y / out_scale)), +-127)
+    float out_scale;
     void* acc_debug;
     float* y16_debug;
     const int32_t* outlier_count;
@@ -104,6 +106,14 @@ __device__ __forceinline__ float dequant_int(int32_t acc, float zw, int32_t rs, 
     float v = __ll2float_rn(c);
     v = __fmul_rn(v, sx);
     return __fmul_rn(v, sw);
+}
+
+// Re-quantized output code ("大模型量化" (Xilyfe), 量化对象 section: the INT32
+// result is scaled back to INT8 before the next layer): the fp32 output y
+// with the next layer's static scale S, clamp(rne(fl32(y / S)), -127, 127).
+__device__ __forceinline__ uint32_t requant_code(float y, float S) {
+    return static_cast<uint32_t>(static_cast<int>(fminf(fmaxf(rintf(__fdiv_rn(y, S)), -127.0f), 127.0f))) &
+           0xFFu;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -331,14 +341,26 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         out[i] = v;
                     }
                 }
-                uint4* yp = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(row) * p.ldy + n0);
+                if (p.yq) {
+                    uint32_t w[8];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (8 * j >= nv) break;
-                    yp[j] = make_uint4(pack_bf16(out[8 * j], out[8 * j + 1]),
-                                       pack_bf16(out[8 * j + 2], out[8 * j + 3]),
-                                       pack_bf16(out[8 * j + 4], out[8 * j + 5]),
-                                       pack_bf16(out[8 * j + 6], out[8 * j + 7]));
+                    for (int j = 0; j < 8; ++j)
+                        w[j] = requant_code(out[4 * j], p.out_scale) | (requant_code(out[4 * j + 1], p.out_scale) << 8) |
+                               (requant_code(out[4 * j + 2], p.out_scale) << 16) |
+                               (requant_code(out[4 * j + 3], p.out_scale) << 24);
+                    uint4* qp = reinterpret_cast<uint4*>(p.yq + static_cast<int64_t>(row) * p.ldy + n0);
+                    qp[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    if (nv > 16) qp[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                } else {
+                    uint4* yp = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(row) * p.ldy + n0);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        if (8 * j >= nv) break;
+                        yp[j] = make_uint4(pack_bf16(out[8 * j], out[8 * j + 1]),
+                                           pack_bf16(out[8 * j + 2], out[8 * j + 3]),
+                                           pack_bf16(out[8 * j + 4], out[8 * j + 5]),
+                                           pack_bf16(out[8 * j + 6], out[8 * j + 7]));
+                    }
                 }
                 if (p.acc_debug) {
                     uint4* ap = reinterpret_cast<uint4*>(static_cast<uint32_t*>(p.acc_debug) +
@@ -600,7 +622,10 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
             }
             if (p.bias) v = __fadd_rn(v, bias);
             if (col_ok) {
-                p.y[static_cast<int64_t>(t) * p.ldy + n] = __float2bfloat16_rn(v);
+                if (p.yq)
+                    p.yq[static_cast<int64_t>(t) * p.ldy + n] = static_cast<int8_t>(requant_code(v, p.out_scale));
+                else
+                    p.y[static_cast<int64_t>(t) * p.ldy + n] = __float2bfloat16_rn(v);
                 if (p.acc_debug)
                     static_cast<uint32_t*>(p.acc_debug)[static_cast<int64_t>(t) * p.n + n] = acc_bits;
             }
@@ -788,6 +813,8 @@ q8_status launch_linear(const LinearArgs& a, cudaStream_t s) {
     ep.bias = a.bias;
     ep.y = a.y;
     ep.ldy = a.ldy;
+    ep.yq = a.yq;
+    ep.out_scale = a.out_scale;
     ep.acc_debug = a.acc_debug;
     ep.y16_debug = a.y16_debug;
     ep.outlier_count = a.outlier_count;

@@ -14,7 +14,8 @@ namespace q8 {
 int* device_status_ptr();
 
 // ---- quantize kernels (q8_quant.cu)
-enum RowOp { kOpActInt8 = 0, kOpActFp8 = 1, kOpWeightAsym = 2, kOpWeightSym = 3, kOpWeightFp8 = 4 };
+enum RowOp { kOpActInt8 = 0, kOpActFp8 = 1, kOpWeightAsym = 2, kOpWeightSym = 3, kOpWeightFp8 = 4,
+             kOpActInt8Static = 6 };
 
 struct RowQuantArgs {
     const void* src;       // rows x k input (f16 / bf16 / f32)
@@ -23,6 +24,7 @@ struct RowQuantArgs {
     int op;                // RowOp
     bool codes_u8;         // asymmetric weights stored as uint8 (q + 128)
     float clip_ub;         // fp8 activations: > 0 clips the row absmax
+    float static_scale;    // kOpActInt8Static: the calibrated scale (> 0)
     const uint8_t* skip;   // [k] columns left out (LLM.int8 outliers); may be null
     void* codes;           // rows x k, row stride k
     float* scale;          // [rows]
@@ -61,6 +63,7 @@ struct LinearArgs {
     const float* zw;                       // null: no zero point
     const float* bias;
     __nv_bfloat16* y;  int64_t ldy;
+    int8_t* yq;  float out_scale;          // non-null yq: int8 output codes (requantized), y unused
     void* acc_debug;                       // m x n (row stride n), or null
     // LLM.int8 outlier stream (all null for plain W8A8)
     const __half* xo; int64_t ldxo;        // m x ldxo fp16 gathered outlier columns

@@ -194,11 +194,14 @@ struct RowConsts {
 };
 
 template <int OP>
-__device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, float clip_ub, float bias) {
+__device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, float clip_ub, float bias,
+                                                float static_scale) {
     RowConsts c;
     c.Z = 0.f;
     c.bias = bias;
-    if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpWeightSym) {
+    if constexpr (OP == kOpActInt8Static) {
+        c.S = static_scale;   // calibrated, > 0 (checked by the caller)
+    } else if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpWeightSym) {
         c.S = __fdiv_rn(amax, 127.0f);
     } else if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
         if (OP == kOpActFp8 && clip_ub > 0.f) amax = fminf(amax, clip_ub);
@@ -206,7 +209,7 @@ __device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, 
     } else {
         c.S = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
     }
-    if (!(c.S >= kEps)) c.S = kEps;
+    if (OP != kOpActInt8Static && !(c.S >= kEps)) c.S = kEps;
     // When S is a power of two, 1/S is exact and so is x * (1/S) = x / S (the
     // product keeps x's significand): no bracket is needed, except for
     // asymmetric codes with an odd Z + bias folded into the rounding constant.
@@ -231,6 +234,12 @@ __device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, 
             const float qhi = __fadd_rn(rintf(__fdiv_rn(hi, c.S)), c.Z);
             c.fast = fmaxf(fabsf(lo), fabsf(hi)) * c.rhi <= kFastLimit && qlo >= -128.0f && qhi <= 127.0f;
             if (exact_rcp && (static_cast<int>(c.Z + bias) & 1) == 0) c.rlo = c.rhi = rd;
+        } else if constexpr (OP == kOpActInt8Static) {
+            // Codes of a static scale may saturate: the fast path (which does
+            // not clamp) needs every |fl32(x / S)| below 127.5, which
+            // absmax * rhi < 127.5 guarantees; other rows are coded exactly.
+            c.fast = amax * c.rhi < 127.5f;
+            if (exact_rcp) c.rlo = c.rhi = rd;
         } else {
             c.fast = amax * c.rhi <= kFastLimit;
             if (exact_rcp) c.rlo = c.rhi = rd;
@@ -419,7 +428,7 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
     constexpr int V = VecOf<T>::N;
     constexpr int RPB = kBlock / TPR;
     constexpr bool kSkip = OP == kOpActInt8Skip;
-    constexpr bool kRowsum = OP == kOpActInt8 || OP == kOpActInt8Skip;
+    constexpr bool kRowsum = OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActInt8Static;
     __shared__ float red[3 * (kBlock / 32)];
     __shared__ int redi[kBlock / 32];
     __shared__ FixQueue fixq[kBlock / 32];
@@ -441,7 +450,8 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
     // its CTAs become resident and load their weights meanwhile (it waits for
     // this grid before reading the codes).  Weight quantizers do not: a GEMM
     // right after one must not load the weight before it is fully written.
-    if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActFp8) pdl_launch_dependents();
+    if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActFp8 || OP == kOpActInt8Static)
+        pdl_launch_dependents();
     pdl_wait();
 
     for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * RPB; row0 < a.rows;
@@ -508,7 +518,7 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
             // One warp of the group works the row constants out for all.
             float* cs = cshare[g];
             if (t < 32) {
-                c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias);
+                c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias, a.static_scale);
                 if (t == 0) {
                     cs[0] = c.S; cs[1] = c.Z; cs[2] = c.bias; cs[3] = c.rlo;
                     cs[4] = c.rhi; cs[5] = c.add; cs[6] = c.fast ? 1.0f : 0.0f;
@@ -518,7 +528,7 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
             c.S = cs[0]; c.Z = cs[1]; c.bias = cs[2]; c.rlo = cs[3];
             c.rhi = cs[4]; c.add = cs[5]; c.fast = cs[6] != 0.0f;
         } else {
-            c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias);
+            c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias, a.static_scale);
         }
 
         // Pass 2: codes.  c.fast and `cached` are the same for the whole warp.
@@ -683,6 +693,7 @@ cudaError_t launch_rows_dtype(const RowQuantArgs& a, cudaStream_t s) {
             }
             return launch_rows_t<T, kOpActInt8>(a, s);
         case kOpActFp8: return launch_rows_t<T, kOpActFp8>(a, s);
+        case kOpActInt8Static: return launch_rows_t<T, kOpActInt8Static>(a, s);
         case kOpWeightAsym: return launch_rows_t<T, kOpWeightAsym>(a, s);
         case kOpWeightSym: return launch_rows_t<T, kOpWeightSym>(a, s);
         case kOpWeightFp8: return launch_rows_t<T, kOpWeightFp8>(a, s);

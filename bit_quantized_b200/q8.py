@@ -36,8 +36,9 @@ Q8_OP_LINEAR_W8A8, Q8_OP_LINEAR_INT8_MIXED = 0, 1
 Q8_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 EXPORTED = [
-    "q8_quantize_weight", "q8_dequantize_weight", "q8_quantize_act", "q8_outlier_quantize_act",
-    "q8_linear_w8a8", "q8_linear_w8a8_dynamic", "q8_linear_int8_mixed",
+    "q8_quantize_weight", "q8_dequantize_weight", "q8_quantize_act", "q8_quantize_act_static",
+    "q8_outlier_quantize_act",
+    "q8_linear_w8a8", "q8_linear_w8a8_requant", "q8_linear_w8a8_dynamic", "q8_linear_int8_mixed",
     "q8_linear_int8_mixed_noalloc",
     "q8_workspace_size", "q8_status_string",
     "q8_get_device_status", "q8_clear_device_status", "q8_device_check", "q8_version",
@@ -61,10 +62,13 @@ _SIG = {
     "q8_quantize_weight": ([_vp, _int, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp], _int),
     "q8_dequantize_weight": ([ctypes.POINTER(CWeight), _int, _vp, _vp], _int),
     "q8_quantize_act": ([_vp, _int, _i64, _i64, _i64, _int, _f, _vp, _vp, _vp, _vp], _int),
+    "q8_quantize_act_static": ([_vp, _int, _i64, _i64, _i64, _f, _vp, _vp, _vp, _vp], _int),
     "q8_outlier_quantize_act": ([_vp, _int, _i64, _i64, _i64, _f, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _vp, _i64, _vp], _int),
     "q8_linear_w8a8": ([ctypes.POINTER(CAct), ctypes.POINTER(CWeight), _vp, _vp, _i64, _vp, _vp,
                         _sz, _vp], _int),
+    "q8_linear_w8a8_requant": ([ctypes.POINTER(CAct), ctypes.POINTER(CWeight), _vp, _f, _vp, _i64,
+                                _vp, _vp], _int),
     "q8_linear_w8a8_dynamic": ([_vp, _int, _i64, _i64, _i64, _int, _f, ctypes.POINTER(CWeight),
                                 _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp], _int),
     "q8_linear_int8_mixed": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeight), _vp, _f, _vp,
@@ -218,6 +222,21 @@ def q8_quantize_act(X: torch.Tensor, scheme: str = "int8", clip_ub: float = 0.0,
     return out
 
 
+def q8_quantize_act_static(X: torch.Tensor, scale: float, out: Optional[QAct] = None,
+                           stream=None) -> QAct:
+    """Static INT8 quantization with a calibrated per-tensor scale (row sums included)."""
+    _cuda(X, "X")
+    m, k = X.shape
+    if out is None:
+        out = QAct(torch.empty((m, k), dtype=torch.int8, device=X.device),
+                   torch.empty(m, dtype=torch.float32, device=X.device),
+                   torch.empty(m, dtype=torch.int32, device=X.device), Q8_S8)
+    _check(_lib.q8_quantize_act_static(_ptr(X), _FLOAT_DT[X.dtype], m, k, X.stride(0), float(scale),
+                                       _ptr(out.codes), _ptr(out.scale), _ptr(out.rowsum),
+                                       _stream(stream)), "q8_quantize_act_static")
+    return out
+
+
 def q8_outlier_quantize_act(X: torch.Tensor, threshold: float = 6.0, gather: bool = True,
                             stream=None) -> dict:
     """LLM.int8 outlier columns + regular-stream INT8 quantization."""
@@ -252,6 +271,20 @@ def q8_linear_w8a8(x: QAct, w: QWeight, bias: Optional[torch.Tensor] = None,
     _check(_lib.q8_linear_w8a8(ctypes.byref(cx), ctypes.byref(cw), _ptr(bias), _ptr(out),
                                out.stride(0), _ptr(acc_debug), None, 0, _stream(stream)),
            "q8_linear_w8a8")
+    return out
+
+
+def q8_linear_w8a8_requant(x: QAct, w: QWeight, out_scale: float, bias: Optional[torch.Tensor] = None,
+                           out: Optional[torch.Tensor] = None, acc_debug: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """INT8 W8A8 linear with the output re-quantized to int8 codes (scale out_scale)."""
+    m, n = x.codes.shape[0], w.codes.shape[0]
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.int8, device=x.codes.device)
+    cx, cw = x.c(), w.c()
+    _check(_lib.q8_linear_w8a8_requant(ctypes.byref(cx), ctypes.byref(cw), _ptr(bias), float(out_scale),
+                                       _ptr(out), out.stride(0), _ptr(acc_debug), _stream(stream)),
+           "q8_linear_w8a8_requant")
     return out
 
 

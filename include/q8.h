@@ -169,6 +169,22 @@ q8_status q8_quantize_act(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
                           float *scale, int32_t *rowsum, q8_stream_t stream);
 
 /*
+ * Static activation quantization with a calibrated per-tensor scale: the scale
+ * is computed once, offline, from a calibration pass and applied to every call
+ * ([Xilyfe] the paragraph on static quantization, 静态量化).  Symmetric INT8,
+ * q = clamp(rne(fl32(x / static_scale)), -127, 127): inputs beyond
+ * 127 * static_scale saturate.  The output is a q8_act like the dynamic one.
+ *   X             device, m x k, Q8_F16 / Q8_BF16 / Q8_F32, row stride ldx.
+ *   static_scale  > 0 and finite, else Q8_ERR_SCHEME.
+ *   codes         device, m x k int8 output, row stride k.
+ *   scale         device [m] output, every entry static_scale.
+ *   rowsum        device [m] int32 output, sum_k q (may be NULL).
+ */
+q8_status q8_quantize_act_static(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
+                                 int64_t ldx, float static_scale, void *codes, float *scale,
+                                 int32_t *rowsum, q8_stream_t stream);
+
+/*
  * LLM.int8 outlier detection fused with the regular stream's quantization
  * ([LLM.int8] 核心思想 and BitsAndBytesConfig: llm_int8_threshold = 6.0).
  * A feature column k is an outlier when some token has |X[m, k]| > threshold
@@ -228,6 +244,23 @@ q8_status q8_outlier_quantize_act(const void *X, q8_dtype x_dtype, int64_t m, in
 q8_status q8_linear_w8a8(const q8_act *x, const q8_weight *w, const float *bias, void *Y,
                          int64_t ldy, void *acc_debug, void *workspace, size_t ws_bytes,
                          q8_stream_t stream);
+
+/*
+ * INT8 W8A8 linear whose output is re-quantized to INT8 codes for the next
+ * layer instead of written as bf16 ([Xilyfe] 量化对象 section: after the INT32
+ * accumulation the result is scaled back into INT8 before it is passed on).
+ * y is the fp32 value q8_linear_w8a8 would round to bf16 (dequant epilogue and
+ * bias); the output is clamp(rne(fl32(y / out_scale)), -127, 127), with
+ * out_scale the next layer's static input scale.
+ *   x, w, bias   as q8_linear_w8a8, INT8 codes only (Q8_ERR_DTYPE for E4M3).
+ *   out_scale    > 0 and finite, else Q8_ERR_SCHEME.
+ *   Yq           device, m x w->n int8 output, row stride ldy (ldy % 16 == 0).
+ *   acc_debug    as q8_linear_w8a8.
+ * The launch-overlap rule of q8_linear_w8a8 applies.
+ */
+q8_status q8_linear_w8a8_requant(const q8_act *x, const q8_weight *w, const float *bias,
+                                 float out_scale, void *Yq, int64_t ldy, void *acc_debug,
+                                 q8_stream_t stream);
 
 /*
  * Dynamic per-token activation quantization and the W8A8 linear in one call:

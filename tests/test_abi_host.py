@@ -186,3 +186,41 @@ def test_device_calls_report_no_device():
     assert q8.q8_device_check() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH, q8.Q8_OK)
     v = ctypes.c_int32(0)
     assert L.q8_get_device_status(None, _ns) == q8.Q8_ERR_NULL
+
+
+def rq(x=None, w=None, Y=FAKE, ldy=64, out_scale=0.05):
+    x = x or _act()
+    w = w or _weight()
+    return L.q8_linear_w8a8_requant(ctypes.byref(x), ctypes.byref(w), None, out_scale, Y, ldy, None, _ns)
+
+
+def test_linear_w8a8_requant_validation():
+    assert rq(Y=None) == q8.Q8_ERR_NULL
+    assert rq(x=_act(rowsum=None)) == q8.Q8_ERR_NULL           # zero point needs row sums
+    assert rq(ldy=32) == q8.Q8_ERR_SHAPE
+    assert rq(x=_act(code_dtype=q8.Q8_E4M3)) == q8.Q8_ERR_DTYPE   # INT8 codes only
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        assert rq(out_scale=bad) == q8.Q8_ERR_SCHEME
+    assert rq(ldy=72) == q8.Q8_ERR_ALIGN                        # int8 rows: ldy % 16
+    assert rq(Y=MIS) == q8.Q8_ERR_ALIGN
+    assert rq(x=_act(m=0)) == q8.Q8_OK                          # empty call
+    if NO_GPU:
+        assert rq() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def qs(X=FAKE, m=16, k=128, ldx=128, scale=0.02, codes=FAKE, sc=FAKE, rs=FAKE, dt=q8.Q8_BF16):
+    return L.q8_quantize_act_static(X, dt, m, k, ldx, scale, codes, sc, rs, _ns)
+
+
+def test_quantize_act_static_validation():
+    assert qs(X=None) == q8.Q8_ERR_NULL
+    assert qs(sc=None) == q8.Q8_ERR_NULL
+    assert qs(k=100, ldx=100) == q8.Q8_ERR_SHAPE                 # K % 32
+    assert qs(ldx=64) == q8.Q8_ERR_SHAPE
+    assert qs(dt=q8.Q8_S8) == q8.Q8_ERR_DTYPE
+    for bad in (0.0, -0.5, float("inf"), float("nan")):
+        assert qs(scale=bad) == q8.Q8_ERR_SCHEME
+    assert qs(X=MIS) == q8.Q8_ERR_ALIGN
+    assert qs(m=0, X=None, codes=None, sc=None) == q8.Q8_OK     # empty call
+    if NO_GPU:
+        assert qs(rs=None) in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
