@@ -539,6 +539,19 @@ def extras(q8, dev, pk):
                 t_w = _time_kernel(lambda: q8.q8_quantize_weight(Wd, w.weight_scheme, w.weight_codes), flush, reps=5)
                 r["weight_quant_us"] = round(t_w * 1e3, 1)
                 r["weight_quant_gbs"] = round(wq_bytes / (t_w * 1e-3) / 1e9, 1)
+            if w.kind == "w8a8_int8":
+                # Static scales (calibrated once; here 1.1 x the batch absmax / 127) and the
+                # linear that re-quantizes its output to INT8 for the next layer.
+                S = float(1.1 * float(Xd.float().abs().max()) / 127)
+                qs = q8.q8_quantize_act_static(Xd, S)
+                t_s = _time_kernel(lambda: q8.q8_quantize_act_static(Xd, S, out=qs), flush)
+                r["static_act_quant_us"] = round(t_s * 1e3, 2)
+                r["static_act_quant_gbs"] = round(act_bytes / (t_s * 1e-3) / 1e9, 1)
+                So = float(1.2 * float(q8.q8_linear_w8a8(qs, qw).float().abs().max()) / 127)
+                Yq = torch.empty((w.m, w.n), dtype=torch.int8, device=dev)
+                t_r = _time_kernel(lambda: q8.q8_linear_w8a8_requant(qs, qw, So, out=Yq), flush)
+                r["requant_gemm_us"] = round(t_r * 1e3, 2)
+                r["requant_gemm_tops"] = round(2.0 * w.m * w.n * w.k / (t_r * 1e-3) / 1e12, 1)
         out[name] = r
         del Xd, Wd
     torch.cuda.synchronize()
