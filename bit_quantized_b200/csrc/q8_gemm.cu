@@ -42,6 +42,7 @@
 
 #include "q8_device.cuh"
 #include "q8_internal.h"
+#include "q8_qmath.cuh"
 
 namespace q8 {
 namespace {
@@ -116,6 +117,60 @@ __device__ __forceinline__ uint32_t requant_code(float y, float S) {
            0xFFu;
 }
 
+// The same code without a division per output: the bracket of the
+// quantizers, 1/S rounded down and up and widened by (1 -+ 2^-23), so that
+// y * rlo and y * rhi enclose fl32(y / S).  Where both ends round to the same
+// integer (RN(y r + 1.5 * 2^23), exact product) that is the code; outputs whose
+// bracket lies beyond 127.5 saturate; the rest (near a rounding boundary) take
+// the division.
+struct Requant {
+    float S, rlo, rhi;
+};
+
+__device__ __forceinline__ Requant requant_consts(float S) {
+    Requant c;
+    c.S = S;
+    float rd, ru;
+    qm::reciprocal_bounds(S, rd, ru);
+    const bool exact = rd == ru;   // S a power of two: y * (1/S) = y / S exactly
+    c.rlo = exact ? rd : __fmul_rd(rd, 1.0f - 0x1p-23f);
+    c.rhi = exact ? ru : __fmul_ru(ru, 1.0f + 0x1p-23f);
+    return c;
+}
+
+// Out of line: the unrolled epilogue stays short (it shares the instruction
+// cache with the MMA warp's loop).
+__device__ __noinline__ uint32_t requant_code_slow(float y, float S) { return requant_code(y, S); }
+
+// Branch-free codes of 4 outputs: both ends of the bracket rounded with
+// RN(y r + 1.5 * 2^23) and clamped to the code range in that domain (exact:
+// the bounds are integers there; values too large for the magic constant still
+// clamp on the right side).  A byte where the ends differ is recomputed by the
+// caller; `diff` gets its bit.
+__device__ __forceinline__ uint32_t requant_codes4(const float* y, const Requant& c, uint32_t& diff, int bit0) {
+    constexpr float lo = qm::kMagic - 127.0f, hi = qm::kMagic + 127.0f;
+    uint32_t w = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float l = fminf(fmaxf(__fmaf_rn(y[e], c.rlo, qm::kMagic), lo), hi);
+        const float h = fminf(fmaxf(__fmaf_rn(y[e], c.rhi, qm::kMagic), lo), hi);
+        w |= (__float_as_uint(l) & 0xFFu) << (8 * e);
+        diff |= (l != h ? 1u : 0u) << (bit0 + e);
+    }
+    return w;
+}
+
+__device__ __forceinline__ uint32_t requant_code_fast(float y, const Requant& c) {
+    const float a = fabsf(y);
+    if (a * c.rhi < 127.5f) {
+        const float l = __fmaf_rn(y, c.rlo, qm::kMagic), h = __fmaf_rn(y, c.rhi, qm::kMagic);
+        if (l == h) return __float_as_uint(l) & 0xFFu;
+    } else if (a * c.rlo > 127.5f) {
+        return y > 0.f ? 127u : 0x81u;   // -127
+    }
+    return requant_code_slow(y, c.S);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     const __nv_bfloat16 lo = __float2bfloat16_rn(a), hi = __float2bfloat16_rn(b);
     return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
@@ -125,7 +180,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // ============================================================================
 // Persistent tile kernel
 // ============================================================================
-template <int BN, int KIND, bool MIXED>
+template <int BN, int KIND, bool MIXED, bool QOUT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmA16,
@@ -341,13 +396,18 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                         out[i] = v;
                     }
                 }
-                if (p.yq) {
-                    uint32_t w[8];
+                if constexpr (QOUT) {
+                    const Requant rq = requant_consts(p.out_scale);
+                    uint32_t w[8], diff = 0u;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        w[j] = requant_code(out[4 * j], p.out_scale) | (requant_code(out[4 * j + 1], p.out_scale) << 8) |
-                               (requant_code(out[4 * j + 2], p.out_scale) << 16) |
-                               (requant_code(out[4 * j + 3], p.out_scale) << 24);
+                    for (int j = 0; j < 8; ++j) w[j] = requant_codes4(&out[4 * j], rq, diff, 4 * j);
+                    if (diff != 0u) {   // rare: outputs near a rounding boundary
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if ((diff >> i) & 1u)
+                                w[i / 4] = (w[i / 4] & ~(0xFFu << (8 * (i % 4)))) |
+                                           (requant_code_slow(out[i], rq.S) << (8 * (i % 4)));
+                    }
                     uint4* qp = reinterpret_cast<uint4*>(p.yq + static_cast<int64_t>(row) * p.ldy + n0);
                     qp[0] = make_uint4(w[0], w[1], w[2], w[3]);
                     if (nv > 16) qp[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -623,7 +683,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
             if (p.bias) v = __fadd_rn(v, bias);
             if (col_ok) {
                 if (p.yq)
-                    p.yq[static_cast<int64_t>(t) * p.ldy + n] = static_cast<int8_t>(requant_code(v, p.out_scale));
+                    p.yq[static_cast<int64_t>(t) * p.ldy + n] = static_cast<int8_t>(requant_code_fast(v, requant_consts(p.out_scale)));
                 else
                     p.y[static_cast<int64_t>(t) * p.ldy + n] = __float2bfloat16_rn(v);
                 if (p.acc_debug)
@@ -689,7 +749,7 @@ cudaError_t set_smem(K kernel, int bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-template <int BN, int KIND, bool MIXED>
+template <int BN, int KIND, bool MIXED, bool QOUT = false>
 q8_status run_tile(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     using C = TileCfg<BN, MIXED>;
     CUtensorMap tA, tB, tA16, tB16;
@@ -704,7 +764,7 @@ q8_status run_tile(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
         tA16 = tA;
         tB16 = tB;
     }
-    auto kern = gemm_tile_kernel<BN, KIND, MIXED>;
+    auto kern = gemm_tile_kernel<BN, KIND, MIXED, QOUT>;
     if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
     const int tiles_m = static_cast<int>((a.m + kBM - 1) / kBM);
     const int tiles_n = static_cast<int>((a.n + BN - 1) / BN);
@@ -791,6 +851,13 @@ q8_status dispatch_kind(const LinearArgs& a, const EpiParams& ep, cudaStream_t s
         if (cost < best_cost) {
             best_cost = cost;
             best = bn;
+        }
+    }
+    if constexpr (KIND != kE4M3) {
+        if (a.yq != nullptr) {   // INT8 output codes
+            if (best == 256) return run_tile<256, KIND, false, true>(a, ep, s);
+            if (best == 224) return run_tile<224, KIND, false, true>(a, ep, s);
+            return run_tile<128, KIND, false, true>(a, ep, s);
         }
     }
     if (best == 256) return run_tile<256, KIND, false>(a, ep, s);
