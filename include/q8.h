@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define Q8_VERSION 1
+#define Q8_VERSION 2
 
 /* Same object as cudaStream_t. */
 typedef struct CUstream_st *q8_stream_t;
