@@ -68,6 +68,8 @@ def lib():
             "or_quant_act_int8": [vp, i64, i64, vp, vp, vp, vp],
             "or_quant_act_fp8": [vp, i64, i64, f, vp, vp],
             "or_quant_act_static": [vp, i64, i64, f, vp, vp, vp],
+            "or_quant_act_smooth": [vp, i64, i64, vp, vp, vp, vp],
+            "or_smooth_weight": [vp, i64, i64, vp, vp],
             "or_requant": [vp, i64, f, vp],
             "or_outlier_columns": [vp, i64, i64, f, vp, vp, vp],
             "or_gemm_int": [vp, i32, i64, vp, i32, i64, i64, vp, i64, vp, i64, vp],
@@ -187,6 +189,28 @@ def quant_act_static(x: np.ndarray, S: float):
     rs = np.empty(m, np.int32)
     lib().or_quant_act_static(_ptr(x), m, k, float(np.float32(S)), _ptr(q), _ptr(Sr), _ptr(rs))
     return q, Sr, rs
+
+
+def quant_act_smooth(x: np.ndarray, mult: np.ndarray):
+    """Dynamic INT8 quantization of fl32(x * mult[col]): (codes, scales, row sums)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    m, k = x.shape
+    mu = np.ascontiguousarray(mult, dtype=np.float32)
+    assert mu.shape == (k,)
+    q = np.empty((m, k), np.int8)
+    S = np.empty(m, np.float32)
+    rs = np.empty(m, np.int32)
+    lib().or_quant_act_smooth(_ptr(x), m, k, _ptr(mu), _ptr(q), _ptr(S), _ptr(rs))
+    return q, S, rs
+
+
+def smooth_weight(w: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """fl32(w * s[col]): the weight side of the smoothing (offline)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    n, k = w.shape
+    out = np.empty((n, k), np.float32)
+    lib().or_smooth_weight(_ptr(w), n, k, _ptr(np.ascontiguousarray(s, dtype=np.float32)), _ptr(out))
+    return out
 
 
 def requant(y: np.ndarray, S: float) -> np.ndarray:

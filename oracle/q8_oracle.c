@@ -318,6 +318,31 @@ void or_quant_act_int8(const float *X, int64_t m, int64_t k, const uint8_t *skip
 }
 
 /*
+ * Dynamic per-token INT8 quantization of a smoothed activation ("大模型量化"
+ * (Xilyfe), algorithm list, SmoothQuant: the activation's outlier channels are
+ * "smoothed" onto the weight side so the activation quantizes easily; the page
+ * gives no formula).  Reading: per input column j a smoothing factor s_j is
+ * chosen offline; the activation is divided by it and the weight column
+ * multiplied by it, which leaves X W^T unchanged.  The division is applied as
+ * a multiplier m_j = RN(1/s_j) supplied by the caller: xs = fl32(x * m_j), then
+ * the dynamic symmetric INT8 quantizer of or_quant_act_int8 runs on xs.  The
+ * weight side, fl32(w * s_j), is plain offline preprocessing (or_smooth_weight).
+ */
+void or_quant_act_smooth(const float *X, int64_t m, int64_t k, const float *mult, int8_t *q,
+                         float *S, int32_t *rowsum) {
+    float *xs = (float *)malloc((size_t)(m * k) * sizeof(float));
+    for (int64_t r = 0; r < m; ++r)
+        for (int64_t j = 0; j < k; ++j) xs[r * k + j] = X[r * k + j] * mult[j];
+    or_quant_act_int8(xs, m, k, NULL, q, S, rowsum);
+    free(xs);
+}
+
+void or_smooth_weight(const float *W, int64_t n, int64_t k, const float *s, float *out) {
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t j = 0; j < k; ++j) out[r * k + j] = W[r * k + j] * s[j];
+}
+
+/*
  * Static (calibrated) symmetric INT8 quantization with one scale for the
  * whole tensor ("大模型量化" (Xilyfe), the paragraph on 静态量化: the scale is
  * worked out once from a calibration pass and reused on every call instead of
