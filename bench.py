@@ -461,7 +461,7 @@ def load_profile_traffic(kernel_tag: str):
 
 # Sources the GEMM kernels are compiled from (a traffic entry stays valid
 # while these are unchanged).
-GEMM_SOURCES = ("q8_device.cuh", "q8_gemm.cu", "q8_internal.h")
+GEMM_SOURCES = ("q8_device.cuh", "q8_gemm.cu", "q8_qmath.cuh")
 
 
 def source_hash() -> str:
@@ -471,8 +471,6 @@ def source_hash() -> str:
     for f in GEMM_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
-    with open(os.path.join(ROOT, "include", "q8.h"), "rb") as fh:
-        h.update(b"q8.h" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -547,6 +545,11 @@ def extras(q8, dev, pk):
                 t_s = _time_kernel(lambda: q8.q8_quantize_act_static(Xd, S, out=qs), flush)
                 r["static_act_quant_us"] = round(t_s * 1e3, 2)
                 r["static_act_quant_gbs"] = round(act_bytes / (t_s * 1e-3) / 1e9, 1)
+                mult = torch.rand(w.k, generator=torch.Generator().manual_seed(1)).add_(0.5).to(dev)
+                qm = q8.q8_quantize_act_smooth(Xd, mult)
+                t_m = _time_kernel(lambda: q8.q8_quantize_act_smooth(Xd, mult, out=qm), flush)
+                r["smooth_act_quant_us"] = round(t_m * 1e3, 2)
+                r["smooth_act_quant_gbs"] = round(act_bytes / (t_m * 1e-3) / 1e9, 1)
                 So = float(1.2 * float(q8.q8_linear_w8a8(qs, qw).float().abs().max()) / 127)
                 Yq = torch.empty((w.m, w.n), dtype=torch.int8, device=dev)
                 t_r = _time_kernel(lambda: q8.q8_linear_w8a8_requant(qs, qw, So, out=Yq), flush)

@@ -220,6 +220,25 @@ q8_status q8_quantize_act_static(const void* X, q8_dtype x_dtype, int64_t m, int
     return launch_status(launch_row_quant(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+q8_status q8_quantize_act_smooth(const void* X, q8_dtype x_dtype, int64_t m, int64_t k, int64_t ldx,
+                                 const float* mult, void* codes, float* scale, int32_t* rowsum,
+                                 q8_stream_t stream) {
+    if (m < 0 || k <= 0 || m > kMaxDim || k > kMaxDim || k % 32 != 0 || ldx < k) return Q8_ERR_SHAPE;
+    if (!float_input(x_dtype)) return Q8_ERR_DTYPE;
+    if (m == 0) return Q8_OK;   // empty call
+    if (!X || !codes || !scale || !mult) return Q8_ERR_NULL;
+    if (!aligned16(X) || !aligned16(codes) || !aligned16(mult) || !ld_ok(ldx, k, x_dtype))
+        return Q8_ERR_ALIGN;
+    q8_status st = check_device();
+    if (st != Q8_OK) return st;
+    RowQuantArgs a = {};
+    a.src = X; a.src_dtype = x_dtype; a.rows = m; a.k = k; a.ld = ldx;
+    a.op = kOpActInt8Smooth;
+    a.mult = mult;
+    a.codes = codes; a.scale = scale; a.rowsum = rowsum;
+    return launch_status(launch_row_quant(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 static q8_status validate_outlier_act(const void* X, q8_dtype x_dtype, int64_t m, int64_t k,
                                       int64_t ldx, void* codes, float* scale, int32_t* rowsum,
                                       uint8_t* mask, int32_t* idx, int32_t* count,

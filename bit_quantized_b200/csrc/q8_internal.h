@@ -15,7 +15,7 @@ int* device_status_ptr();
 
 // ---- quantize kernels (q8_quant.cu)
 enum RowOp { kOpActInt8 = 0, kOpActFp8 = 1, kOpWeightAsym = 2, kOpWeightSym = 3, kOpWeightFp8 = 4,
-             kOpActInt8Static = 6 };
+             kOpActInt8Static = 6, kOpActInt8Smooth = 7 };
 
 struct RowQuantArgs {
     const void* src;       // rows x k input (f16 / bf16 / f32)
@@ -25,6 +25,7 @@ struct RowQuantArgs {
     bool codes_u8;         // asymmetric weights stored as uint8 (q + 128)
     float clip_ub;         // fp8 activations: > 0 clips the row absmax
     float static_scale;    // kOpActInt8Static: the calibrated scale (> 0)
+    const float* mult;     // kOpActInt8Smooth: [k] per-column multipliers (1 / smoothing factor)
     const uint8_t* skip;   // [k] columns left out (LLM.int8 outliers); may be null
     void* codes;           // rows x k, row stride k
     float* scale;          // [rows]

@@ -201,7 +201,8 @@ __device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, 
     c.bias = bias;
     if constexpr (OP == kOpActInt8Static) {
         c.S = static_scale;   // calibrated, > 0 (checked by the caller)
-    } else if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpWeightSym) {
+    } else if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActInt8Smooth ||
+                         OP == kOpWeightSym) {
         c.S = __fdiv_rn(amax, 127.0f);
     } else if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
         if (OP == kOpActFp8 && clip_ub > 0.f) amax = fminf(amax, clip_ub);
@@ -249,16 +250,39 @@ __device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, 
     return c;
 }
 
+// Multipliers of a vector's columns (activation smoothing), from L1.
+template <int V>
+__device__ __forceinline__ void load_mult(const float* mult, int64_t j, float (&m)[V]) {
+    const float4* p = reinterpret_cast<const float4*>(mult + j * V);
+    const float4 a = __ldg(p);
+    m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w;
+    if constexpr (V == 8) {
+        const float4 b = __ldg(p + 1);
+        m[4] = b.x; m[5] = b.y; m[6] = b.z; m[7] = b.w;
+    }
+}
+
+// Unpacked values of a vector; smoothed activations are fl32(x * m) per column.
+template <typename T, int OP>
+__device__ __forceinline__ void values_of(const uint4 u, const float* mv, float (&v)[VecOf<T>::N]) {
+    unpack_vec<T>(u, v);
+    if constexpr (OP == kOpActInt8Smooth) {
+#pragma unroll
+        for (int e = 0; e < VecOf<T>::N; ++e) v[e] = __fmul_rn(v[e], mv[e]);
+    }
+}
+
 // Fast codes of one vector from the lower end of the bracket, and per word the
 // code bytes where the upper end disagrees.  keep clears the bytes of left-out
 // columns (all ones otherwise); their disagreements do not count.
 template <typename T, int OP>
 __device__ __forceinline__ void fast_codes(const uint4 u, const RowConsts& c, const uint2 keep,
-                                           uint32_t (&words)[2], uint32_t (&diff)[2]) {
+                                           uint32_t (&words)[2], uint32_t (&diff)[2],
+                                           const float* mv = nullptr) {
     constexpr int V = VecOf<T>::N;
     const uint32_t kp[2] = {keep.x, keep.y};
     float v[V];
-    unpack_vec<T>(u, v);
+    values_of<T, OP>(u, mv, v);
     words[1] = diff[1] = 0u;
     if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
         const float2 L = splat2(c.rlo), H = splat2(c.rhi);
@@ -298,10 +322,12 @@ __device__ __forceinline__ void fast_codes(const uint4 u, const RowConsts& c, co
 // runs for a few elements in a thousand.
 template <typename T, int OP>
 __device__ __noinline__ uint2 exact_codes(const uint4 u, float S, float Z, float bias, uint2 redo,
-                                          uint2 words) {
+                                          uint2 words, const float* mult_vec) {
     constexpr int V = VecOf<T>::N;
     float v[V];
-    unpack_vec<T>(u, v);
+    float mv[V];
+    if constexpr (OP == kOpActInt8Smooth) load_mult<V>(mult_vec, 0, mv);
+    values_of<T, OP>(u, mv, v);
     uint32_t w[2] = {words.x, words.y};
     const uint32_t r[2] = {redo.x, redo.y};
     for (int e = 0; e < V; ++e) {
@@ -345,11 +371,14 @@ struct FixQueue {
 
 // Pushes the flagged elements of one vector (bytes of d that are nonzero).
 // Out of line, so the unrolled pass keeps a small instruction footprint.
-template <typename T>
-__device__ __noinline__ void push_flagged(const uint4 u, uint2 d, uint2 w, int pos0, FixQueue* q) {
+template <typename T, int OP>
+__device__ __noinline__ void push_flagged(const uint4 u, uint2 d, uint2 w, int pos0, FixQueue* q,
+                                          const float* mult_vec) {
     constexpr int V = VecOf<T>::N;
     float v[V];
-    unpack_vec<T>(u, v);
+    float mv[V];
+    if constexpr (OP == kOpActInt8Smooth) load_mult<V>(mult_vec, 0, mv);
+    values_of<T, OP>(u, mv, v);
     const uint32_t dd[2] = {d.x, d.y}, ww[2] = {w.x, w.y};
 #pragma unroll
     for (int e = 0; e < V; ++e) {
@@ -397,9 +426,17 @@ __device__ __forceinline__ uint4 zero_skipped16(uint4 u, const uint2 mb) {
 }
 
 template <typename T, int OP>
-__device__ __forceinline__ void accumulate_stats(const uint4 u, RowStats& st) {
+__device__ __forceinline__ void accumulate_stats(const uint4 u, RowStats& st, const float* mv = nullptr) {
     constexpr int V = VecOf<T>::N;
-    if constexpr (sizeof(T) == 2) {
+    if constexpr (OP == kOpActInt8Smooth) {
+        float v[V];
+        values_of<T, OP>(u, mv, v);
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+            st.lo = fminf(st.lo, v[e]);
+            st.hi = fmaxf(st.hi, v[e]);
+        }
+    } else if constexpr (sizeof(T) == 2) {
         using T2 = typename std::conditional<std::is_same<T, __half>::value, __half2, __nv_bfloat162>::type;
         const T2* p2 = reinterpret_cast<const T2*>(&u);
         T2 m2 = __hmax2(p2[0], p2[1]), l2 = __hmin2(p2[0], p2[1]);
@@ -428,7 +465,9 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
     constexpr int V = VecOf<T>::N;
     constexpr int RPB = kBlock / TPR;
     constexpr bool kSkip = OP == kOpActInt8Skip;
-    constexpr bool kRowsum = OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActInt8Static;
+    constexpr bool kRowsum = OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActInt8Static ||
+                             OP == kOpActInt8Smooth;
+    constexpr bool kSmooth = OP == kOpActInt8Smooth;
     __shared__ float red[3 * (kBlock / 32)];
     __shared__ int redi[kBlock / 32];
     __shared__ FixQueue fixq[kBlock / 32];
@@ -450,7 +489,8 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
     // its CTAs become resident and load their weights meanwhile (it waits for
     // this grid before reading the codes).  Weight quantizers do not: a GEMM
     // right after one must not load the weight before it is fully written.
-    if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActFp8 || OP == kOpActInt8Static)
+    if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActFp8 || OP == kOpActInt8Static ||
+                  OP == kOpActInt8Smooth)
         pdl_launch_dependents();
     pdl_wait();
 
@@ -493,7 +533,13 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
                         const uint2 kp = keep_of(t + static_cast<int64_t>(i) * TPR);
                         raw[i] = zero_skipped16(raw[i], make_uint2(~kp.x, ~kp.y));
                     }
-                    accumulate_stats<T, OP>(raw[i], st);
+                    if constexpr (kSmooth) {
+                        float mv[V];
+                        load_mult<V>(a.mult, t + static_cast<int64_t>(i) * TPR, mv);
+                        accumulate_stats<T, OP>(raw[i], st, mv);
+                    } else {
+                        accumulate_stats<T, OP>(raw[i], st);
+                    }
                 }
             }
         };
@@ -506,7 +552,13 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
                     const uint2 kp = keep_of(j);
                     u = zero_skipped16(u, make_uint2(~kp.x, ~kp.y));
                 }
-                accumulate_stats<T, OP>(u, st);
+                if constexpr (kSmooth) {
+                    float mv[V];
+                    load_mult<V>(a.mult, j, mv);
+                    accumulate_stats<T, OP>(u, st, mv);
+                } else {
+                    accumulate_stats<T, OP>(u, st);
+                }
             }
         }
         st.amax = fmaxf(st.hi, -st.lo);
@@ -562,12 +614,18 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
                     const bool valid = FULL || i < nv;
                     const uint2 kp = valid ? keep_of(t + static_cast<int64_t>(i) * TPR) : make_uint2(~0u, ~0u);
                     uint32_t words[2], d[2];
-                    fast_codes<T, OP>(raw[i], c, kp, words, d);   // zero vectors: d = 0
+                    float mv[V];
+                    if constexpr (kSmooth) {
+                        if (valid) load_mult<V>(a.mult, t + static_cast<int64_t>(i) * TPR, mv);
+                        else for (int e = 0; e < V; ++e) mv[e] = 0.f;
+                    }
+                    fast_codes<T, OP>(raw[i], c, kp, words, d, mv);   // zero vectors: d = 0
                     if (valid) finish(words[0], words[1], dst + i * TPR * V);
                     if (__any_sync(0xffffffffu, (d[0] | d[1]) != 0u)) {
                         if ((d[0] | d[1]) != 0u)
-                            push_flagged<T>(raw[i], make_uint2(d[0], d[1]), make_uint2(words[0], words[1]),
-                                            (t + i * TPR) * V, q);
+                            push_flagged<T, OP>(raw[i], make_uint2(d[0], d[1]), make_uint2(words[0], words[1]),
+                                                (t + i * TPR) * V, q,
+                                                kSmooth ? a.mult + (t + static_cast<int64_t>(i) * TPR) * V : nullptr);
                         __syncwarp();
                         if (q->n >= kDrainAt) drain();
                     }
@@ -587,10 +645,13 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
                 const uint4 u = ld_stream16(src_row + j * V);
                 const uint2 kp = keep_of(j);
                 uint32_t words[2] = {0u, 0u}, d[2] = {~0u, ~0u};
-                if (c.fast) fast_codes<T, OP>(u, c, kp, words, d);
+                float mv[V];
+                if constexpr (kSmooth) load_mult<V>(a.mult, j, mv);
+                if (c.fast) fast_codes<T, OP>(u, c, kp, words, d, mv);
                 if ((d[0] | d[1]) != 0u) {
                     const uint2 e = exact_codes<T, OP>(u, c.S, c.Z, c.bias, make_uint2(d[0], d[1]),
-                                                       make_uint2(words[0], words[1]));
+                                                       make_uint2(words[0], words[1]),
+                                                       kSmooth ? a.mult + j * V : nullptr);
                     words[0] = e.x & kp.x;
                     words[1] = e.y & kp.y;
                 }
@@ -694,6 +755,7 @@ cudaError_t launch_rows_dtype(const RowQuantArgs& a, cudaStream_t s) {
             return launch_rows_t<T, kOpActInt8>(a, s);
         case kOpActFp8: return launch_rows_t<T, kOpActFp8>(a, s);
         case kOpActInt8Static: return launch_rows_t<T, kOpActInt8Static>(a, s);
+        case kOpActInt8Smooth: return launch_rows_t<T, kOpActInt8Smooth>(a, s);
         case kOpWeightAsym: return launch_rows_t<T, kOpWeightAsym>(a, s);
         case kOpWeightSym: return launch_rows_t<T, kOpWeightSym>(a, s);
         case kOpWeightFp8: return launch_rows_t<T, kOpWeightFp8>(a, s);

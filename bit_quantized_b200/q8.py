@@ -37,6 +37,7 @@ Q8_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 EXPORTED = [
     "q8_quantize_weight", "q8_dequantize_weight", "q8_quantize_act", "q8_quantize_act_static",
+    "q8_quantize_act_smooth",
     "q8_outlier_quantize_act",
     "q8_linear_w8a8", "q8_linear_w8a8_requant", "q8_linear_w8a8_dynamic", "q8_linear_int8_mixed",
     "q8_linear_int8_mixed_noalloc",
@@ -63,6 +64,7 @@ _SIG = {
     "q8_dequantize_weight": ([ctypes.POINTER(CWeight), _int, _vp, _vp], _int),
     "q8_quantize_act": ([_vp, _int, _i64, _i64, _i64, _int, _f, _vp, _vp, _vp, _vp], _int),
     "q8_quantize_act_static": ([_vp, _int, _i64, _i64, _i64, _f, _vp, _vp, _vp, _vp], _int),
+    "q8_quantize_act_smooth": ([_vp, _int, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp], _int),
     "q8_outlier_quantize_act": ([_vp, _int, _i64, _i64, _i64, _f, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _vp, _i64, _vp], _int),
     "q8_linear_w8a8": ([ctypes.POINTER(CAct), ctypes.POINTER(CWeight), _vp, _vp, _i64, _vp, _vp,
@@ -234,6 +236,23 @@ def q8_quantize_act_static(X: torch.Tensor, scale: float, out: Optional[QAct] = 
     _check(_lib.q8_quantize_act_static(_ptr(X), _FLOAT_DT[X.dtype], m, k, X.stride(0), float(scale),
                                        _ptr(out.codes), _ptr(out.scale), _ptr(out.rowsum),
                                        _stream(stream)), "q8_quantize_act_static")
+    return out
+
+
+def q8_quantize_act_smooth(X: torch.Tensor, mult: torch.Tensor, out: Optional[QAct] = None,
+                           stream=None) -> QAct:
+    """Dynamic INT8 quantization of X * mult (per-column smoothing multipliers, fp32 [k])."""
+    _cuda(X, "X")
+    m, k = X.shape
+    if not mult.is_cuda or mult.dtype != torch.float32 or mult.shape != (k,) or not mult.is_contiguous():
+        raise ValueError("mult must be a contiguous CUDA float32 tensor of shape (k,)")
+    if out is None:
+        out = QAct(torch.empty((m, k), dtype=torch.int8, device=X.device),
+                   torch.empty(m, dtype=torch.float32, device=X.device),
+                   torch.empty(m, dtype=torch.int32, device=X.device), Q8_S8)
+    _check(_lib.q8_quantize_act_smooth(_ptr(X), _FLOAT_DT[X.dtype], m, k, X.stride(0), _ptr(mult),
+                                       _ptr(out.codes), _ptr(out.scale), _ptr(out.rowsum),
+                                       _stream(stream)), "q8_quantize_act_smooth")
     return out
 
 

@@ -57,7 +57,7 @@
 extern "C" {
 #endif
 
-#define Q8_VERSION 2
+#define Q8_VERSION 3
 
 /* Same object as cudaStream_t. */
 typedef struct CUstream_st *q8_stream_t;
@@ -182,6 +182,22 @@ q8_status q8_quantize_act(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
  */
 q8_status q8_quantize_act_static(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
                                  int64_t ldx, float static_scale, void *codes, float *scale,
+                                 int32_t *rowsum, q8_stream_t stream);
+
+/*
+ * Dynamic per-token INT8 quantization of a smoothed activation ([Xilyfe]
+ * algorithm list, SmoothQuant: outlier channels of the activation are moved
+ * onto the weight, which leaves X W^T unchanged and makes the activation easy
+ * to quantize).  Column j is multiplied by mult[j] = RN(1 / s_j) before the
+ * quantizer of q8_quantize_act (Q8_SYM_INT8) runs: xs = fl32(x * mult[j]),
+ * S = max(fl32(max|xs| / 127), 1e-8), q = clamp(rne(fl32(xs / S)), -127, 127).
+ * The smoothing factors s_j are chosen offline; the weight is smoothed offline
+ * too (W[:, j] * s_j) and quantized with q8_quantize_weight.
+ *   mult     device [k] float, 16-byte aligned.
+ *   others   as q8_quantize_act with Q8_SYM_INT8.
+ */
+q8_status q8_quantize_act_smooth(const void *X, q8_dtype x_dtype, int64_t m, int64_t k,
+                                 int64_t ldx, const float *mult, void *codes, float *scale,
                                  int32_t *rowsum, q8_stream_t stream);
 
 /*

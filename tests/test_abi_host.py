@@ -224,3 +224,18 @@ def test_quantize_act_static_validation():
     assert qs(m=0, X=None, codes=None, sc=None) == q8.Q8_OK     # empty call
     if NO_GPU:
         assert qs(rs=None) in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def qsm(X=FAKE, m=16, k=128, ldx=128, mult=FAKE, codes=FAKE, sc=FAKE, rs=FAKE, dt=q8.Q8_BF16):
+    return L.q8_quantize_act_smooth(X, dt, m, k, ldx, mult, codes, sc, rs, _ns)
+
+
+def test_quantize_act_smooth_validation():
+    assert qsm(mult=None) == q8.Q8_ERR_NULL
+    assert qsm(X=None) == q8.Q8_ERR_NULL
+    assert qsm(k=100, ldx=100) == q8.Q8_ERR_SHAPE
+    assert qsm(dt=q8.Q8_U8) == q8.Q8_ERR_DTYPE
+    assert qsm(mult=MIS) == q8.Q8_ERR_ALIGN
+    assert qsm(m=0, X=None, mult=None) == q8.Q8_OK               # empty call
+    if NO_GPU:
+        assert qsm() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
