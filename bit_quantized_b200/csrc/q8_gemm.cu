@@ -479,7 +479,7 @@ struct DecodeCfg {
     static constexpr int SMEM = STAGES * STAGE + RED_BYTES + 1024;
 };
 
-template <int NT, int KIND>
+template <int NT, int KIND, bool QOUT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                    const EpiParams p, int num_kb, int kb_per_split, int splits, int nstages) {
@@ -682,7 +682,7 @@ gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constan
             }
             if (p.bias) v = __fadd_rn(v, bias);
             if (col_ok) {
-                if (p.yq)
+                if constexpr (QOUT)
                     p.yq[static_cast<int64_t>(t) * p.ldy + n] = static_cast<int8_t>(requant_code_fast(v, requant_consts(p.out_scale)));
                 else
                     p.y[static_cast<int64_t>(t) * p.ldy + n] = __float2bfloat16_rn(v);
@@ -788,14 +788,14 @@ q8_status run_tile(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     return Q8_OK;
 }
 
-template <int NT, int KIND>
+template <int NT, int KIND, bool QOUT = false>
 q8_status run_decode(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     using C = DecodeCfg<NT, KIND>;
     CUtensorMap tW, tX;
     if (!make_map(&tW, a.b_codes, false, a.k, a.n, a.ldb, kBKB, kBM) ||
         !make_map(&tX, a.a_codes, false, a.k, a.m, a.lda, kBKB, NT))
         return Q8_ERR_CUDA;
-    auto kern = gemm_decode_kernel<NT, KIND>;
+    auto kern = gemm_decode_kernel<NT, KIND, QOUT>;
     if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
     const int tiles_n = static_cast<int>((a.n + kBM - 1) / kBM);
     const int num_kb = static_cast<int>((a.k + kBKB - 1) / kBKB);
@@ -835,6 +835,13 @@ q8_status run_decode(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
 
 template <int KIND>
 q8_status dispatch_kind(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
+    if constexpr (KIND != kE4M3) {
+        if (a.yq != nullptr && a.m <= 64) {   // INT8 output codes
+            if (a.m <= 16) return run_decode<16, KIND, true>(a, ep, s);
+            if (a.m <= 32) return run_decode<32, KIND, true>(a, ep, s);
+            return run_decode<64, KIND, true>(a, ep, s);
+        }
+    }
     if (a.m <= 16) return run_decode<16, KIND>(a, ep, s);
     if (a.m <= 32) return run_decode<32, KIND>(a, ep, s);
     if (a.m <= 64) return run_decode<64, KIND>(a, ep, s);

@@ -35,7 +35,8 @@ def _static_check(X: torch.Tensor, S: float, what: str):
 
 @pytest.mark.parametrize("m,k,dtype", [(16, 4096, torch.bfloat16), (2048, 4096, torch.bfloat16),
                                        (4096, 8192, torch.bfloat16), (5, 160, torch.float32),
-                                       (3, 96, torch.float16), (33, 8192, torch.float16)])
+                                       (3, 96, torch.float16), (33, 8192, torch.float16),
+                                       (2, 32768, torch.bfloat16)])   # longer than the register cache
 def test_static_act_scales(m, k, dtype):
     X = workloads.random_matrix(m, k, dtype, seed=m + k)
     amax = float(X.float().abs().max())
@@ -54,7 +55,8 @@ def test_static_act_midpoints():
 
 @pytest.mark.parametrize("m,n,k,codes,wscheme", [(16, 4096, 4096, "u8", "asym"),
                                                  (256, 512, 1024, "s8", "sym"),
-                                                 (3, 208, 160, "s8", "asym")])
+                                                 (3, 208, 160, "s8", "asym"),
+                                                 (40, 512, 1024, "u8", "asym")])   # NT = 64 decode
 def test_requant_linear(m, n, k, codes, wscheme):
     X = workloads.random_matrix(m, k, torch.bfloat16, seed=m + 2 * n)
     W = workloads.random_matrix(n, k, torch.bfloat16, seed=n + k, std=0.02)
