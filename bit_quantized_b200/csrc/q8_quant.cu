@@ -15,6 +15,12 @@
 //               Lightning Fabric, sections 2.1 and 2.3)
 //   FP8         S = max(min(absmax, ub) / 448, 1e-8), q = e4m3_rne_satfinite(x / S)
 //               (Transformers FP8 (W8A8) / FBGEMM page, sections 5.1, 5.2 and 6)
+//   static      S given (calibrated offline), q = clamp(rne(x / S), -127, 127)
+//               ("大模型量化" (Xilyfe), the paragraph on static quantization)
+//   smoothed    xs = x * m_col (m = 1 / smoothing factor), then symmetric on xs
+//               (same page, algorithm list, SmoothQuant)
+// Every x / S above is the IEEE fp32 quotient; the kernels reach its rounding
+// without a division per element (see "Codes of one 16-byte vector" below).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
