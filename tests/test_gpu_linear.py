@@ -240,6 +240,17 @@ def test_mixed_many_outliers():
     assert count > 64
 
 
+def test_mixed_more_tiles_than_sms():
+    # 1152 x 2560: 9 x 20 = 180 tiles of 128 x 128, more than one wave of the
+    # persistent grid (148 CTAs), so CTAs run two tiles with both TMEM buffers.
+    X = workloads.random_matrix(1152, 512, torch.float16, seed=59)
+    X[:, [5, 77, 300]] *= 14
+    W = workloads.random_matrix(2560, 512, torch.float16, seed=60, std=0.02)
+    rows = P.sample_indices(1152, 256, 3)
+    cols = P.sample_indices(2560, 512, 4)
+    _mixed_case(X, W, 6.0, rows=rows, cols=cols, what="mixed 1152x2560")
+
+
 def test_device_status_clean():
     assert q8.q8_get_device_status() == 0
 
