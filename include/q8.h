@@ -6,7 +6,10 @@
  *   - dynamic per-token activation quantization (symmetric INT8 with row sums,
  *     or FP8 E4M3 with an upper-bound clip);
  *   - the W8A8 GEMM with INT32 / FP32 accumulation and a dequant epilogue;
- *   - the LLM.int8 mixed decomposition (outlier feature columns in fp16).
+ *   - the LLM.int8 mixed decomposition (outlier feature columns in fp16);
+ *   - around it: activations with a static (calibrated) scale, smoothed
+ *     activations (SmoothQuant-style per-column multipliers), and a W8A8 linear
+ *     that re-quantizes its output to INT8 for the next layer.
  *
  * Notation follows the pages' linear map Q = round(R / S) + Z, R = S (Q - Z):
  * `scale` is S, the dequant multiplier, and `zero_point` is Z, an integer held
@@ -35,8 +38,9 @@
  *   Alignment   every pointer 16-byte aligned; every leading dimension a
  *               multiple of 16 bytes.
  *   Values      inputs must be finite; NaN and Inf inputs give unspecified codes.
- *   Rounding    round-half-to-even everywhere; q = rne(fl32(x / S)) with an
- *               IEEE fp32 division, so codes are bit-exact with a scalar
+ *   Rounding    round-half-to-even everywhere; q = rne(fl32(x / S)) for the
+ *               IEEE fp32 quotient (the kernels reach its rounding without a
+ *               division per element), so codes are bit-exact with a scalar
  *               reference; S is floored at 1e-8 ([Xilyfe] QuantConfig eps).
  *   Errors      every call returns a q8_status and never prints, throws or
  *               aborts.  Arguments are validated on the host before anything is
