@@ -645,7 +645,9 @@ def run_reference(args, world, rank):
             "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3" if w.kind == "w8a8_fp8" else "s8",
             "data": "synthetic",
-            "config": {"workload": args.workload, "m_tokens": w.m, "n_out": w.n, "k_in": w.k},
+            "config": {"workload": args.workload, "m_tokens": w.m, "n_out": w.n, "k_in": w.k,
+                       **describe(w), "parallelism": f"dp{world} (independent batches per GPU)",
+                       "timing": "host wall clock of the oracle on the host cores, bounded sample per step"},
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": O.threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
