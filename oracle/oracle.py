@@ -65,6 +65,8 @@ def lib():
             "or_quant_weight_asym": [vp, i64, i64, i32, vp, vp, vp],
             "or_quant_weight_sym": [vp, i64, i64, i32, vp, vp],
             "or_quant_weight_fp8": [vp, i64, i64, vp, vp],
+            "or_quant_weight_group": [vp, i64, i64, i32, i64, vp, vp],
+            "or_dequant_group16": [vp, vp, i64, i64, i64, i32, vp],
             "or_quant_act_int8": [vp, i64, i64, vp, vp, vp, vp],
             "or_quant_act_fp8": [vp, i64, i64, f, vp, vp],
             "or_quant_act_static": [vp, i64, i64, f, vp, vp, vp],
@@ -165,6 +167,44 @@ def quant_weight(w: np.ndarray, scheme: str, codes: str = "s8", bits: int = 8):
         L.or_quant_weight_fp8(_ptr(w), n, k, _ptr(q), _ptr(S))
         return q, S, None
     raise ValueError(scheme)
+
+
+def quant_weight_group(w: np.ndarray, g: int, bits: int = 4):
+    """Group-wise symmetric weights: every g consecutive values of a row share
+    one absmax scale.  Returns (q int8 N x K in [-qmax, qmax], S N x K/g)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    n, k = w.shape
+    assert k % g == 0
+    q = np.empty((n, k), np.int8)
+    S = np.empty((n, k // g), np.float32)
+    lib().or_quant_weight_group(_ptr(w), n, k, bits, g, _ptr(q), _ptr(S))
+    return q, S
+
+
+def dequant_group16(q: np.ndarray, S: np.ndarray, g: int, fmt: str) -> np.ndarray:
+    """16-bit bits of fl32(S[n, k/g] * q[n, k]) rounded to fmt ("f16"/"bf16")."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    S = np.ascontiguousarray(S, dtype=np.float32)
+    n, k = q.shape
+    out = np.empty((n, k), np.uint16)
+    lib().or_dequant_group16(_ptr(q), _ptr(S), n, k, g, _FMT[fmt], _ptr(out))
+    return out
+
+
+def linear_w4a16(x: np.ndarray, q: np.ndarray, S: np.ndarray, g: int, fmt: str,
+                 bias=None, rows=None, cols=None):
+    """Group-quantized weight times 16-bit activations.
+
+    x: M x K fp32 holding fmt values.  The weight is dequantized to fmt
+    (dequant_group16), the products are summed in double and rounded once to
+    fp32, then y = fl32(y + bias[n]); Y = bf16_rne(y).  Returns (y, Y)."""
+    k = q.shape[1]
+    w16 = widen16(dequant_group16(q, S, g, fmt), fmt)
+    c = _index(cols, q.shape[0])
+    y = outlier_gemm(x, w16, np.arange(k, dtype=np.int32), rows, c)
+    if bias is not None:
+        y = (y + np.asarray(bias, np.float32)[c][None, :]).astype(np.float32)
+    return y, round16(y, "bf16")
 
 
 # ---------------------------------------------------------------- activations

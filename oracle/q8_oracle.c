@@ -230,25 +230,64 @@ void or_quant_weight_asym(const float *W, int64_t n, int64_t k, int bits,
  * [Xilyfe] QuantInt8._quantize sketch.  Worked examples with b = 4 sit in the
  * [Xilyfe] GGUF section.
  */
+/* One block of `len` weights: S = fl32(max|w| / qmax), eps floor,
+ * q = clamp(rne(fl32(w / S)), -qmax, qmax). */
+static void sym_block(const float *w, int64_t len, double qmax, int8_t *q, float *S) {
+    float a = 0.0f;
+    for (int64_t j = 0; j < len; ++j) {
+        float v = fabsf(w[j]);
+        if (v > a) a = v;
+    }
+    float s = a / (float)qmax;
+    if (!(s >= OR_EPS)) s = OR_EPS;
+    for (int64_t j = 0; j < len; ++j) {
+        float t = w[j] / s;
+        q[j] = (int8_t)clampd(rne((double)t), -qmax, qmax);
+    }
+    *S = s;
+}
+
 void or_quant_weight_sym(const float *W, int64_t n, int64_t k, int bits,
                          int8_t *q, float *S) {
     const double qmax = ldexp(1.0, bits - 1) - 1.0;
 #pragma omp parallel for schedule(static)
-    for (int64_t r = 0; r < n; ++r) {
-        const float *w = W + r * k;
-        float a = 0.0f;
+    for (int64_t r = 0; r < n; ++r) sym_block(W + r * k, k, qmax, q + r * k, &S[r]);
+}
+
+/*
+ * Group-wise symmetric b-bit weights.  [CSDN] 2.2 (granularity table): one
+ * scale per group of 64-128 consecutive parameters; [Xilyfe] GGUF section:
+ * the row is cut into blocks and each block gets its own absmax scale, with
+ * qmax = 2^(b-1) - 1 (7 for 4 bits).  Every group of g consecutive weights
+ * along a row is one block of the symmetric rule above.  S is n x (k / g),
+ * row-major: S[r * (k / g) + j] belongs to weights r, j*g .. j*g + g - 1.
+ */
+void or_quant_weight_group(const float *W, int64_t n, int64_t k, int bits, int64_t g,
+                           int8_t *q, float *S) {
+    const double qmax = ldexp(1.0, bits - 1) - 1.0;
+    const int64_t ng = k / g;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t j = 0; j < ng; ++j)
+            sym_block(W + r * k + j * g, g, qmax, q + r * k + j * g, &S[r * ng + j]);
+}
+
+/*
+ * The 16-bit weight a group-quantized layer multiplies when its activations
+ * are 16-bit (W4A16: the weight is brought back to the activation's format,
+ * r = S q, [Xilyfe] "量化是什么" with Z = 0):
+ * out[r, j] = round16(fl32(S[r, j / g] * q[r, j]), fmt), fmt 0 fp16, 1 bf16.
+ */
+void or_dequant_group16(const int8_t *q, const float *S, int64_t n, int64_t k, int64_t g,
+                        int fmt, uint16_t *out) {
+    build_tables();
+    const int64_t ng = k / g;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r)
         for (int64_t j = 0; j < k; ++j) {
-            float v = fabsf(w[j]);
-            if (v > a) a = v;
+            float v = S[r * ng + j / g] * (float)q[r * k + j];
+            out[r * k + j] = (uint16_t)enc_format((double)v, fmt == 0 ? OR_F16 : OR_BF16);
         }
-        float s = a / (float)qmax;
-        if (!(s >= OR_EPS)) s = OR_EPS;
-        for (int64_t j = 0; j < k; ++j) {
-            float t = w[j] / s;
-            q[r * k + j] = (int8_t)clampd(rne((double)t), -qmax, qmax);
-        }
-        S[r] = s;
-    }
 }
 
 /*
