@@ -555,6 +555,18 @@ def extras(q8, dev, pk):
                 t_r = _time_kernel(lambda: q8.q8_linear_w8a8_requant(qs, qw, So, out=Yq), flush)
                 r["requant_gemm_us"] = round(t_r * 1e3, 2)
                 r["requant_gemm_tops"] = round(2.0 * w.m * w.n * w.k / (t_r * 1e-3) / 1e12, 1)
+                # Group-wise 4-bit weights (groups of 128 along K) with the same
+                # bf16 activations: codes k/2 bytes per row + fp32 scales, X, Y.
+                g4 = q8.q8_quantize_weight_g4(Wd, 128)
+                Y4 = torch.empty((w.m, w.n), dtype=torch.bfloat16, device=dev)
+                t_4 = _time_kernel(lambda: q8.q8_linear_w4a16(Xd, g4, out=Y4), flush)
+                b4 = w.n * w.k // 2 + 4 * w.n * (w.k // 128) + 2 * w.m * w.k + 2 * w.m * w.n
+                r["w4a16_us"] = round(t_4 * 1e3, 2)
+                r["w4a16_tflops"] = round(2.0 * w.m * w.n * w.k / (t_4 * 1e-3) / 1e12, 1)
+                r["w4a16_gbs"] = round(b4 / (t_4 * 1e-3) / 1e9, 1)
+                r["w4a16_frac_hbm"] = round(b4 / (t_4 * 1e-3) / 1e9 / pk["hbm_gbs"], 4)
+                r["w4a16_frac_bf16_peak"] = round(2.0 * w.m * w.n * w.k / (t_4 * 1e-3) / 1e12
+                                                  / pk["bf16_tflops"], 4)
         out[name] = r
         del Xd, Wd
     torch.cuda.synchronize()

@@ -459,6 +459,57 @@ q8_status q8_linear_int8_mixed(const void* X, q8_dtype x_dtype, int64_t m, int64
     return Q8_OK;
 }
 
+q8_status q8_quantize_weight_g4(const void* W, q8_dtype w_dtype, int64_t n, int64_t k,
+                                int64_t ldw, int32_t group, void* codes, int64_t ldc,
+                                float* scale, q8_stream_t stream) {
+    if (w_dtype != Q8_F16 && w_dtype != Q8_BF16) return Q8_ERR_DTYPE;
+    if (group != 32 && group != 64 && group != 128) return Q8_ERR_SCHEME;
+    if (n < 0 || k <= 0 || n > kMaxDim || k > kMaxDim || k % 32 != 0 || k % group != 0 ||
+        n % 16 != 0 || ldw < k || ldc < k / 2)
+        return Q8_ERR_SHAPE;
+    if (n == 0) return Q8_OK;
+    if (!W || !codes || !scale) return Q8_ERR_NULL;
+    if (!aligned16(W) || !ld_ok(ldw, k, w_dtype) || !aligned16(codes) || ldc % 16 != 0 ||
+        !aligned16(scale))
+        return Q8_ERR_ALIGN;
+    q8_status st = check_device();
+    if (st != Q8_OK) return st;
+    return launch_status(launch_group_quant(W, w_dtype, n, k, ldw, group,
+                                            static_cast<uint8_t*>(codes), ldc, scale,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+q8_status q8_linear_w4a16(const void* X, q8_dtype x_dtype, int64_t m, int64_t k, int64_t ldx,
+                          const q8_weight_g4* w, const float* bias, void* Y, int64_t ldy,
+                          q8_stream_t stream) {
+    if (!w) return Q8_ERR_NULL;
+    if (x_dtype != Q8_F16 && x_dtype != Q8_BF16) return Q8_ERR_DTYPE;
+    if (w->group != 32 && w->group != 64 && w->group != 128) return Q8_ERR_SCHEME;
+    if (w->n < 0 || w->k <= 0 || w->n > kMaxDim || w->k > kMaxDim || w->k % 32 != 0 ||
+        w->k % w->group != 0 || w->n % 16 != 0 || w->ld < w->k / 2)
+        return Q8_ERR_SHAPE;
+    // token tiles of up to 256 along the grid's z dimension (at most 65535)
+    if (m < 0 || m > int64_t(65535) * 256 || k != w->k || ldx < k || ldy < w->n) return Q8_ERR_SHAPE;
+    if (m == 0 || w->n == 0) return Q8_OK;   // empty call
+    if (!X || !Y || !w->codes || !w->scale) return Q8_ERR_NULL;
+    if (!aligned16(X) || !ld_ok(ldx, k, x_dtype) || !aligned16(Y) || ldy % 8 != 0 ||
+        !aligned16(w->codes) || w->ld % 16 != 0 || !aligned16(w->scale) ||
+        (bias && !aligned16(bias)))
+        return Q8_ERR_ALIGN;
+    q8_status st = check_device();
+    if (st != Q8_OK) return st;
+    W4Args a = {};
+    a.x = X; a.x_bf16 = x_dtype == Q8_BF16;
+    a.m = m; a.k = k; a.ldx = ldx;
+    a.codes = w->codes; a.ldc = w->ld;
+    a.scale = w->scale;
+    a.n = w->n;
+    a.group = w->group;
+    a.bias = bias;
+    a.y = static_cast<__nv_bfloat16*>(Y); a.ldy = ldy;
+    return launch_w4a16(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 q8_status q8_get_device_status(int32_t* out, q8_stream_t stream) {
     if (!out) return Q8_ERR_NULL;
     q8_status st = check_device();

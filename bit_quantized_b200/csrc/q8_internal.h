@@ -76,5 +76,23 @@ struct LinearArgs {
 
 q8_status launch_linear(const LinearArgs& a, cudaStream_t s);
 
+// ---- group-wise 4-bit weights (q8_w4.cu)
+cudaError_t launch_group_quant(const void* W, q8_dtype dt, int64_t n, int64_t k, int64_t ldw,
+                               int group, uint8_t* codes, int64_t ldc, float* scale,
+                               cudaStream_t s);
+
+struct W4Args {
+    const void* x; bool x_bf16;            // m x k activations (bf16 or fp16), row stride ldx
+    int64_t m, k, ldx;
+    const void* codes; int64_t ldc;        // n x k/2 packed nibbles (q + 8), row stride ldc bytes
+    const float* scale;                    // (k / group) x n, group-major
+    int64_t n;
+    int group;                             // 32, 64 or 128
+    const float* bias;
+    __nv_bfloat16* y; int64_t ldy;
+};
+
+q8_status launch_w4a16(const W4Args& a, cudaStream_t s);
+
 
 }  // namespace q8

@@ -1,0 +1,553 @@
+// Group-wise 4-bit weights with 16-bit activations (W4A16) on the sm_100a
+// tensor cores.
+//
+// What is computed (quantization overview "大模型量化技术", 2.2 granularity
+// table: one scale per group of consecutive parameters; "大模型量化" (Xilyfe),
+// GGUF section: absmax per block, qmax = 2^(4-1) - 1 = 7):
+//   weights  S[j, r] = fl32(max |w| over group j of row r / 7), eps floor 1e-8
+//            q = clamp(rne(fl32(w / S)), -7, 7), stored as the nibble q + 8
+//   linear   w~ = round16(fl32(S q)) in the activation's 16-bit format,
+//            y = sum_k x w~ (fp32 in TMEM), y = fl32(y + bias[n]), Y = bf16(y)
+//
+// Storage: codes are n x k/2 bytes, element 2j in the low nibble of byte j and
+// element 2j+1 in the high nibble; scales are group-major, scale[j * n + r], so
+// the 128 rows of a tile read one contiguous 512-byte run per group.
+//
+// w4a16_kernel: a CTA owns 128 output channels (the MMA's M side, one TMEM
+// lane each) and NT tokens (the MMA's N side).  For small token counts the K
+// range is split across the CTAs of a cluster and the fp32 partials are summed
+// through distributed shared memory in rank order, as in the int8 decode GEMM.
+//   warp 0     one lane streams the packed codes and the scales of each
+//              64-deep K slice into a ring of staging slots (TMA, no swizzle);
+//   warp 1     TMEM allocation; one lane issues tcgen05.mma kind::f16;
+//   warps 2-5  dequantize: thread r expands row r's 64 codes of a slice into
+//              16-bit values written directly in the 128-byte-swizzled K-major
+//              layout the MMA reads (thread 0 also starts the activation
+//              tile's TMA into the same stage); then the same warps run the
+//              epilogue.
+// No TMA multicast is used.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "q8_device.cuh"
+#include "q8_internal.h"
+
+namespace q8 {
+namespace {
+
+constexpr float kEps = 1e-8f;
+
+// ============================================================================
+// Weight quantizer: one thread per group
+// ============================================================================
+__device__ __forceinline__ float widen1(__half h) { return __half2float(h); }
+__device__ __forceinline__ float widen1(__nv_bfloat16 h) { return __bfloat162float(h); }
+
+template <typename T>
+__device__ __forceinline__ void widen8(const uint4& v, float (&f)[8]) {
+    const T* h = reinterpret_cast<const T*>(&v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = widen1(h[i]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+group_quant_kernel(const T* __restrict__ W, int64_t n, int64_t k, int64_t ldw, int g,
+                   uint8_t* __restrict__ codes, int64_t ldc, float* __restrict__ scale) {
+    const int64_t ng = k / g;
+    const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (id >= n * ng) return;
+    const int64_t row = id / ng, grp = id % ng;
+    const T* w = W + row * ldw + grp * g;
+    float a = 0.f;
+    for (int j = 0; j < g; j += 8) {
+        float f[8];
+        widen8<T>(*reinterpret_cast<const uint4*>(w + j), f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(f[i]));
+    }
+    float S = __fdiv_rn(a, 7.0f);
+    if (!(S >= kEps)) S = kEps;
+    uint8_t* out = codes + row * ldc + grp * (g / 2);
+    for (int j = 0; j < g; j += 32) {
+        uint32_t word[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            float f[8];
+            widen8<T>(*reinterpret_cast<const uint4*>(w + j + 8 * v), f);
+            uint32_t packed = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                int q = __float2int_rn(__fdiv_rn(f[i], S));
+                q = q < -7 ? -7 : (q > 7 ? 7 : q);
+                packed |= static_cast<uint32_t>(q + 8) << (4 * i);
+            }
+            word[v] = packed;
+        }
+        *reinterpret_cast<uint4*>(out + j / 2) = make_uint4(word[0], word[1], word[2], word[3]);
+    }
+    scale[grp * n + row] = S;
+}
+
+// ============================================================================
+// W4A16 GEMM
+// ============================================================================
+constexpr int kThreads = 192;
+constexpr int kBM = 128;                        // weight rows per CTA (MMA M)
+constexpr int kBK = 64;                         // K elements per stage (128 bytes of 16-bit)
+constexpr int kABytes = kBM * kBK * 2;          // 16 KB dequantized weight slice
+constexpr int kQBytes = kBM * kBK / 2;          // 4 KB packed codes
+constexpr int kQSlot = kQBytes + 2 * kBM * 4;   // codes + up to two groups of scales
+constexpr int kMaxA = 4;
+constexpr int kMaxQ = 8;
+
+template <int NT>
+struct W4Cfg {
+    static constexpr int X_BYTES = NT * kBK * 2;
+    static constexpr bool SPLIT = NT <= 64;     // K split across a cluster
+    static constexpr int RED_BYTES = SPLIT ? (NT + 8) * kBM * 4 : 0;
+    static constexpr int TMEM_COLS = NT < 32 ? 32 : NT;
+};
+
+struct W4Params {
+    int m, n;
+    const float* bias;
+    __nv_bfloat16* y;
+    int64_t ldy;
+    int* status;
+};
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack16x2(float lo, float hi) {
+    if constexpr (BF16) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&v);
+    } else {
+        const __half2 v = __floats2half2_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t*>(&v);
+    }
+}
+
+// Eight codes (one 32-bit word, element i in bits 4i..4i+3) -> eight 16-bit
+// values round16(fl32(s * (nibble - 8))), packed in pairs.
+template <bool BF16>
+__device__ __forceinline__ uint4 dequant8(uint32_t word, float s) {
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const uint32_t b = word >> (8 * e);
+        // 2^23 + nibble, minus 2^23 + 8: the code q as an exact float
+        const float q0 = __fsub_rn(__uint_as_float(0x4B000000u | (b & 15u)), 8388616.0f);
+        const float q1 = __fsub_rn(__uint_as_float(0x4B000000u | ((b >> 4) & 15u)), 8388616.0f);
+        o[e] = pack16x2<BF16>(__fmul_rn(s, q0), __fmul_rn(s, q1));
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <int NT, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
+             const __grid_constant__ CUtensorMap tmX, const W4Params p, int num_kb,
+             int kb_per_split, int splits, int astages, int qstages, int group) {
+    using C = W4Cfg<NT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* a_ring = smem;
+    uint8_t* x_ring = a_ring + astages * kABytes;
+    uint8_t* q_ring = x_ring + astages * C::X_BYTES;
+    uint32_t* red = reinterpret_cast<uint32_t*>(q_ring + qstages * kQSlot);  // [rank][tok][128]
+
+    __shared__ __align__(8) uint64_t q_full[kMaxQ];
+    __shared__ __align__(8) uint64_t q_empty[kMaxQ];
+    __shared__ __align__(8) uint64_t a_full[kMaxA];
+    __shared__ __align__(8) uint64_t a_empty[kMaxA];
+    __shared__ __align__(8) uint64_t tfull_bar;
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const int tn = blockIdx.x;                                  // 128 output channels
+    const int m0 = static_cast<int>(blockIdx.z) * NT;           // first token of the tile
+    const uint32_t rank = splits > 1 ? cluster_ctarank() : 0u;  // split index along K
+    const int kb0 = static_cast<int>(rank) * kb_per_split;
+    const int kb1 = min(num_kb, kb0 + kb_per_split);
+    const int my_kb = kb1 > kb0 ? kb1 - kb0 : 0;
+    const int gps = group < kBK ? kBK / group : 1;             // scale groups per stage
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < qstages; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 4);
+        }
+        for (int s = 0; s < astages; ++s) {
+            mbar_init(&a_full[s], 5);      // 4 dequant warps + the activation TMA's expect_tx
+            mbar_init(&a_empty[s], 1);
+        }
+        mbar_init(&tfull_bar, 1);
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+    pdl_launch_dependents();
+
+    if (warp == 0) {
+        // Codes and scales do not depend on the previous kernel: no wait.
+        if (elect_one()) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmS);
+            int qs = 0;
+            uint32_t qph = 0, issued = 0, last_par = 0;
+            bool ok = true;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                if (!mbar_wait(&q_empty[qs], qph ^ 1, &abort_sh, p.status)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* dst = q_ring + qs * kQSlot;
+                mbar_arrive_expect_tx(&q_full[qs], kQBytes + gps * kBM * 4);
+                tma_load_2d(dst, &tmQ, &q_full[qs], kb * (kBK / 2), tn * kBM);
+                tma_load_2d(dst + kQBytes, &tmS, &q_full[qs], tn * kBM, (kb * kBK) / group);
+                issued |= 1u << qs;
+                last_par = (last_par & ~(1u << qs)) | (qph << qs);
+                if (++qs == qstages) {
+                    qs = 0;
+                    qph ^= 1;
+                }
+            }
+            if (!ok)
+                for (int s = 0; s < qstages; ++s)
+                    if (issued & (1u << s)) mbar_wait(&q_full[s], (last_par >> s) & 1, nullptr, nullptr);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (elect_one()) {
+            const uint32_t idesc = make_idesc(1, BF16 ? 1 : 0, BF16 ? 1 : 0, kBM, NT);
+            int as = 0;
+            uint32_t aph = 0;
+            bool ok = true;
+            for (int i = 0; i < my_kb; ++i) {
+                if (!mbar_wait(&a_full[as], aph, &abort_sh, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t ad = sdesc_kmajor_sw128(smem_addr(a_ring + as * kABytes));
+                const uint64_t bd = sdesc_kmajor_sw128(smem_addr(x_ring + as * C::X_BYTES));
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)   // four K = 16 steps of 32 bytes
+                    mma_issue<kKindF16>(tmem_base, ad + 2 * ks, bd + 2 * ks, idesc, (i | ks) != 0);
+                tc_commit(&a_empty[as]);
+                if (++as == astages) {
+                    as = 0;
+                    aph ^= 1;
+                }
+            }
+            tc_commit(ok ? &tfull_bar : &drain_bar);
+            if (!ok) mbar_wait(&drain_bar, 0, nullptr, nullptr);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- dequantize
+        const int ct = threadIdx.x - 64;           // weight row of the tile
+        const uint32_t a_row = smem_addr(a_ring) + ct * 128;
+        const int sw = ct & 7;
+        pdl_wait();                                // the activations come from the previous kernel
+        int qs = 0, as = 0;
+        uint32_t qph = 0, aph = 0, x_issued = 0, x_par = 0;
+        for (int i = 0; i < my_kb; ++i) {
+            const int kb = kb0 + i;
+            if (!mbar_wait(&q_full[qs], qph, &abort_sh, p.status)) break;
+            if (!mbar_wait(&a_empty[as], aph ^ 1, &abort_sh, p.status)) break;
+            if (ct == 0) {
+                mbar_arrive_expect_tx(&a_full[as], C::X_BYTES);
+                tma_load_2d(x_ring + as * C::X_BYTES, &tmX, &a_full[as], kb * kBK, m0);
+                x_issued |= 1u << as;
+                x_par = (x_par & ~(1u << as)) | (aph << as);
+            }
+            const uint8_t* qsl = q_ring + qs * kQSlot;
+            const uint4 c0 = *reinterpret_cast<const uint4*>(qsl + ct * 32);
+            const uint4 c1 = *reinterpret_cast<const uint4*>(qsl + ct * 32 + 16);
+            const float* ssl = reinterpret_cast<const float*>(qsl + kQBytes);
+            const float s0 = ssl[ct];
+            const float s1 = gps == 2 ? ssl[kBM + ct] : s0;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_empty[qs]);
+            const uint32_t dst = a_row + as * kABytes;
+            const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const uint4 v = dequant8<BF16>(w[c], c < 4 ? s0 : s1);
+                st_shared_v4(dst + ((c ^ sw) << 4), v.x, v.y, v.z, v.w);
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&a_full[as]);
+            if (++qs == qstages) {
+                qs = 0;
+                qph ^= 1;
+            }
+            if (++as == astages) {
+                as = 0;
+                aph ^= 1;
+            }
+        }
+        if (abort_sh && ct == 0)   // let the activation loads already issued land
+            for (int s = 0; s < astages; ++s)
+                if (x_issued & (1u << s)) mbar_wait(&a_full[s], (x_par >> s) & 1, nullptr, nullptr);
+
+        // ---------------- epilogue
+        const int q = warp & 3;                    // TMEM lane quarter of this warp
+        const int ch = q * 32 + lane;
+        const int n = tn * kBM + ch;
+        const bool col_ok = n < p.n;
+        const float bias = (col_ok && p.bias) ? p.bias[n] : 0.f;
+        const bool have = my_kb > 0 && mbar_wait(&tfull_bar, 0, &abort_sh, p.status);
+        if (have) tc_fence_after();
+        __syncwarp();
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+        if (splits == 1) {
+            for (int c = 0; c < NT && m0 + c < p.m; c += 16) {
+                uint32_t r[16];
+                tmem_ld16(tb + c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int t = m0 + c + i;
+                    if (have && col_ok && t < p.m) {
+                        float v = __uint_as_float(r[i]);
+                        if (p.bias) v = __fadd_rn(v, bias);
+                        p.y[static_cast<int64_t>(t) * p.ldy + n] = __float2bfloat16_rn(v);
+                    }
+                }
+            }
+        } else if constexpr (C::SPLIT) {
+            // Push this rank's partial of token t to rank t % splits, slot
+            // [rank][t / splits][channel].
+            const int tpo = (NT + splits - 1) / splits;
+            const uint32_t red_base = smem_addr(red);
+#pragma unroll
+            for (int c = 0; c < NT; c += 16) {
+                uint32_t r[16];
+                tmem_ld16(tb + c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int t = c + i;
+                    const uint32_t owner = static_cast<uint32_t>(t % splits);
+                    const uint32_t off = ((rank * tpo + t / splits) * kBM + ch) * 4u;
+                    st_shared_cluster_u32(map_shared_rank(red_base + off, owner), have ? r[i] : 0u);
+                }
+            }
+        }
+        __syncwarp();
+    }
+
+    if constexpr (C::SPLIT) {
+        if (splits > 1) {
+            __syncthreads();
+            cluster_sync();
+            if (warp >= 2) {
+                const int q = warp & 3;
+                const int ch = q * 32 + lane;
+                const int n = tn * kBM + ch;
+                const int tpo = (NT + splits - 1) / splits;
+                if (n < p.n) {
+                    const float bias = p.bias ? p.bias[n] : 0.f;
+                    for (int t = static_cast<int>(rank); t < NT && m0 + t < p.m; t += splits) {
+                        const int tl = t / splits;
+                        float s = 0.f;
+                        for (int r = 0; r < splits; ++r)
+                            s = __fadd_rn(s, __uint_as_float(red[(r * tpo + tl) * kBM + ch]));
+                        if (p.bias) s = __fadd_rn(s, bias);
+                        p.y[static_cast<int64_t>(m0 + t) * p.ldy + n] = __float2bfloat16_rn(s);
+                    }
+                }
+            }
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ============================================================================
+// Host side
+// ============================================================================
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                uint64_t outer, uint64_t ld_bytes, uint32_t box_inner, uint32_t box_outer,
+                CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {ld_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+template <int NT, bool BF16>
+q8_status run_w4(const W4Args& a, cudaStream_t s) {
+    using C = W4Cfg<NT>;
+    CUtensorMap tQ, tS, tX;
+    const int gps = a.group < kBK ? kBK / a.group : 1;
+    if (!make_map2d(&tQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.codes, a.k / 2, a.n, a.ldc, kBK / 2, kBM,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map2d(&tS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.scale, a.n, a.k / a.group, a.n * 4, kBM,
+                    gps, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map2d(&tX, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                    a.x, a.k, a.m, a.ldx * 2, kBK, NT, CU_TENSOR_MAP_SWIZZLE_128B))
+        return Q8_ERR_CUDA;
+    const int tiles_n = static_cast<int>((a.n + kBM - 1) / kBM);
+    const int tiles_m = static_cast<int>((a.m + NT - 1) / NT);
+    const int num_kb = static_cast<int>((a.k + kBK - 1) / kBK);
+    int splits = 1, per = num_kb;
+    int astages, qstages;
+    if constexpr (C::SPLIT) {
+        // Split K over a cluster (at most 8, every split non-empty) so that the
+        // grid fills the SMs at two CTAs per SM.
+        int want = 2 * sm_count() / (tiles_n * tiles_m);
+        if (want < 1) want = 1;
+        if (want > 8) want = 8;
+        if (want > num_kb) want = num_kb;
+        per = (num_kb + want - 1) / want;
+        splits = (num_kb + per - 1) / per;
+        astages = NT == 64 ? 4 : 3;
+        qstages = NT == 16 ? 8 : NT == 32 ? 6 : 8;
+    } else {
+        astages = NT == 128 ? 4 : 3;
+        qstages = 8;
+    }
+    if (astages > per) astages = per;
+    if (qstages > per) qstages = per;
+    const int smem = astages * (kABytes + C::X_BYTES) + qstages * kQSlot + C::RED_BYTES + 1024;
+
+    auto kern = w4a16_kernel<NT, BF16>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    W4Params p;
+    p.m = static_cast<int>(a.m);
+    p.n = static_cast<int>(a.n);
+    p.bias = a.bias;
+    p.y = a.y;
+    p.ldy = a.ldy;
+    p.status = device_status_ptr();
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_n), static_cast<unsigned>(splits),
+                       static_cast<unsigned>(tiles_m));
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+    if (splits > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 1;
+        attr[na].val.clusterDim.y = static_cast<unsigned>(splits);
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    if (cudaLaunchKernelEx(&cfg, kern, tQ, tS, tX, p, num_kb, per, splits, astages, qstages,
+                           a.group) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    return Q8_OK;
+}
+
+template <bool BF16>
+q8_status dispatch_w4(const W4Args& a, cudaStream_t s) {
+    if (a.m <= 16) return run_w4<16, BF16>(a, s);
+    if (a.m <= 32) return run_w4<32, BF16>(a, s);
+    if (a.m <= 64) return run_w4<64, BF16>(a, s);
+    if (a.m <= 128) return run_w4<128, BF16>(a, s);
+    return run_w4<256, BF16>(a, s);
+}
+
+}  // namespace
+
+cudaError_t launch_group_quant(const void* W, q8_dtype dt, int64_t n, int64_t k, int64_t ldw,
+                               int group, uint8_t* codes, int64_t ldc, float* scale,
+                               cudaStream_t s) {
+    const int64_t groups = n * (k / group);
+    if (groups == 0) return cudaSuccess;
+    const unsigned blocks = static_cast<unsigned>((groups + 255) / 256);
+    if (dt == Q8_F16)
+        group_quant_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), n, k, ldw,
+                                                         group, codes, ldc, scale);
+    else
+        group_quant_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(W), n, k, ldw, group, codes, ldc, scale);
+    return cudaGetLastError();
+}
+
+q8_status launch_w4a16(const W4Args& a, cudaStream_t s) {
+    if (a.m == 0 || a.n == 0) return Q8_OK;
+    return a.x_bf16 ? dispatch_w4<true>(a, s) : dispatch_w4<false>(a, s);
+}
+
+}  // namespace q8

@@ -41,6 +41,7 @@ EXPORTED = [
     "q8_outlier_quantize_act",
     "q8_linear_w8a8", "q8_linear_w8a8_requant", "q8_linear_w8a8_dynamic", "q8_linear_int8_mixed",
     "q8_linear_int8_mixed_noalloc",
+    "q8_quantize_weight_g4", "q8_linear_w4a16",
     "q8_workspace_size", "q8_status_string",
     "q8_get_device_status", "q8_clear_device_status", "q8_device_check", "q8_version",
 ]
@@ -56,6 +57,12 @@ class CAct(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("code_dtype", ctypes.c_int),
                 ("scale", ctypes.c_void_p), ("rowsum", ctypes.c_void_p),
                 ("m", ctypes.c_int64), ("k", ctypes.c_int64), ("ld", ctypes.c_int64)]
+
+
+class CWeightG4(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scale", ctypes.c_void_p),
+                ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("ld", ctypes.c_int64),
+                ("group", ctypes.c_int32)]
 
 
 _i64, _int, _f, _vp, _sz = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
@@ -77,6 +84,10 @@ _SIG = {
                               _vp, _i64, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _int),
     "q8_linear_int8_mixed_noalloc": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeight), _vp,
                                       _f, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp], _int),
+    "q8_quantize_weight_g4": ([_vp, _int, _i64, _i64, _i64, ctypes.c_int32, _vp, _i64, _vp, _vp],
+                              _int),
+    "q8_linear_w4a16": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeightG4), _vp, _vp, _i64,
+                         _vp], _int),
     "q8_workspace_size": ([_int, _i64, _i64, _i64], _sz),
     "q8_status_string": ([_int], ctypes.c_char_p),
     "q8_get_device_status": ([_vp, _vp], _int),
@@ -364,6 +375,54 @@ def q8_linear_int8_mixed(X: torch.Tensor, w: QWeight, threshold: float = 6.0,
         _ptr(dbg["acc"]) if dbg else None, _ptr(dbg["y16"]) if dbg else None,
         _ptr(workspace), workspace.numel(), _stream(stream)), "q8_linear_int8_mixed")
     return (out, dbg) if debug else out
+
+
+@dataclasses.dataclass
+class QWeightG4:
+    """A group-wise 4-bit weight (device tensors): codes n x k/2 uint8 (two
+    nibbles q + 8 per byte, low nibble first), scale (k/group) x n fp32."""
+    codes: torch.Tensor
+    scale: torch.Tensor
+    group: int
+
+    @property
+    def n(self) -> int:
+        return self.codes.shape[0]
+
+    @property
+    def k(self) -> int:
+        return self.scale.shape[0] * self.group
+
+    def c(self) -> CWeightG4:
+        return CWeightG4(self.codes.data_ptr(), self.scale.data_ptr(), self.n, self.k,
+                         self.codes.stride(0), self.group)
+
+
+def q8_quantize_weight_g4(W: torch.Tensor, group: int = 128, stream=None) -> QWeightG4:
+    """Group-wise symmetric 4-bit weight quantization (see q8_quantize_weight_g4 in q8.h)."""
+    _cuda(W, "W")
+    n, k = W.shape
+    codes = torch.empty((n, k // 2), dtype=torch.uint8, device=W.device)
+    scale = torch.empty((max(k // group, 1) if k % group == 0 else 1, n), dtype=torch.float32,
+                        device=W.device)
+    _check(_lib.q8_quantize_weight_g4(_ptr(W), _FLOAT_DT.get(W.dtype, -1), n, k, W.stride(0),
+                                      int(group), _ptr(codes), codes.stride(0), _ptr(scale),
+                                      _stream(stream)), "q8_quantize_weight_g4")
+    return QWeightG4(codes, scale, int(group))
+
+
+def q8_linear_w4a16(X: torch.Tensor, w: QWeightG4, bias: Optional[torch.Tensor] = None,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """W4A16 linear: bf16/fp16 X times the group-wise 4-bit weight; bf16 M x N output."""
+    _cuda(X, "X")
+    m, k = X.shape
+    if out is None:
+        out = torch.empty((m, w.n), dtype=torch.bfloat16, device=X.device)
+    cw = w.c()
+    _check(_lib.q8_linear_w4a16(_ptr(X), _FLOAT_DT.get(X.dtype, -1), m, k, X.stride(0),
+                                ctypes.byref(cw), _ptr(bias), _ptr(out), out.stride(0),
+                                _stream(stream)), "q8_linear_w4a16")
+    return out
 
 
 def q8_get_device_status(stream=None) -> int:

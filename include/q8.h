@@ -9,7 +9,9 @@
  *   - the LLM.int8 mixed decomposition (outlier feature columns in fp16);
  *   - around it: activations with a static (calibrated) scale, smoothed
  *     activations (SmoothQuant-style per-column multipliers), and a W8A8 linear
- *     that re-quantizes its output to INT8 for the next layer.
+ *     that re-quantizes its output to INT8 for the next layer;
+ *   - group-wise 4-bit weights with one absmax scale per group of 32-128
+ *     values along K, multiplied with 16-bit activations (W4A16).
  *
  * Notation follows the pages' linear map Q = round(R / S) + Z, R = S (Q - Z):
  * `scale` is S, the dequant multiplier, and `zero_point` is Z, an integer held
@@ -18,7 +20,8 @@
  *   [CSDN]     "大模型量化技术" overview (devpress.csdn.net), sections 2.1-2.3
  *   [FBGEMM]   "Transformers FP8 (W8A8) 量化实战：基于 FBGEMM", sections 5.1-5.3, 6
  *   [LLM.int8] "Transformers 单 GPU 高效推理：bitsandbytes LLM.int8 8-bit 混合精度量化"
- *   [Xilyfe]   "大模型量化" (xilyfe.github.io): symmetric, asymmetric, INT32 accumulator
+ *   [Xilyfe]   "大模型量化" (xilyfe.github.io): symmetric, asymmetric, INT32 accumulator,
+ *              GGUF block quantization
  *
  * Conventions shared by every entry point
  *   Layout      all matrices are row-major 2-D: X is M x K (tokens x features),
@@ -61,7 +64,7 @@
 extern "C" {
 #endif
 
-#define Q8_VERSION 3
+#define Q8_VERSION 4
 
 /* Same object as cudaStream_t. */
 typedef struct CUstream_st *q8_stream_t;
@@ -281,6 +284,62 @@ q8_status q8_linear_w8a8(const q8_act *x, const q8_weight *w, const float *bias,
 q8_status q8_linear_w8a8_requant(const q8_act *x, const q8_weight *w, const float *bias,
                                  float out_scale, void *Yq, int64_t ldy, void *acc_debug,
                                  q8_stream_t stream);
+
+/* A group-wise 4-bit weight: n x k values, one fp32 scale per group of
+ * `group` consecutive values along K ([CSDN] 2.2 granularity table: one scale
+ * per group of 64-128 parameters; [Xilyfe] GGUF section: each block of a row
+ * has its own absmax scale).  Dequantized value: scale * (nibble - 8).
+ *   codes   n x k/2 bytes, row stride ld bytes (ld >= k/2, ld % 16 == 0);
+ *           byte j of a row holds element 2j in its low nibble and element
+ *           2j+1 in its high nibble, each as q + 8 with q in [-7, 7].
+ *   scale   (k / group) x n fp32, GROUP-major: scale[j * n + r] belongs to row
+ *           r, elements j*group .. j*group + group - 1.
+ *   group   32, 64 or 128; k % group == 0. */
+typedef struct {
+    const void *codes;
+    const float *scale;
+    int64_t n, k, ld;
+    int32_t group;
+} q8_weight_g4;
+
+/*
+ * Group-wise symmetric 4-bit weight quantization ([Xilyfe] GGUF section:
+ * s = absmax / 7 per block, codes round(w / s); [CSDN] 2.2 group granularity).
+ * For each row r and group j: S = fl32(max |w| / 7), floored at 1e-8;
+ * q = clamp(rne(fl32(w / S)), -7, 7).  Bit-exact with a scalar reference.
+ *
+ *   W       device, n x k, Q8_F16 or Q8_BF16, row stride ldw (elements).
+ *   group   32, 64 or 128 (Q8_ERR_SCHEME otherwise); k % group == 0 and
+ *           k % 32 == 0, n % 16 == 0 (Q8_ERR_SHAPE).
+ *   codes   device output, n x k/2 bytes, row stride ldc bytes (ldc >= k/2,
+ *           ldc % 16 == 0), layout of q8_weight_g4.
+ *   scale   device output, (k / group) x n fp32, group-major.
+ * One launch; offline (once per weight).
+ */
+q8_status q8_quantize_weight_g4(const void *W, q8_dtype w_dtype, int64_t n, int64_t k,
+                                int64_t ldw, int32_t group, void *codes, int64_t ldc,
+                                float *scale, q8_stream_t stream);
+
+/*
+ * W4A16 linear: Y = X W~^T (+ bias), W~ the group-wise 4-bit weight brought
+ * back to the activation's 16-bit format.  The weight of each K slice is
+ * dequantized in shared memory, w~ = round16(fl32(S * q)), and multiplied on
+ * the tensor cores with fp32 accumulation; y = fl32(y + bias[n]); Y = bf16(y).
+ * The fp32 accumulation order is not specified (results agree with an exact
+ * sum of the same w~ within the fp32 accumulation bound).
+ *
+ *   X       device, m x k activations, Q8_BF16 or Q8_F16 (Q8_ERR_DTYPE
+ *           otherwise), row stride ldx (elements, 16-byte multiple).
+ *   w       group-wise weight with w->k == k (Q8_ERR_SHAPE otherwise).
+ *   bias    device [w->n] fp32, or NULL.
+ *   Y       device, m x w->n bf16, row stride ldy (ldy % 8 == 0).
+ * One launch.  It may start before the previous kernel on `stream` has ended
+ * (programmatic dependent launch) and waits for it before reading X or
+ * writing Y.
+ */
+q8_status q8_linear_w4a16(const void *X, q8_dtype x_dtype, int64_t m, int64_t k, int64_t ldx,
+                          const q8_weight_g4 *w, const float *bias, void *Y, int64_t ldy,
+                          q8_stream_t stream);
 
 /*
  * Dynamic per-token activation quantization and the W8A8 linear in one call:

@@ -239,3 +239,53 @@ def test_quantize_act_smooth_validation():
     assert qsm(m=0, X=None, mult=None) == q8.Q8_OK               # empty call
     if NO_GPU:
         assert qsm() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def qg4(W=FAKE, dt=q8.Q8_BF16, n=256, k=512, ldw=512, group=128, codes=FAKE, ldc=256, sc=FAKE):
+    return L.q8_quantize_weight_g4(W, dt, n, k, ldw, group, codes, ldc, sc, _ns)
+
+
+def test_quantize_weight_g4_validation():
+    assert qg4(W=None) == q8.Q8_ERR_NULL
+    assert qg4(sc=None) == q8.Q8_ERR_NULL
+    assert qg4(dt=q8.Q8_F32) == q8.Q8_ERR_DTYPE
+    for bad in (16, 48, 256):
+        assert qg4(group=bad) == q8.Q8_ERR_SCHEME
+    assert qg4(k=480, ldw=480) == q8.Q8_ERR_SHAPE               # k % group
+    assert qg4(n=200) == q8.Q8_ERR_SHAPE                         # n % 16
+    assert qg4(ldc=128) == q8.Q8_ERR_SHAPE                       # ldc < k / 2
+    assert qg4(ldc=264) == q8.Q8_ERR_ALIGN                       # ldc % 16
+    assert qg4(codes=MIS) == q8.Q8_ERR_ALIGN
+    assert qg4(n=0, W=None, codes=None, sc=None) == q8.Q8_OK      # empty call
+    if NO_GPU:
+        assert qg4() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def _wg4(n=256, k=512, ld=256, group=64, codes=FAKE, scale=FAKE):
+    return q8.CWeightG4(codes, scale, n, k, ld, group)
+
+
+def lw4(X=FAKE, dt=q8.Q8_BF16, m=16, k=512, ldx=512, w=None, bias=None, Y=FAKE, ldy=256):
+    w = w or _wg4()
+    return L.q8_linear_w4a16(X, dt, m, k, ldx, ctypes.byref(w), bias, Y, ldy, _ns)
+
+
+def test_linear_w4a16_validation():
+    assert L.q8_linear_w4a16(FAKE, q8.Q8_BF16, 16, 512, 512, None, None, FAKE, 256, _ns) == q8.Q8_ERR_NULL
+    assert lw4(Y=None) == q8.Q8_ERR_NULL
+    assert lw4(w=_wg4(scale=None)) == q8.Q8_ERR_NULL
+    assert lw4(dt=q8.Q8_S8) == q8.Q8_ERR_DTYPE
+    assert lw4(dt=q8.Q8_F32) == q8.Q8_ERR_DTYPE
+    assert lw4(w=_wg4(group=96)) == q8.Q8_ERR_SCHEME
+    assert lw4(k=256, ldx=256) == q8.Q8_ERR_SHAPE                # k != w.k
+    assert lw4(w=_wg4(ld=128)) == q8.Q8_ERR_SHAPE                # ld < k / 2
+    assert lw4(w=_wg4(n=200, ld=256)) == q8.Q8_ERR_SHAPE         # n % 16
+    assert lw4(ldy=128) == q8.Q8_ERR_SHAPE                       # ldy < n
+    assert lw4(m=65535 * 256 + 1) == q8.Q8_ERR_SHAPE
+    assert lw4(ldy=260) == q8.Q8_ERR_ALIGN
+    assert lw4(X=MIS) == q8.Q8_ERR_ALIGN
+    assert lw4(bias=MIS) == q8.Q8_ERR_ALIGN
+    assert lw4(w=_wg4(ld=264)) == q8.Q8_ERR_ALIGN
+    assert lw4(m=0, X=None, Y=None) == q8.Q8_OK                  # empty call
+    if NO_GPU:
+        assert lw4() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)

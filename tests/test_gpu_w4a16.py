@@ -1,0 +1,120 @@
+"""GPU parity of the group-wise 4-bit weight quantizer and the W4A16 linear.
+
+Codes and scales are compared bit for bit with the oracle.  Outputs are
+compared with the oracle's double-accumulated product of the same 16-bit
+dequantized weight within the fp32-accumulation bound of tests/parity.py:
+    |Y - y_ref| <= 2 ulp_bf16(y_ref) + K 2^-22 (|x| |w~|^T)[m, n]
+Shapes cover every token tile (16, 32, 64, 128, 256), K split across a
+cluster and not, a half-filled last K slice (K = 96 with groups of 32),
+ragged token and channel tails, both 16-bit activation formats, and the
+q_proj-sized decode case in full.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import oracle as O
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+from bit_quantized_b200 import q8  # noqa: E402
+
+DEV = "cuda:0"
+
+
+def _unpack(codes: torch.Tensor) -> np.ndarray:
+    b = codes.cpu().numpy().astype(np.int16)
+    q = np.empty((b.shape[0], 2 * b.shape[1]), np.int16)
+    q[:, 0::2] = (b & 15) - 8
+    q[:, 1::2] = (b >> 4) - 8
+    return q.astype(np.int8)
+
+
+def _quant_case(W: torch.Tensor, g: int, what: str):
+    w32 = P.host_f32(W)
+    qw = q8.q8_quantize_weight_g4(W.to(DEV), g)
+    torch.cuda.synchronize()
+    q_ref, S_ref = O.quant_weight_group(w32, g)
+    P.assert_equal(_unpack(qw.codes), q_ref, what + " codes")
+    P.assert_equal(qw.scale.cpu().numpy().T, S_ref, what + " scales")
+    return qw, w32, q_ref, S_ref
+
+
+@pytest.mark.parametrize("n,k,g,dt", [(256, 512, 32, torch.bfloat16),
+                                      (272, 384, 128, torch.float16),
+                                      (48, 96, 32, torch.bfloat16),
+                                      (4096, 4096, 128, torch.bfloat16)])
+def test_group_quant_bit_exact(n, k, g, dt):
+    W = workloads.random_matrix(n, k, dt, seed=n + k + g, std=0.02)
+    _quant_case(W, g, f"{n}x{k} g{g}")
+
+
+def test_group_quant_ties_zero_groups_and_saturation():
+    k, g = 128, 32
+    W = torch.zeros(16, k)
+    W[0, :32] = torch.tensor([7.0, 3.5, -3.5, 2.5, 0.5, -0.5, 1.5] + [0.0] * 25)   # S = 1, ties
+    W[1, 32:64] = torch.linspace(-1.0, 1.0, 32)
+    W[2, 64:96] = 3.0e4                         # one value repeated: every code 7
+    W[3, 96:] = -1.0e-9                         # below the eps floor: S = 1e-8, codes -0 -> 0
+    qw, _, q_ref, S_ref = _quant_case(W.to(torch.bfloat16), g, "ties")
+    assert q_ref[0, :7].tolist() == [7, 4, -4, 2, 0, 0, 2]
+
+
+def _linear_case(m, n, k, g, dt, seed, bias=False, what=""):
+    X = workloads.random_matrix(m, k, dt, seed)
+    W = workloads.random_matrix(n, k, dt, seed + 1, std=0.02)
+    qw, w32, q_ref, S_ref = _quant_case(W, g, what)
+    x32 = P.host_f32(X)
+    b = (np.random.default_rng(seed).standard_normal(n) * 0.1).astype(np.float32) if bias else None
+    Y = q8.q8_linear_w4a16(X.to(DEV), qw, bias=None if b is None else torch.from_numpy(b).to(DEV))
+    torch.cuda.synchronize()
+    assert q8.q8_get_device_status() == 0
+    fmt = P.FMT[dt]
+    y_ref, _ = O.linear_w4a16(x32, q_ref, S_ref, g, fmt, bias=b)
+    wd = O.widen16(O.dequant_group16(q_ref, S_ref, g, fmt), fmt).astype(np.float64)
+    extra = k * 2.0 ** -22 * (np.abs(x32.astype(np.float64)) @ np.abs(wd).T)
+    return P.assert_bf16_within(P.bf16_bits(Y), y_ref, extra, what)
+
+
+@pytest.mark.parametrize("m,n,k,g,dt", [
+    (1, 256, 512, 64, torch.bfloat16),       # one token, K split
+    (3, 208, 160, 32, torch.bfloat16),       # ragged channels and a half K slice
+    (16, 384, 96, 32, torch.float16),        # two K slices, the second half empty
+    (30, 512, 1024, 128, torch.bfloat16),    # token tile 32
+    (40, 272, 512, 64, torch.float16),       # token tile 64, ragged channels
+    (100, 256, 512, 32, torch.bfloat16),     # token tile 128, no split
+    (300, 384, 256, 128, torch.float16),     # two token tiles of 256, ragged
+])
+def test_linear_w4a16_shapes(m, n, k, g, dt):
+    _linear_case(m, n, k, g, dt, seed=m * 7 + n, bias=(m % 2 == 0), what=f"{m}x{n}x{k} g{g}")
+
+
+def test_linear_w4a16_decode_q_proj_full():
+    # The decode weight recipe at q_proj size, 16 tokens, groups of 128.
+    X, W, _ = workloads.make_inputs("decode_q_proj")
+    qw, w32, q_ref, S_ref = _quant_case(W, 128, "decode weights")
+    x32 = P.host_f32(X)
+    Y = q8.q8_linear_w4a16(X.to(DEV), qw)
+    torch.cuda.synchronize()
+    y_ref, _ = O.linear_w4a16(x32, q_ref, S_ref, 128, "bf16")
+    wd = O.widen16(O.dequant_group16(q_ref, S_ref, 128, "bf16"), "bf16").astype(np.float64)
+    extra = 4096 * 2.0 ** -22 * (np.abs(x32.astype(np.float64)) @ np.abs(wd).T)
+    P.assert_bf16_within(P.bf16_bits(Y), y_ref, extra, "decode w4a16")
+
+
+def test_linear_w4a16_after_producer_kernel():
+    # X written by the kernel just before the linear on the same stream: the
+    # linear's early start must still read the finished X.
+    m, n, k, g = 16, 512, 1024, 64
+    W = workloads.random_matrix(n, k, torch.bfloat16, 5, std=0.02)
+    qw = q8.q8_quantize_weight_g4(W.to(DEV), g)
+    X0 = workloads.random_matrix(m, k, torch.bfloat16, 6).to(DEV)
+    for _ in range(3):
+        X = X0 * 2.0                            # producer kernel
+        Y = q8.q8_linear_w4a16(X, qw)
+    Y_sep = q8.q8_linear_w4a16(X0 * 2.0, qw)
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), Y_sep.view(torch.int16))
+    assert q8.q8_get_device_status() == 0
