@@ -102,16 +102,19 @@ constexpr int kBM = 128;                        // weight rows per CTA (MMA M)
 constexpr int kBK = 64;                         // K elements per stage (128 bytes of 16-bit)
 constexpr int kABytes = kBM * kBK * 2;          // 16 KB dequantized weight slice
 constexpr int kQBytes = kBM * kBK / 2;          // 4 KB packed codes
-constexpr int kQSlot = kQBytes + 2 * kBM * 4;   // codes + up to two groups of scales
+constexpr int kSBytes = 2 * kBM * 4;            // room for two groups of scales
 constexpr int kMaxA = 4;
 constexpr int kMaxQ = 8;
 
+// Staging slot of one K slice: [activation tile, 128-byte swizzled][codes][scales].
 template <int NT>
 struct W4Cfg {
     static constexpr int X_BYTES = NT * kBK * 2;
+    static constexpr int QSLOT = X_BYTES + kQBytes + kSBytes;
     static constexpr bool SPLIT = NT <= 64;     // K split across a cluster
     static constexpr int RED_BYTES = SPLIT ? (NT + 8) * kBM * 4 : 0;
     static constexpr int TMEM_COLS = NT < 32 ? 32 : NT;
+    static_assert(QSLOT % 1024 == 0, "staging slots keep 1024-byte alignment");
 };
 
 struct W4Params {
@@ -144,18 +147,34 @@ __device__ __forceinline__ uint32_t pack16x2(float lo, float hi) {
     }
 }
 
-// Eight codes (one 32-bit word, element i in bits 4i..4i+3) -> eight 16-bit
-// values round16(fl32(s * (nibble - 8))), packed in pairs.
+__device__ __forceinline__ uint64_t pair(uint32_t lo, uint32_t hi) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "r"(lo), "r"(hi));
+    return v;
+}
+
+// Eight codes (one 32-bit word; byte e holds element 2e in its low nibble and
+// 2e+1 in its high nibble) -> eight 16-bit values round16(fl32(s * q)),
+// q = nibble - 8, packed in element order.  `s2` holds s twice.
+//   The float with bits 0x4B0000nn is 2^23 + nn; subtracting 2^23 + 8 leaves q
+//   exactly.  Both lanes of each f32x2 step round to nearest like the scalar
+//   operations, so the products are fl32(s * q).
 template <bool BF16>
-__device__ __forceinline__ uint4 dequant8(uint32_t word, float s) {
+__device__ __forceinline__ uint4 dequant8(uint32_t word, uint64_t s2) {
+    const uint32_t lo = word & 0x0F0F0F0Fu;          // elements 0, 2, 4, 6
+    const uint32_t hi = (word >> 4) & 0x0F0F0F0Fu;   // elements 1, 3, 5, 7
+    const uint64_t magic = 0x4B0000084B000008ull;    // {2^23 + 8, 2^23 + 8}
     uint32_t o[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const uint32_t b = word >> (8 * e);
-        // 2^23 + nibble, minus 2^23 + 8: the code q as an exact float
-        const float q0 = __fsub_rn(__uint_as_float(0x4B000000u | (b & 15u)), 8388616.0f);
-        const float q1 = __fsub_rn(__uint_as_float(0x4B000000u | ((b >> 4) & 15u)), 8388616.0f);
-        o[e] = pack16x2<BF16>(__fmul_rn(s, q0), __fmul_rn(s, q1));
+        const uint32_t sel = 0x7540u | static_cast<uint32_t>(e);   // byte e, 0, 0, 0x4B
+        const uint64_t v = pair(__byte_perm(lo, 0x4B000000u, sel), __byte_perm(hi, 0x4B000000u, sel));
+        uint64_t q, r;
+        asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(q) : "l"(v), "l"(magic));
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(q), "l"(s2));
+        uint32_t f0, f1;
+        asm("mov.b64 {%0, %1}, %2;" : "=r"(f0), "=r"(f1) : "l"(r));
+        o[e] = pack16x2<BF16>(__uint_as_float(f0), __uint_as_float(f1));
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
@@ -170,14 +189,14 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* a_ring = smem;
-    uint8_t* x_ring = a_ring + astages * kABytes;
-    uint8_t* q_ring = x_ring + astages * C::X_BYTES;
-    uint32_t* red = reinterpret_cast<uint32_t*>(q_ring + qstages * kQSlot);  // [rank][tok][128]
+    uint8_t* q_ring = a_ring + astages * kABytes;
+    uint32_t* red = reinterpret_cast<uint32_t*>(q_ring + qstages * C::QSLOT);  // [rank][tok][128]
 
-    __shared__ __align__(8) uint64_t q_full[kMaxQ];
-    __shared__ __align__(8) uint64_t q_empty[kMaxQ];
-    __shared__ __align__(8) uint64_t a_full[kMaxA];
-    __shared__ __align__(8) uint64_t a_empty[kMaxA];
+    __shared__ __align__(8) uint64_t q_full[kMaxQ];    // codes + scales landed
+    __shared__ __align__(8) uint64_t x_full[kMaxQ];    // activation tile landed
+    __shared__ __align__(8) uint64_t q_empty[kMaxQ];   // slot consumed by the MMAs
+    __shared__ __align__(8) uint64_t a_full[kMaxA];    // 16-bit weight slice written
+    __shared__ __align__(8) uint64_t a_empty[kMaxA];   // weight slice consumed
     __shared__ __align__(8) uint64_t tfull_bar;
     __shared__ __align__(8) uint64_t drain_bar;
     __shared__ uint32_t tmem_base_sh;
@@ -192,14 +211,16 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     const int kb1 = min(num_kb, kb0 + kb_per_split);
     const int my_kb = kb1 > kb0 ? kb1 - kb0 : 0;
     const int gps = group < kBK ? kBK / group : 1;             // scale groups per stage
+    const uint32_t qs_tx = kQBytes + gps * kBM * 4;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < qstages; ++s) {
             mbar_init(&q_full[s], 1);
-            mbar_init(&q_empty[s], 4);
+            mbar_init(&x_full[s], 1);
+            mbar_init(&q_empty[s], 1);
         }
         for (int s = 0; s < astages; ++s) {
-            mbar_init(&a_full[s], 5);      // 4 dequant warps + the activation TMA's expect_tx
+            mbar_init(&a_full[s], 4);      // one arrival per dequantizing warp
             mbar_init(&a_empty[s], 1);
         }
         mbar_init(&tfull_bar, 1);
@@ -218,22 +239,41 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
     pdl_launch_dependents();
 
     if (warp == 0) {
-        // Codes and scales do not depend on the previous kernel: no wait.
         if (elect_one()) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmS);
-            int qs = 0;
-            uint32_t qph = 0, issued = 0, last_par = 0;
+            tma_prefetch_desc(&tmX);
+            // Codes and scales do not depend on the previous kernel: the first
+            // ring of them goes out before the programmatic-launch wait, the
+            // activation tiles of the same slots right after it.
+            const int first = my_kb < qstages ? my_kb : qstages;
+            for (int i = 0; i < first; ++i) {
+                uint8_t* dst = q_ring + i * C::QSLOT;
+                mbar_arrive_expect_tx(&q_full[i], qs_tx);
+                tma_load_2d(dst + C::X_BYTES, &tmQ, &q_full[i], (kb0 + i) * (kBK / 2), tn * kBM);
+                tma_load_2d(dst + C::X_BYTES + kQBytes, &tmS, &q_full[i], tn * kBM,
+                            ((kb0 + i) * kBK) / group);
+            }
+            pdl_wait();
+            for (int i = 0; i < first; ++i) {
+                mbar_arrive_expect_tx(&x_full[i], C::X_BYTES);
+                tma_load_2d(q_ring + i * C::QSLOT, &tmX, &x_full[i], (kb0 + i) * kBK, m0);
+            }
+            uint32_t issued = (1u << first) - 1u, last_par = 0;
+            int qs = first == qstages ? 0 : first;
+            uint32_t qph = first == qstages ? 1u : 0u;
             bool ok = true;
-            for (int kb = kb0; kb < kb1; ++kb) {
+            for (int kb = kb0 + first; kb < kb1; ++kb) {
                 if (!mbar_wait(&q_empty[qs], qph ^ 1, &abort_sh, p.status)) {
                     ok = false;
                     break;
                 }
-                uint8_t* dst = q_ring + qs * kQSlot;
-                mbar_arrive_expect_tx(&q_full[qs], kQBytes + gps * kBM * 4);
-                tma_load_2d(dst, &tmQ, &q_full[qs], kb * (kBK / 2), tn * kBM);
-                tma_load_2d(dst + kQBytes, &tmS, &q_full[qs], tn * kBM, (kb * kBK) / group);
+                uint8_t* dst = q_ring + qs * C::QSLOT;
+                mbar_arrive_expect_tx(&q_full[qs], qs_tx);
+                tma_load_2d(dst + C::X_BYTES, &tmQ, &q_full[qs], kb * (kBK / 2), tn * kBM);
+                tma_load_2d(dst + C::X_BYTES + kQBytes, &tmS, &q_full[qs], tn * kBM, (kb * kBK) / group);
+                mbar_arrive_expect_tx(&x_full[qs], C::X_BYTES);
+                tma_load_2d(dst, &tmX, &x_full[qs], kb * kBK, m0);
                 issued |= 1u << qs;
                 last_par = (last_par & ~(1u << qs)) | (qph << qs);
                 if (++qs == qstages) {
@@ -243,30 +283,39 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             }
             if (!ok)
                 for (int s = 0; s < qstages; ++s)
-                    if (issued & (1u << s)) mbar_wait(&q_full[s], (last_par >> s) & 1, nullptr, nullptr);
+                    if (issued & (1u << s)) {
+                        mbar_wait(&q_full[s], (last_par >> s) & 1, nullptr, nullptr);
+                        mbar_wait(&x_full[s], (last_par >> s) & 1, nullptr, nullptr);
+                    }
         }
         __syncwarp();
     } else if (warp == 1) {
         if (elect_one()) {
             const uint32_t idesc = make_idesc(1, BF16 ? 1 : 0, BF16 ? 1 : 0, kBM, NT);
-            int as = 0;
-            uint32_t aph = 0;
+            int as = 0, qs = 0;
+            uint32_t aph = 0, qph = 0;
             bool ok = true;
             for (int i = 0; i < my_kb; ++i) {
-                if (!mbar_wait(&a_full[as], aph, &abort_sh, p.status)) {
+                if (!mbar_wait(&a_full[as], aph, &abort_sh, p.status) ||
+                    !mbar_wait(&x_full[qs], qph, &abort_sh, p.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint64_t ad = sdesc_kmajor_sw128(smem_addr(a_ring + as * kABytes));
-                const uint64_t bd = sdesc_kmajor_sw128(smem_addr(x_ring + as * C::X_BYTES));
+                const uint64_t bd = sdesc_kmajor_sw128(smem_addr(q_ring + qs * C::QSLOT));
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)   // four K = 16 steps of 32 bytes
                     mma_issue<kKindF16>(tmem_base, ad + 2 * ks, bd + 2 * ks, idesc, (i | ks) != 0);
                 tc_commit(&a_empty[as]);
+                tc_commit(&q_empty[qs]);
                 if (++as == astages) {
                     as = 0;
                     aph ^= 1;
+                }
+                if (++qs == qstages) {
+                    qs = 0;
+                    qph ^= 1;
                 }
             }
             tc_commit(ok ? &tfull_bar : &drain_bar);
@@ -278,32 +327,23 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         const int ct = threadIdx.x - 64;           // weight row of the tile
         const uint32_t a_row = smem_addr(a_ring) + ct * 128;
         const int sw = ct & 7;
-        pdl_wait();                                // the activations come from the previous kernel
         int qs = 0, as = 0;
-        uint32_t qph = 0, aph = 0, x_issued = 0, x_par = 0;
+        uint32_t qph = 0, aph = 0;
         for (int i = 0; i < my_kb; ++i) {
-            const int kb = kb0 + i;
             if (!mbar_wait(&q_full[qs], qph, &abort_sh, p.status)) break;
-            if (!mbar_wait(&a_empty[as], aph ^ 1, &abort_sh, p.status)) break;
-            if (ct == 0) {
-                mbar_arrive_expect_tx(&a_full[as], C::X_BYTES);
-                tma_load_2d(x_ring + as * C::X_BYTES, &tmX, &a_full[as], kb * kBK, m0);
-                x_issued |= 1u << as;
-                x_par = (x_par & ~(1u << as)) | (aph << as);
-            }
-            const uint8_t* qsl = q_ring + qs * kQSlot;
+            const uint8_t* qsl = q_ring + qs * C::QSLOT + C::X_BYTES;
             const uint4 c0 = *reinterpret_cast<const uint4*>(qsl + ct * 32);
             const uint4 c1 = *reinterpret_cast<const uint4*>(qsl + ct * 32 + 16);
             const float* ssl = reinterpret_cast<const float*>(qsl + kQBytes);
-            const float s0 = ssl[ct];
-            const float s1 = gps == 2 ? ssl[kBM + ct] : s0;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&q_empty[qs]);
+            const uint32_t s0 = __float_as_uint(ssl[ct]);
+            const uint32_t s1 = gps == 2 ? __float_as_uint(ssl[kBM + ct]) : s0;
+            if (!mbar_wait(&a_empty[as], aph ^ 1, &abort_sh, p.status)) break;
             const uint32_t dst = a_row + as * kABytes;
             const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            const uint64_t s20 = pair(s0, s0), s21 = pair(s1, s1);
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-                const uint4 v = dequant8<BF16>(w[c], c < 4 ? s0 : s1);
+                const uint4 v = dequant8<BF16>(w[c], c < 4 ? s20 : s21);
                 st_shared_v4(dst + ((c ^ sw) << 4), v.x, v.y, v.z, v.w);
             }
             fence_async_smem();
@@ -318,9 +358,8 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
                 aph ^= 1;
             }
         }
-        if (abort_sh && ct == 0)   // let the activation loads already issued land
-            for (int s = 0; s < astages; ++s)
-                if (x_issued & (1u << s)) mbar_wait(&a_full[s], (x_par >> s) & 1, nullptr, nullptr);
+        // Y may still be in use by the previous kernel until it has finished.
+        pdl_wait();
 
         // ---------------- epilogue
         const int q = warp & 3;                    // TMEM lane quarter of this warp
@@ -461,22 +500,24 @@ q8_status run_w4(const W4Args& a, cudaStream_t s) {
     int astages, qstages;
     if constexpr (C::SPLIT) {
         // Split K over a cluster (at most 8, every split non-empty) so that the
-        // grid fills the SMs at two CTAs per SM.
-        int want = 2 * sm_count() / (tiles_n * tiles_m);
+        // grid fills the SMs in one wave: two CTAs per SM for token tiles of 16
+        // and 32, one for 64 (its staging and reduction buffers take more than
+        // half an SM's shared memory).
+        int want = (NT == 64 ? 1 : 2) * sm_count() / (tiles_n * tiles_m);
         if (want < 1) want = 1;
         if (want > 8) want = 8;
         if (want > num_kb) want = num_kb;
         per = (num_kb + want - 1) / want;
         splits = (num_kb + per - 1) / per;
-        astages = NT == 64 ? 4 : 3;
-        qstages = NT == 16 ? 8 : NT == 32 ? 6 : 8;
+        astages = NT == 64 ? 3 : 2;
+        qstages = NT == 32 ? 6 : 8;
     } else {
-        astages = NT == 128 ? 4 : 3;
-        qstages = 8;
+        astages = NT == 128 ? 3 : 2;
+        qstages = NT == 128 ? 6 : 4;
     }
     if (astages > per) astages = per;
     if (qstages > per) qstages = per;
-    const int smem = astages * (kABytes + C::X_BYTES) + qstages * kQSlot + C::RED_BYTES + 1024;
+    const int smem = astages * kABytes + qstages * C::QSLOT + C::RED_BYTES + 1024;
 
     auto kern = w4a16_kernel<NT, BF16>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
