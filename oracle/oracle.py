@@ -67,6 +67,7 @@ def lib():
             "or_quant_weight_fp8": [vp, i64, i64, vp, vp],
             "or_quant_weight_group": [vp, i64, i64, i32, i64, vp, vp],
             "or_dequant_group16": [vp, vp, i64, i64, i64, i32, vp],
+            "or_quant_weight_q4k": [vp, i64, i64, vp, vp, vp, vp, vp],
             "or_quant_act_int8": [vp, i64, i64, vp, vp, vp, vp],
             "or_quant_act_fp8": [vp, i64, i64, f, vp, vp],
             "or_quant_act_static": [vp, i64, i64, f, vp, vp, vp],
@@ -179,6 +180,23 @@ def quant_weight_group(w: np.ndarray, g: int, bits: int = 4):
     S = np.empty((n, k // g), np.float32)
     lib().or_quant_weight_group(_ptr(w), n, k, bits, g, _ptr(q), _ptr(S))
     return q, S
+
+
+def quant_weight_q4k(w: np.ndarray):
+    """Q4_K two-level scales over super blocks of 8 x 32 weights.
+
+    Returns a dict: q (int8 N x K), s_sub, q_sub, S_eff (N x K/32) and
+    s_super (N x K/256).  S_eff is the per-32 scale the weight is dequantized
+    with (dequant_group16 / linear_w4a16 with g = 32)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    n, k = w.shape
+    assert k % 256 == 0
+    out = {"q": np.empty((n, k), np.int8), "s_sub": np.empty((n, k // 32), np.float32),
+           "s_super": np.empty((n, k // 256), np.float32),
+           "q_sub": np.empty((n, k // 32), np.uint8), "S_eff": np.empty((n, k // 32), np.float32)}
+    lib().or_quant_weight_q4k(_ptr(w), n, k, _ptr(out["q"]), _ptr(out["s_sub"]),
+                              _ptr(out["s_super"]), _ptr(out["q_sub"]), _ptr(out["S_eff"]))
+    return out
 
 
 def dequant_group16(q: np.ndarray, S: np.ndarray, g: int, fmt: str) -> np.ndarray:

@@ -273,6 +273,41 @@ void or_quant_weight_group(const float *W, int64_t n, int64_t k, int bits, int64
 }
 
 /*
+ * GGUF Q4_K-style two-level scales ([Xilyfe] GGUF section, Q4_K simulation):
+ * a super block is 8 sub-blocks of 32 weights along a row.  Each sub-block is
+ * one symmetric 4-bit block (or_quant_weight_group with g = 32: s_sub =
+ * absmax / 7, codes from the unquantized s_sub, as the page's step 3 does);
+ * then the 8 sub-block scales are quantized like a second set of weights by
+ * absmax over 15 levels (they are never negative):
+ *   s_super = fl32(max_j s_sub[j] / 15),
+ *   q_sub[j] = clamp(rne(fl32(s_sub[j] / s_super)), 0, 15),
+ * and the scale a sub-block is dequantized with is
+ *   S_eff[j] = fl32(s_super * q_sub[j]).
+ * Layouts: q n x k; s_sub, q_sub, S_eff n x (k / 32); s_super n x (k / 256).
+ */
+void or_quant_weight_q4k(const float *W, int64_t n, int64_t k, int8_t *q, float *s_sub,
+                         float *s_super, uint8_t *q_sub, float *S_eff) {
+    const int64_t ns = k / 32, nb = k / 256;
+    or_quant_weight_group(W, n, k, 4, 32, q, s_sub);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n; ++r)
+        for (int64_t b = 0; b < nb; ++b) {
+            const float *ss = s_sub + r * ns + b * 8;
+            float mx = ss[0];
+            for (int j = 1; j < 8; ++j)
+                if (ss[j] > mx) mx = ss[j];
+            float sup = mx / 15.0f;
+            s_super[r * nb + b] = sup;
+            for (int j = 0; j < 8; ++j) {
+                float t = ss[j] / sup;
+                double c = clampd(rne((double)t), 0.0, 15.0);
+                q_sub[r * ns + b * 8 + j] = (uint8_t)c;
+                S_eff[r * ns + b * 8 + j] = sup * (float)c;
+            }
+        }
+}
+
+/*
  * The 16-bit weight a group-quantized layer multiplies when its activations
  * are 16-bit (W4A16: the weight is brought back to the activation's format,
  * r = S q, [Xilyfe] "量化是什么" with Z = 0):

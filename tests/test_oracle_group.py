@@ -152,3 +152,47 @@ def test_linear_w4a16_matches_fp64_matmul(fmt):
     # selecting rows and columns picks the same values
     ys, _ = O.linear_w4a16(x, q, S, g, fmt, bias=bias, rows=[6, 0], cols=[47, 3, 5])
     assert np.array_equal(ys, y[[6, 0]][:, [47, 3, 5]])
+
+
+# ------------------------------------------------------------------ Q4_K two-level scales
+
+def test_q4k_page_example_super_scale():
+    # The page's three sub-blocks (4 values each, padded with zeros to the
+    # 32-value sub-blocks of Q4_K; zeros leave each absmax unchanged) and five
+    # empty sub-blocks make one 256-value super block.
+    g = _golden("worked_examples_4bit.json")["q4k_sub_blocks"]
+    w = np.zeros((1, 256), np.float32)
+    for j, blk in enumerate(g["blocks"]):
+        w[0, 32 * j:32 * j + 4] = blk
+    r = O.quant_weight_q4k(w)
+    assert np.allclose(r["s_sub"][0, :3], g["scales_printed"], atol=0.0006)
+    assert abs(float(r["s_super"][0, 0]) - g["super_scale_printed"]) < 5e-5
+    assert r["q_sub"][0].tolist() == [5, 15, 1, 0, 0, 0, 0, 0]      # 0.457/0.0857, 15, 0.071/0.0857
+    for j, codes in enumerate(g["codes_by_rule"]):
+        assert r["q"][0, 32 * j:32 * j + 4].tolist() == codes
+
+
+def test_q4k_invariants_and_nearest_sub_codes():
+    rng = np.random.default_rng(11)
+    w = (rng.standard_normal((12, 512)) * 0.02).astype(np.float32)
+    w[:, 40:72] *= np.float32(8.0)                  # uneven sub-block ranges
+    r = O.quant_weight_q4k(w)
+    q32, S32 = O.quant_weight_group(w, 32)
+    assert np.array_equal(r["q"], q32) and np.array_equal(r["s_sub"], S32)
+    ss = r["s_sub"].reshape(12, 2, 8)
+    sup = r["s_super"]
+    assert np.array_equal(sup, (ss.max(axis=2) / np.float32(15)).astype(np.float32))
+    qs = r["q_sub"].reshape(12, 2, 8)
+    assert qs.max() <= 15
+    top = np.take_along_axis(qs, ss.argmax(axis=2)[..., None], 2)[..., 0]
+    assert np.all(top == 15)
+    for i in range(12):
+        for b in range(2):
+            s = Fraction(float(sup[i, b]))
+            for j in range(8):
+                t = Fraction(float(ss[i, b, j])) / s
+                best = min(range(16), key=lambda c: (abs(t - c), c % 2))
+                assert qs[i, b, j] == best
+    eff = r["S_eff"].reshape(12, 2, 8).astype(np.float64)
+    assert np.all(np.abs(eff - ss) <= sup[..., None] * (0.5 + 2.0 ** -20))
+    assert np.array_equal(eff, (sup[..., None] * qs.astype(np.float32)).astype(np.float64))
