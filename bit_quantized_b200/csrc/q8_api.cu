@@ -479,6 +479,38 @@ q8_status q8_quantize_weight_g4(const void* W, q8_dtype w_dtype, int64_t n, int6
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+q8_status q8_quantize_weight_q4k(const void* W, q8_dtype w_dtype, int64_t n, int64_t k,
+                                 int64_t ldw, void* codes, int64_t ldc, float* scale,
+                                 uint8_t* sub_codes, float* super_scale, q8_stream_t stream) {
+    if (w_dtype != Q8_F16 && w_dtype != Q8_BF16) return Q8_ERR_DTYPE;
+    if (n < 0 || k <= 0 || n > kMaxDim || k > kMaxDim || k % 256 != 0 || n % 16 != 0 || ldw < k ||
+        ldc < k / 2)
+        return Q8_ERR_SHAPE;
+    if (n == 0) return Q8_OK;
+    if (!W || !codes || !scale || !sub_codes || !super_scale) return Q8_ERR_NULL;
+    if (!aligned16(W) || !ld_ok(ldw, k, w_dtype) || !aligned16(codes) || ldc % 16 != 0 ||
+        !aligned16(scale) || !aligned16(sub_codes) || !aligned16(super_scale))
+        return Q8_ERR_ALIGN;
+    q8_status st = check_device();
+    if (st != Q8_OK) return st;
+    return launch_status(launch_q4k_quant(W, w_dtype, n, k, ldw, static_cast<uint8_t*>(codes), ldc,
+                                          scale, sub_codes, super_scale,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+q8_status q8_expand_q4k_scales(const uint8_t* sub_codes, const float* super_scale, int64_t n,
+                               int64_t k, float* scale, q8_stream_t stream) {
+    if (n < 0 || k <= 0 || n > kMaxDim || k > kMaxDim || k % 256 != 0 || n % 16 != 0)
+        return Q8_ERR_SHAPE;
+    if (n == 0) return Q8_OK;
+    if (!sub_codes || !super_scale || !scale) return Q8_ERR_NULL;
+    if (!aligned16(sub_codes) || !aligned16(super_scale) || !aligned16(scale)) return Q8_ERR_ALIGN;
+    q8_status st = check_device();
+    if (st != Q8_OK) return st;
+    return launch_status(launch_q4k_expand(sub_codes, super_scale, n, k, scale,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
 q8_status q8_linear_w4a16(const void* X, q8_dtype x_dtype, int64_t m, int64_t k, int64_t ldx,
                           const q8_weight_g4* w, const float* bias, void* Y, int64_t ldy,
                           q8_stream_t stream) {

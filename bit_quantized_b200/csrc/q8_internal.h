@@ -81,6 +81,12 @@ cudaError_t launch_group_quant(const void* W, q8_dtype dt, int64_t n, int64_t k,
                                int group, uint8_t* codes, int64_t ldc, float* scale,
                                cudaStream_t s);
 
+cudaError_t launch_q4k_quant(const void* W, q8_dtype dt, int64_t n, int64_t k, int64_t ldw,
+                             uint8_t* codes, int64_t ldc, float* scale, uint8_t* sub_codes,
+                             float* super_scale, cudaStream_t s);
+cudaError_t launch_q4k_expand(const uint8_t* sub_codes, const float* super_scale, int64_t n,
+                              int64_t k, float* scale, cudaStream_t s);
+
 struct W4Args {
     const void* x; bool x_bf16;            // m x k activations (bf16 or fp16), row stride ldx
     int64_t m, k, ldx;

@@ -9,6 +9,10 @@
 //   linear   w~ = round16(fl32(S q)) in the activation's 16-bit format,
 //            y = sum_k x w~ (fp32 in TMEM), y = fl32(y + bias[n]), Y = bf16(y)
 //
+// Q4_K ("大模型量化" (Xilyfe), GGUF section, Q4_K simulation): groups of 32
+// whose scales are quantized again per super block of 8, s_super = max / 15,
+// 4-bit sub-scale codes; the kernel multiplies with fl32(s_super * code).
+//
 // Storage: codes are n x k/2 bytes, element 2j in the low nibble of byte j and
 // element 2j+1 in the high nibble; scales are group-major, scale[j * n + r], so
 // the 128 rows of a tile read one contiguous 512-byte run per group.
@@ -92,6 +96,85 @@ group_quant_kernel(const T* __restrict__ W, int64_t n, int64_t k, int64_t ldw, i
         *reinterpret_cast<uint4*>(out + j / 2) = make_uint4(word[0], word[1], word[2], word[3]);
     }
     scale[grp * n + row] = S;
+}
+
+// ============================================================================
+// Q4_K two-level scales: one thread per super block of 8 x 32 weights
+// ============================================================================
+// Sub-blocks are quantized exactly as groups of 32 above (codes from the
+// unquantized sub-block scale); then s_super = fl32(max s_sub / 15) and the
+// sub-block scale codes are clamp(rne(fl32(s_sub / s_super)), 0, 15).  The
+// effective scale fl32(s_super * code) goes to the group-major scale array the
+// W4A16 kernel reads; the compact form (two sub-scale codes per byte, low
+// nibble = even sub-block, and the fp32 s_super) is written for storage.
+template <typename T>
+__global__ void __launch_bounds__(256)
+q4k_quant_kernel(const T* __restrict__ W, int64_t n, int64_t k, int64_t ldw,
+                 uint8_t* __restrict__ codes, int64_t ldc, float* __restrict__ scale,
+                 uint8_t* __restrict__ sub_codes, float* __restrict__ super_scale) {
+    const int64_t nb = k / 256;
+    const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (id >= n * nb) return;
+    const int64_t row = id / nb, blk = id % nb;
+    float ss[8];
+#pragma unroll 1
+    for (int j = 0; j < 8; ++j) {
+        const T* w = W + row * ldw + blk * 256 + j * 32;
+        float f[4][8];
+        float a = 0.f;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            widen8<T>(*reinterpret_cast<const uint4*>(w + 8 * v), f[v]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(f[v][i]));
+        }
+        float S = __fdiv_rn(a, 7.0f);
+        if (!(S >= kEps)) S = kEps;
+        uint32_t word[4];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            uint32_t packed = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                int q = __float2int_rn(__fdiv_rn(f[v][i], S));
+                q = q < -7 ? -7 : (q > 7 ? 7 : q);
+                packed |= static_cast<uint32_t>(q + 8) << (4 * i);
+            }
+            word[v] = packed;
+        }
+        *reinterpret_cast<uint4*>(codes + row * ldc + blk * 128 + j * 16) =
+            make_uint4(word[0], word[1], word[2], word[3]);
+        ss[j] = S;
+    }
+    float mx = ss[0];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) mx = ss[j] > mx ? ss[j] : mx;
+    const float sup = __fdiv_rn(mx, 15.0f);
+    super_scale[blk * n + row] = sup;
+    uint32_t pk = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        int c = __float2int_rn(__fdiv_rn(ss[j], sup));
+        c = c < 0 ? 0 : (c > 15 ? 15 : c);
+        scale[(blk * 8 + j) * n + row] = __fmul_rn(sup, static_cast<float>(c));
+        pk |= static_cast<uint32_t>(c) << (4 * j);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        sub_codes[(blk * 4 + j) * n + row] = static_cast<uint8_t>(pk >> (8 * j));
+}
+
+// scale[j * n + r] = fl32(s_super[(j / 8) * n + r] * code_j), code_j from the
+// compact sub-scale codes.
+__global__ void __launch_bounds__(256)
+q4k_expand_kernel(const uint8_t* __restrict__ sub_codes, const float* __restrict__ super_scale,
+                  int64_t n, int64_t k, float* __restrict__ scale) {
+    const int64_t total = n * (k / 32);
+    const int64_t id = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (id >= total) return;
+    const int64_t j = id / n, r = id % n;
+    const uint32_t c = (sub_codes[(j / 2) * n + r] >> (4 * (j & 1))) & 15u;
+    scale[id] = __fmul_rn(super_scale[(j / 8) * n + r], static_cast<float>(c));
 }
 
 // ============================================================================
@@ -583,6 +666,31 @@ cudaError_t launch_group_quant(const void* W, q8_dtype dt, int64_t n, int64_t k,
     else
         group_quant_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(W), n, k, ldw, group, codes, ldc, scale);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_q4k_quant(const void* W, q8_dtype dt, int64_t n, int64_t k, int64_t ldw,
+                             uint8_t* codes, int64_t ldc, float* scale, uint8_t* sub_codes,
+                             float* super_scale, cudaStream_t s) {
+    const int64_t blocks_total = n * (k / 256);
+    if (blocks_total == 0) return cudaSuccess;
+    const unsigned blocks = static_cast<unsigned>((blocks_total + 255) / 256);
+    if (dt == Q8_F16)
+        q4k_quant_kernel<__half><<<blocks, 256, 0, s>>>(static_cast<const __half*>(W), n, k, ldw,
+                                                       codes, ldc, scale, sub_codes, super_scale);
+    else
+        q4k_quant_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(W), n, k, ldw, codes, ldc, scale, sub_codes,
+            super_scale);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_q4k_expand(const uint8_t* sub_codes, const float* super_scale, int64_t n,
+                              int64_t k, float* scale, cudaStream_t s) {
+    const int64_t total = n * (k / 32);
+    if (total == 0) return cudaSuccess;
+    q4k_expand_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, s>>>(sub_codes, super_scale,
+                                                                                 n, k, scale);
     return cudaGetLastError();
 }
 

@@ -41,7 +41,7 @@ EXPORTED = [
     "q8_outlier_quantize_act",
     "q8_linear_w8a8", "q8_linear_w8a8_requant", "q8_linear_w8a8_dynamic", "q8_linear_int8_mixed",
     "q8_linear_int8_mixed_noalloc",
-    "q8_quantize_weight_g4", "q8_linear_w4a16",
+    "q8_quantize_weight_g4", "q8_quantize_weight_q4k", "q8_expand_q4k_scales", "q8_linear_w4a16",
     "q8_workspace_size", "q8_status_string",
     "q8_get_device_status", "q8_clear_device_status", "q8_device_check", "q8_version",
 ]
@@ -86,6 +86,8 @@ _SIG = {
                                       _f, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp], _int),
     "q8_quantize_weight_g4": ([_vp, _int, _i64, _i64, _i64, ctypes.c_int32, _vp, _i64, _vp, _vp],
                               _int),
+    "q8_quantize_weight_q4k": ([_vp, _int, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _vp], _int),
+    "q8_expand_q4k_scales": ([_vp, _vp, _i64, _i64, _vp, _vp], _int),
     "q8_linear_w4a16": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeightG4), _vp, _vp, _i64,
                          _vp], _int),
     "q8_workspace_size": ([_int, _i64, _i64, _i64], _sz),
@@ -409,6 +411,35 @@ def q8_quantize_weight_g4(W: torch.Tensor, group: int = 128, stream=None) -> QWe
                                       int(group), _ptr(codes), codes.stride(0), _ptr(scale),
                                       _stream(stream)), "q8_quantize_weight_g4")
     return QWeightG4(codes, scale, int(group))
+
+
+def q8_quantize_weight_q4k(W: torch.Tensor, stream=None):
+    """GGUF Q4_K-style weights (see q8_quantize_weight_q4k in q8.h).
+
+    Returns (QWeightG4 with group 32 and the effective scales, sub_codes
+    (k/64) x n uint8, super_scale (k/256) x n fp32)."""
+    _cuda(W, "W")
+    n, k = W.shape
+    dev = W.device
+    codes = torch.empty((n, k // 2), dtype=torch.uint8, device=dev)
+    scale = torch.empty((k // 32, n), dtype=torch.float32, device=dev)
+    sub = torch.empty((max(k // 64, 1), n), dtype=torch.uint8, device=dev)
+    sup = torch.empty((max(k // 256, 1), n), dtype=torch.float32, device=dev)
+    _check(_lib.q8_quantize_weight_q4k(_ptr(W), _FLOAT_DT.get(W.dtype, -1), n, k, W.stride(0),
+                                       _ptr(codes), codes.stride(0), _ptr(scale), _ptr(sub),
+                                       _ptr(sup), _stream(stream)), "q8_quantize_weight_q4k")
+    return QWeightG4(codes, scale, 32), sub, sup
+
+
+def q8_expand_q4k_scales(sub_codes: torch.Tensor, super_scale: torch.Tensor, k: int,
+                         out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The (k/32) x n effective scales of compact Q4_K scales."""
+    n = super_scale.shape[1]
+    if out is None:
+        out = torch.empty((k // 32, n), dtype=torch.float32, device=super_scale.device)
+    _check(_lib.q8_expand_q4k_scales(_ptr(sub_codes), _ptr(super_scale), n, k, _ptr(out),
+                                     _stream(stream)), "q8_expand_q4k_scales")
+    return out
 
 
 def q8_linear_w4a16(X: torch.Tensor, w: QWeightG4, bias: Optional[torch.Tensor] = None,

@@ -11,7 +11,8 @@
  *     activations (SmoothQuant-style per-column multipliers), and a W8A8 linear
  *     that re-quantizes its output to INT8 for the next layer;
  *   - group-wise 4-bit weights with one absmax scale per group of 32-128
- *     values along K, multiplied with 16-bit activations (W4A16).
+ *     values along K (optionally with GGUF Q4_K-style quantized group scales),
+ *     multiplied with 16-bit activations (W4A16).
  *
  * Notation follows the pages' linear map Q = round(R / S) + Z, R = S (Q - Z):
  * `scale` is S, the dequant multiplier, and `zero_point` is Z, an integer held
@@ -64,7 +65,7 @@
 extern "C" {
 #endif
 
-#define Q8_VERSION 4
+#define Q8_VERSION 5
 
 /* Same object as cudaStream_t. */
 typedef struct CUstream_st *q8_stream_t;
@@ -319,6 +320,40 @@ typedef struct {
 q8_status q8_quantize_weight_g4(const void *W, q8_dtype w_dtype, int64_t n, int64_t k,
                                 int64_t ldw, int32_t group, void *codes, int64_t ldc,
                                 float *scale, q8_stream_t stream);
+
+/*
+ * GGUF Q4_K-style weights ([Xilyfe] GGUF section, Q4_K simulation): groups of
+ * 32 along K (sub-blocks) quantized as q8_quantize_weight_g4 with group 32,
+ * whose scales are quantized again per super block of 8 sub-blocks (256
+ * values): s_super = fl32(max s_sub / 15), sub-scale codes
+ * c = clamp(rne(fl32(s_sub / s_super)), 0, 15).  The weight codes come from the
+ * unquantized sub-block scale (the page's order); a sub-block is dequantized
+ * with fl32(s_super * c).  Bit-exact with a scalar reference.
+ *
+ *   W            device, n x k, Q8_F16 or Q8_BF16, row stride ldw; k % 256 == 0,
+ *                n % 16 == 0 (Q8_ERR_SHAPE).
+ *   codes, ldc   device output, as q8_quantize_weight_g4.
+ *   scale        device output, (k / 32) x n fp32, group-major: the effective
+ *                scales fl32(s_super * c), so {codes, scale, group = 32} is a
+ *                q8_weight_g4 for q8_linear_w4a16.
+ *   sub_codes    device output, (k / 64) x n bytes: byte [j][r] holds the codes
+ *                of sub-blocks 2j (low nibble) and 2j+1 (high nibble) of row r.
+ *   super_scale  device output, (k / 256) x n fp32.
+ * sub_codes and super_scale are the compact stored form (0.53 bytes per 32
+ * weights instead of 4); q8_expand_q4k_scales rebuilds `scale` from them.
+ */
+q8_status q8_quantize_weight_q4k(const void *W, q8_dtype w_dtype, int64_t n, int64_t k,
+                                 int64_t ldw, void *codes, int64_t ldc, float *scale,
+                                 uint8_t *sub_codes, float *super_scale, q8_stream_t stream);
+
+/*
+ * scale[j * n + r] = fl32(super_scale[(j / 8) * n + r] * c_j) for the compact
+ * Q4_K scales written by q8_quantize_weight_q4k (layouts as there); the result
+ * is bit-identical to the `scale` output of that call.  k % 256 == 0,
+ * n % 16 == 0.  One launch.
+ */
+q8_status q8_expand_q4k_scales(const uint8_t *sub_codes, const float *super_scale, int64_t n,
+                               int64_t k, float *scale, q8_stream_t stream);
 
 /*
  * W4A16 linear: Y = X W~^T (+ bias), W~ the group-wise 4-bit weight brought

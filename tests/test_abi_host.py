@@ -289,3 +289,31 @@ def test_linear_w4a16_validation():
     assert lw4(m=0, X=None, Y=None) == q8.Q8_OK                  # empty call
     if NO_GPU:
         assert lw4() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def q4k(W=FAKE, dt=q8.Q8_BF16, n=256, k=512, ldw=512, codes=FAKE, ldc=256, sc=FAKE, sub=FAKE, sup=FAKE):
+    return L.q8_quantize_weight_q4k(W, dt, n, k, ldw, codes, ldc, sc, sub, sup, _ns)
+
+
+def test_quantize_weight_q4k_validation():
+    assert q4k(sub=None) == q8.Q8_ERR_NULL
+    assert q4k(sup=None) == q8.Q8_ERR_NULL
+    assert q4k(dt=q8.Q8_F32) == q8.Q8_ERR_DTYPE
+    assert q4k(k=384, ldw=384, ldc=192) == q8.Q8_ERR_SHAPE      # k % 256
+    assert q4k(n=40) == q8.Q8_ERR_SHAPE
+    assert q4k(ldc=128) == q8.Q8_ERR_SHAPE
+    assert q4k(sub=MIS) == q8.Q8_ERR_ALIGN
+    assert q4k(ldc=264) == q8.Q8_ERR_ALIGN
+    assert q4k(n=0, W=None) == q8.Q8_OK
+    if NO_GPU:
+        assert q4k() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def test_expand_q4k_scales_validation():
+    f = L.q8_expand_q4k_scales
+    assert f(None, FAKE, 256, 512, FAKE, _ns) == q8.Q8_ERR_NULL
+    assert f(FAKE, FAKE, 256, 320, FAKE, _ns) == q8.Q8_ERR_SHAPE
+    assert f(FAKE, MIS, 256, 512, FAKE, _ns) == q8.Q8_ERR_ALIGN
+    assert f(None, None, 0, 512, None, _ns) == q8.Q8_OK
+    if NO_GPU:
+        assert f(FAKE, FAKE, 256, 512, FAKE, _ns) in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)

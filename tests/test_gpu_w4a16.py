@@ -7,7 +7,9 @@ dequantized weight within the fp32-accumulation bound of tests/parity.py:
 Shapes cover every token tile (16, 32, 64, 128, 256), K split across a
 cluster and not, a half-filled last K slice (K = 96 with groups of 32),
 ragged token and channel tails, both 16-bit activation formats, and the
-q_proj-sized decode case in full.
+q_proj-sized decode case in full.  Q4_K two-level scales (codes, sub-scale
+codes, super scales, effective scales, and their expansion from the compact
+form) are bit-exact too.
 """
 import numpy as np
 import pytest
@@ -118,3 +120,47 @@ def test_linear_w4a16_after_producer_kernel():
     torch.cuda.synchronize()
     assert torch.equal(Y.view(torch.int16), Y_sep.view(torch.int16))
     assert q8.q8_get_device_status() == 0
+
+
+# ------------------------------------------------------------------ Q4_K two-level scales
+
+def _unpack_sub(sub: torch.Tensor) -> np.ndarray:
+    b = sub.cpu().numpy()
+    out = np.empty((2 * b.shape[0], b.shape[1]), np.uint8)
+    out[0::2] = b & 15
+    out[1::2] = b >> 4
+    return out.T                                   # n x k/32
+
+
+@pytest.mark.parametrize("n,k,dt", [(256, 512, torch.bfloat16), (48, 1024, torch.float16),
+                                    (4096, 4096, torch.bfloat16)])
+def test_q4k_quant_bit_exact(n, k, dt):
+    W = workloads.random_matrix(n, k, dt, seed=n + 3 * k, std=0.02)
+    W[:, 40:72] *= 8.0                             # uneven sub-block ranges
+    w32 = P.host_f32(W)
+    qw, sub, sup = q8.q8_quantize_weight_q4k(W.to(DEV))
+    torch.cuda.synchronize()
+    r = O.quant_weight_q4k(w32)
+    P.assert_equal(_unpack(qw.codes), r["q"], "q4k codes")
+    P.assert_equal(_unpack_sub(sub), r["q_sub"], "q4k sub-scale codes")
+    P.assert_equal(sup.cpu().numpy().T, r["s_super"], "q4k super scales")
+    P.assert_equal(qw.scale.cpu().numpy().T, r["S_eff"], "q4k effective scales")
+    again = q8.q8_expand_q4k_scales(sub, sup, k)
+    torch.cuda.synchronize()
+    P.assert_equal(again.cpu().numpy(), qw.scale.cpu().numpy(), "expanded scales")
+
+
+def test_q4k_linear():
+    m, n, k = 16, 512, 1024
+    X = workloads.random_matrix(m, k, torch.bfloat16, 21)
+    W = workloads.random_matrix(n, k, torch.bfloat16, 22, std=0.02)
+    W[:, 64:96] *= 20.0                            # one loud sub-block per row
+    qw, sub, sup = q8.q8_quantize_weight_q4k(W.to(DEV))
+    Y = q8.q8_linear_w4a16(X.to(DEV), qw)
+    torch.cuda.synchronize()
+    r = O.quant_weight_q4k(P.host_f32(W))
+    x32 = P.host_f32(X)
+    y_ref, _ = O.linear_w4a16(x32, r["q"], r["S_eff"], 32, "bf16")
+    wd = O.widen16(O.dequant_group16(r["q"], r["S_eff"], 32, "bf16"), "bf16").astype(np.float64)
+    extra = k * 2.0 ** -22 * (np.abs(x32.astype(np.float64)) @ np.abs(wd).T)
+    P.assert_bf16_within(P.bf16_bits(Y), y_ref, extra, "q4k linear")
