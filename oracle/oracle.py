@@ -365,6 +365,30 @@ def linear_w8a8_fp8(xq, Sx, wq, Sw, bias=None, rows=None, cols=None):
     return acc, y, round16(y, "bf16")
 
 
+def linear_moe_fp8(xq, Sx, wq, Sw, offsets, n: int, bias=None, rows=None):
+    """Grouped FP8 rowwise linear of a mixture-of-experts layer.
+
+    [FBGEMM] 5.4 (Llama4 experts): the experts' weights sit in one tensor, one
+    FP8 block with per-row scales per expert, and each expert's tokens are
+    quantized and multiplied with f8f8bf16_rowwise on their own.  Tokens are
+    sorted by expert: rows offsets[e] .. offsets[e+1]-1 of xq use expert e,
+    whose weight is rows e*n .. e*n+n-1 of the stacked wq (scales Sw, bias
+    stacked the same way).  Each block is linear_w8a8_fp8.  Returns
+    (y fp32 len(rows) x n, Y bf16 bits)."""
+    off = [int(v) for v in offsets]
+    m = np.asarray(xq).shape[0]
+    r_all = _index(rows, m)
+    y = np.zeros((r_all.size, n), np.float32)
+    for e in range(len(off) - 1):
+        sel = np.nonzero((r_all >= off[e]) & (r_all < off[e + 1]))[0]
+        if sel.size == 0:
+            continue
+        _, ye, _ = linear_w8a8_fp8(xq, Sx, wq, Sw, bias, rows=r_all[sel],
+                                   cols=np.arange(e * n, (e + 1) * n))
+        y[sel] = ye
+    return y, round16(y, "bf16")
+
+
 def dequant_weight_f16(wq, Sw, Zw, colidx, rows=None) -> np.ndarray:
     """fp16 bits of S (q - Z) for the given weight columns (nr x ncols)."""
     wq = np.ascontiguousarray(wq)
