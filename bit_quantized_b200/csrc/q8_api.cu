@@ -542,6 +542,36 @@ q8_status q8_linear_w4a16(const void* X, q8_dtype x_dtype, int64_t m, int64_t k,
     return launch_w4a16(a, reinterpret_cast<cudaStream_t>(stream));
 }
 
+q8_status q8_linear_fp8_grouped(const q8_act* x, const q8_weight* w, int64_t num_experts,
+                                const int32_t* offsets, const float* bias, void* Y, int64_t ldy,
+                                q8_stream_t stream) {
+    if (!x || !w) return Q8_ERR_NULL;
+    q8_status st = check_weight(w);
+    if (st != Q8_OK) return st;
+    if (x->code_dtype != Q8_E4M3 || w->code_dtype != Q8_E4M3) return Q8_ERR_DTYPE;
+    if (num_experts < 1 || num_experts > 4096 || w->n % num_experts != 0) return Q8_ERR_SHAPE;
+    const int64_t n = w->n / num_experts;
+    if (n % 16 != 0 || x->m < 0 || x->m > kMaxDim || x->k != w->k || x->ld < x->k || ldy < n ||
+        (x->m + 127) / 128 + num_experts > 65535)
+        return Q8_ERR_SHAPE;
+    if (x->m == 0 || n == 0) return Q8_OK;   // empty call
+    if (!x->codes || !x->scale || !offsets || !Y) return Q8_ERR_NULL;
+    if (!aligned16(x->codes) || x->ld % 16 != 0 || !aligned16(x->scale) || !aligned16(Y) ||
+        ldy % 8 != 0 || (bias && !aligned16(bias)) || (reinterpret_cast<uintptr_t>(offsets) & 3u))
+        return Q8_ERR_ALIGN;
+    st = check_device();
+    if (st != Q8_OK) return st;
+    MoeArgs a = {};
+    a.m = x->m; a.k = x->k;
+    a.x_codes = x->codes; a.ldx = x->ld; a.sx = x->scale;
+    a.experts = num_experts; a.n = n;
+    a.w_codes = w->codes; a.ldw = w->ld; a.sw = w->scale;
+    a.offsets = offsets;
+    a.bias = bias;
+    a.y = static_cast<__nv_bfloat16*>(Y); a.ldy = ldy;
+    return launch_moe_fp8(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
 q8_status q8_get_device_status(int32_t* out, q8_stream_t stream) {
     if (!out) return Q8_ERR_NULL;
     q8_status st = check_device();

@@ -100,5 +100,20 @@ struct W4Args {
 
 q8_status launch_w4a16(const W4Args& a, cudaStream_t s);
 
+// ---- grouped FP8 GEMM for mixture-of-experts layers (q8_moe.cu)
+struct MoeArgs {
+    int64_t m, k;                          // tokens sorted by expert, reduction depth
+    const void* x_codes; int64_t ldx;      // m x k e4m3, row stride ldx bytes
+    const float* sx;                       // [m]
+    int64_t experts, n;                    // experts, output channels per expert
+    const void* w_codes; int64_t ldw;      // experts*n x k e4m3, row stride ldw bytes
+    const float* sw;                       // [experts * n]
+    const int32_t* offsets;                // device [experts + 1]
+    const float* bias;                     // [experts * n] or null
+    __nv_bfloat16* y; int64_t ldy;
+};
+
+q8_status launch_moe_fp8(const MoeArgs& a, cudaStream_t s);
+
 
 }  // namespace q8

@@ -42,6 +42,7 @@ EXPORTED = [
     "q8_linear_w8a8", "q8_linear_w8a8_requant", "q8_linear_w8a8_dynamic", "q8_linear_int8_mixed",
     "q8_linear_int8_mixed_noalloc",
     "q8_quantize_weight_g4", "q8_quantize_weight_q4k", "q8_expand_q4k_scales", "q8_linear_w4a16",
+    "q8_linear_fp8_grouped",
     "q8_workspace_size", "q8_status_string",
     "q8_get_device_status", "q8_clear_device_status", "q8_device_check", "q8_version",
 ]
@@ -88,6 +89,8 @@ _SIG = {
                               _int),
     "q8_quantize_weight_q4k": ([_vp, _int, _i64, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _vp], _int),
     "q8_expand_q4k_scales": ([_vp, _vp, _i64, _i64, _vp, _vp], _int),
+    "q8_linear_fp8_grouped": ([ctypes.POINTER(CAct), ctypes.POINTER(CWeight), _i64, _vp, _vp, _vp,
+                               _i64, _vp], _int),
     "q8_linear_w4a16": ([_vp, _int, _i64, _i64, _i64, ctypes.POINTER(CWeightG4), _vp, _vp, _i64,
                          _vp], _int),
     "q8_workspace_size": ([_int, _i64, _i64, _i64], _sz),
@@ -453,6 +456,24 @@ def q8_linear_w4a16(X: torch.Tensor, w: QWeightG4, bias: Optional[torch.Tensor] 
     _check(_lib.q8_linear_w4a16(_ptr(X), _FLOAT_DT.get(X.dtype, -1), m, k, X.stride(0),
                                 ctypes.byref(cw), _ptr(bias), _ptr(out), out.stride(0),
                                 _stream(stream)), "q8_linear_w4a16")
+    return out
+
+
+def q8_linear_fp8_grouped(x: QAct, w: QWeight, num_experts: int, offsets: torch.Tensor,
+                          bias: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """Grouped FP8 rowwise linear (mixture of experts): tokens sorted by expert,
+    offsets a CUDA int32 tensor of num_experts + 1 entries; returns bf16 M x n."""
+    if not offsets.is_cuda or offsets.dtype != torch.int32 or offsets.numel() != num_experts + 1:
+        raise ValueError("offsets must be a CUDA int32 tensor of num_experts + 1 entries")
+    m = x.codes.shape[0]
+    n = w.codes.shape[0] // num_experts
+    if out is None:
+        out = torch.empty((m, n), dtype=torch.bfloat16, device=x.codes.device)
+    cx, cw = x.c(), w.c()
+    _check(_lib.q8_linear_fp8_grouped(ctypes.byref(cx), ctypes.byref(cw), int(num_experts),
+                                      _ptr(offsets.contiguous()), _ptr(bias), _ptr(out),
+                                      out.stride(0), _stream(stream)), "q8_linear_fp8_grouped")
     return out
 
 

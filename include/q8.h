@@ -12,7 +12,8 @@
  *     that re-quantizes its output to INT8 for the next layer;
  *   - group-wise 4-bit weights with one absmax scale per group of 32-128
  *     values along K (optionally with GGUF Q4_K-style quantized group scales),
- *     multiplied with 16-bit activations (W4A16).
+ *     multiplied with 16-bit activations (W4A16);
+ *   - the grouped FP8 rowwise linear of mixture-of-experts layers.
  *
  * Notation follows the pages' linear map Q = round(R / S) + Z, R = S (Q - Z):
  * `scale` is S, the dequant multiplier, and `zero_point` is Z, an integer held
@@ -65,7 +66,7 @@
 extern "C" {
 #endif
 
-#define Q8_VERSION 5
+#define Q8_VERSION 6
 
 /* Same object as cudaStream_t. */
 typedef struct CUstream_st *q8_stream_t;
@@ -375,6 +376,38 @@ q8_status q8_expand_q4k_scales(const uint8_t *sub_codes, const float *super_scal
 q8_status q8_linear_w4a16(const void *X, q8_dtype x_dtype, int64_t m, int64_t k, int64_t ldx,
                           const q8_weight_g4 *w, const float *bias, void *Y, int64_t ldy,
                           q8_stream_t stream);
+
+/*
+ * Grouped FP8 rowwise linear of a mixture-of-experts layer ([FBGEMM] 5.4,
+ * Llama4 experts: the experts' FP8 weights are stored together with per-row
+ * scales, and each expert's tokens are quantized and multiplied with
+ * f8f8bf16_rowwise on their own).  Tokens are sorted by expert: rows
+ * offsets[e] .. offsets[e+1]-1 of x use expert e, whose weight is rows
+ * e*n .. e*n+n-1 of w (n = w->n / num_experts), with the same scales and bias
+ * rows.  Per token and channel: acc = sum_k e4m3 x e4m3 (fp32),
+ * y = fl32(fl32(acc * Sx[m]) * Sw[e*n + j]) (+ bias[e*n + j]), Y = bf16(y).
+ * Quantize the sorted activations with q8_quantize_act(Q8_FP8_E4M3): its
+ * per-token scales are the same whether taken per expert or over all tokens.
+ *
+ *   x            E4M3 activation codes, x->m tokens sorted by expert.
+ *   w            E4M3 weights of all experts stacked, w->n = num_experts * n,
+ *                per-row scales; n % 16 == 0.
+ *   num_experts  1 .. 4096; ceil(x->m / 128) + num_experts <= 65535.
+ *   offsets      device int32 [num_experts + 1], non-decreasing, offsets[0] = 0,
+ *                offsets[num_experts] = x->m (typically the previous kernel's
+ *                routing result).  Out-of-range values are clamped to
+ *                [0, x->m], so no call writes outside Y; rows no expert
+ *                covers are left unwritten.
+ *   bias         device fp32 [w->n] (per expert, stacked), or NULL.
+ *   Y            device, x->m x n bf16 (sorted token order), row stride ldy
+ *                (ldy % 8 == 0).
+ * One launch; the fp32 accumulation order is not specified (the FP8 bound of
+ * q8_linear_w8a8 applies).  It may start before the previous kernel on
+ * `stream` has ended and waits for it before reading anything.
+ */
+q8_status q8_linear_fp8_grouped(const q8_act *x, const q8_weight *w, int64_t num_experts,
+                                const int32_t *offsets, const float *bias, void *Y, int64_t ldy,
+                                q8_stream_t stream);
 
 /*
  * Dynamic per-token activation quantization and the W8A8 linear in one call:

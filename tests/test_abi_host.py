@@ -317,3 +317,27 @@ def test_expand_q4k_scales_validation():
     assert f(None, None, 0, 512, None, _ns) == q8.Q8_OK
     if NO_GPU:
         assert f(FAKE, FAKE, 256, 512, FAKE, _ns) in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def lmoe(x=None, w=None, E=4, offsets=FAKE, bias=None, Y=FAKE, ldy=64):
+    x = x or _act(code_dtype=q8.Q8_E4M3, rowsum=None)
+    w = w or _weight(code_dtype=q8.Q8_E4M3, zp=None, n=256)
+    return L.q8_linear_fp8_grouped(ctypes.byref(x), ctypes.byref(w), E, offsets, bias, Y, ldy, _ns)
+
+
+def test_linear_fp8_grouped_validation():
+    assert L.q8_linear_fp8_grouped(None, None, 4, FAKE, None, FAKE, 64, _ns) == q8.Q8_ERR_NULL
+    assert lmoe(offsets=None) == q8.Q8_ERR_NULL
+    assert lmoe(Y=None) == q8.Q8_ERR_NULL
+    assert lmoe(x=_act()) == q8.Q8_ERR_DTYPE                     # INT8 activations
+    assert lmoe(w=_weight(zp=None, n=256)) == q8.Q8_ERR_DTYPE    # INT8 weights
+    assert lmoe(E=0) == q8.Q8_ERR_SHAPE
+    assert lmoe(E=3) == q8.Q8_ERR_SHAPE                          # n not divisible by experts
+    assert lmoe(E=32) == q8.Q8_ERR_SHAPE                         # 8 channels per expert
+    assert lmoe(ldy=16) == q8.Q8_ERR_SHAPE                       # ldy < n
+    assert lmoe(ldy=68) == q8.Q8_ERR_ALIGN
+    assert lmoe(offsets=FAKE + 2) == q8.Q8_ERR_ALIGN
+    assert lmoe(bias=MIS) == q8.Q8_ERR_ALIGN
+    assert lmoe(x=_act(code_dtype=q8.Q8_E4M3, rowsum=None, m=0), Y=None) == q8.Q8_OK
+    if NO_GPU:
+        assert lmoe() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
