@@ -569,8 +569,36 @@ def extras(q8, dev, pk):
                                                   / pk["bf16_tflops"], 4)
         out[name] = r
         del Xd, Wd
+    out["moe_fp8_grouped"] = moe_extra(q8, dev, pk, flush)
     torch.cuda.synchronize()
     return out
+
+
+def moe_extra(q8, dev, pk, flush):
+    """Grouped FP8 rowwise linear of a mixture-of-experts layer: 16 experts of
+    2048 x 4096 (e4m3 weights, 134 MB, beyond L2) and 4096 tokens, each routed
+    to a seeded uniformly drawn expert."""
+    E, n, k, m = 16, 2048, 4096, 4096
+    g = torch.Generator().manual_seed(5)
+    pick = torch.randint(0, E, (m,), generator=g)
+    counts = torch.bincount(pick, minlength=E)
+    off = torch.zeros(E + 1, dtype=torch.int32)
+    off[1:] = torch.cumsum(counts, 0).to(torch.int32)
+    X = workloads.random_matrix(m, k, torch.bfloat16, 6).to(dev)
+    W = workloads.random_matrix(E * n, k, torch.bfloat16, 7, 0.02).to(dev)
+    qa = q8.q8_quantize_act(X, "fp8", clip_ub=1200.0)
+    qw = q8.q8_quantize_weight(W, "fp8", "e4m3")
+    del W
+    offd = off.to(dev)
+    Y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    t = _time_kernel(lambda: q8.q8_linear_fp8_grouped(qa, qw, E, offd, out=Y), flush)
+    tops = 2.0 * m * n * k / (t * 1e-3) / 1e12
+    int8_peak = pk["bf16_tflops"] * NOMINAL_INT8_OVER_BF16
+    return {"shape": f"{E} experts x {n} x {k}, {m} tokens (max {int(counts.max())}, "
+                     f"min {int(counts.min())} per expert)",
+            "grouped_us": round(t * 1e3, 2), "grouped_tops": round(tops, 1),
+            "grouped_frac_fp8_peak": round(tops / int8_peak, 4),
+            "grouped_gbs": round((m * k + E * n * k + 2 * m * n) / (t * 1e-3) / 1e9, 1)}
 
 
 # ---------------------------------------------------------------- CPU oracle
