@@ -648,10 +648,25 @@ def cpu_baseline(name: str, seconds: float = 10.0):
             break
     dt = time.perf_counter() - t0
     what = "full steps" if rows_n == w.m else f"steps on {rows_n} of {w.m} token rows"
-    return {"value": round(done * ops / dt / 1e12, 6), "unit": UNIT, "cores": O.threads(),
+    cores = O.threads()
+    # The same step on one host thread, for a quarter of the time.
+    O.set_threads(1)
+    try:
+        done1, t1 = 0, time.perf_counter()
+        while True:
+            oracle_step(O, w, x32, q, rows, cols)
+            done1 += 1
+            if time.perf_counter() - t1 >= seconds / 4:
+                break
+        dt1 = time.perf_counter() - t1
+    finally:
+        O.set_threads(cores)
+    return {"value": round(done * ops / dt / 1e12, 6), "unit": UNIT, "cores": cores,
             "kind": "oracle",
             "sample": f"{done} {what} of {name} ({w.m}x{w.n}x{w.k}: activation quantization + "
-                      f"GEMM + epilogue) in {dt:.1f} s; weight quantization excluded as on the GPU"}
+                      f"GEMM + epilogue) in {dt:.1f} s; weight quantization excluded as on the GPU",
+            "one_thread": {"value": round(done1 * ops / dt1 / 1e12, 6), "unit": UNIT,
+                           "sample": f"{done1} {what} in {dt1:.1f} s on 1 thread"}}
 
 
 def run_reference(args, world, rank):
