@@ -43,7 +43,12 @@ bool ld_ok(int64_t ld, int64_t cols, q8_dtype d) {
 constexpr int64_t kMaxDim = (int64_t(1) << 31) - 1;
 constexpr int64_t kMaxKInt8 = 32768;
 
-q8_status check_device() {
+// Armed failure (q8_inject_failure): after `g_inject_skip` more validated
+// calls, the next one returns `g_inject_code` before anything is enqueued.
+int g_inject_code = 0;
+int g_inject_skip = 0;
+
+q8_status device_ready() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         cudaGetLastError();
@@ -60,6 +65,24 @@ q8_status check_device() {
         g_arch_ok[dev] = (major == 10 && minor == 0) ? 1 : 2;
     }
     return g_arch_ok[dev] == 1 ? Q8_OK : Q8_ERR_UNSUPPORTED_ARCH;
+}
+
+// The last step of every launching entry point's checks: an armed injected
+// failure, then the device.
+q8_status check_device() {
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_inject_code != 0) {
+            if (g_inject_skip > 0) {
+                --g_inject_skip;
+            } else {
+                const q8_status code = static_cast<q8_status>(g_inject_code);
+                g_inject_code = 0;
+                return code;
+            }
+        }
+    }
+    return device_ready();
 }
 
 q8_status launch_status(cudaError_t e) {
@@ -125,7 +148,16 @@ const char* q8_status_string(q8_status s) {
     return "unknown status";
 }
 
-q8_status q8_device_check(void) { return check_device(); }
+q8_status q8_device_check(void) { return device_ready(); }
+
+q8_status q8_inject_failure(q8_status code, int32_t skip) {
+    if (code < Q8_OK || code > Q8_ERR_CUDA) return Q8_ERR_SCHEME;
+    if (skip < 0) return Q8_ERR_SHAPE;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_inject_code = code;
+    g_inject_skip = code == Q8_OK ? 0 : skip;
+    return Q8_OK;
+}
 
 size_t q8_workspace_size(int op, int64_t m, int64_t n, int64_t k) {
     if (op != Q8_OP_LINEAR_INT8_MIXED || m < 0 || n < 0 || k < 0) return 0;
@@ -574,7 +606,7 @@ q8_status q8_linear_fp8_grouped(const q8_act* x, const q8_weight* w, int64_t num
 
 q8_status q8_get_device_status(int32_t* out, q8_stream_t stream) {
     if (!out) return Q8_ERR_NULL;
-    q8_status st = check_device();
+    q8_status st = device_ready();
     if (st != Q8_OK) return st;
     int* p = device_status_ptr();
     if (!p) return Q8_ERR_CUDA;
@@ -590,7 +622,7 @@ q8_status q8_get_device_status(int32_t* out, q8_stream_t stream) {
 }
 
 q8_status q8_clear_device_status(q8_stream_t stream) {
-    q8_status st = check_device();
+    q8_status st = device_ready();
     if (st != Q8_OK) return st;
     int* p = device_status_ptr();
     if (!p) return Q8_ERR_CUDA;

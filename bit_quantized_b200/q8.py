@@ -45,6 +45,7 @@ EXPORTED = [
     "q8_linear_fp8_grouped",
     "q8_workspace_size", "q8_status_string",
     "q8_get_device_status", "q8_clear_device_status", "q8_device_check", "q8_version",
+    "q8_inject_failure",
 ]
 
 
@@ -98,6 +99,7 @@ _SIG = {
     "q8_get_device_status": ([_vp, _vp], _int),
     "q8_clear_device_status": ([_vp], _int),
     "q8_device_check": ([], _int),
+    "q8_inject_failure": ([_int, ctypes.c_int32], _int),
     "q8_version": ([], _int),
 }
 for _name, (_args, _res) in _SIG.items():
@@ -132,6 +134,12 @@ def q8_version() -> int:
 
 def q8_device_check() -> int:
     return int(_lib.q8_device_check())
+
+
+def q8_inject_failure(code: int, skip: int = 0) -> None:
+    """Arm a one-shot host-side failure: after `skip` more validated calls, the
+    next one returns `code` (raised as Q8Error by this binding); Q8_OK disarms."""
+    _check(_lib.q8_inject_failure(int(code), int(skip)), "q8_inject_failure")
 
 
 def q8_workspace_size(op: int, m: int, n: int, k: int) -> int:

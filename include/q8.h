@@ -66,7 +66,7 @@
 extern "C" {
 #endif
 
-#define Q8_VERSION 6
+#define Q8_VERSION 7
 
 /* Same object as cudaStream_t. */
 typedef struct CUstream_st *q8_stream_t;
@@ -517,6 +517,18 @@ q8_status q8_clear_device_status(q8_stream_t stream);
 /* Q8_OK when the current device can run this library, else
  * Q8_ERR_UNSUPPORTED_ARCH or Q8_ERR_CUDA (host). */
 q8_status q8_device_check(void);
+
+/*
+ * Host-side fault injection, for testing a caller's error handling (host).
+ * Arms a one-shot failure: after `skip` more calls that pass their argument
+ * validation, the next such call returns `code` without enqueuing anything;
+ * then the hook is disarmed.  Calls that fail validation do not count.
+ * Applies to every entry point that launches work (not to q8_device_check,
+ * q8_get_device_status or q8_clear_device_status).  code = Q8_OK disarms.
+ * Returns Q8_ERR_SCHEME for a code that is not a q8_status, Q8_ERR_SHAPE for
+ * skip < 0.  Process-wide; safe to call from any thread.
+ */
+q8_status q8_inject_failure(q8_status code, int32_t skip);
 
 /* Q8_VERSION of the built library (host). */
 int q8_version(void);

@@ -341,3 +341,29 @@ def test_linear_fp8_grouped_validation():
     assert lmoe(x=_act(code_dtype=q8.Q8_E4M3, rowsum=None, m=0), Y=None) == q8.Q8_OK
     if NO_GPU:
         assert lmoe() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
+def test_injected_failure_propagates_and_disarms():
+    inj = L.q8_inject_failure
+    try:
+        assert inj(99, 0) == q8.Q8_ERR_SCHEME
+        assert inj(q8.Q8_ERR_LAUNCH, -1) == q8.Q8_ERR_SHAPE
+        assert inj(q8.Q8_ERR_LAUNCH, 0) == q8.Q8_OK
+        assert qs(X=None) == q8.Q8_ERR_NULL            # failed validation: not counted
+        assert q8.q8_device_check() != q8.Q8_ERR_LAUNCH # status calls are not affected
+        assert qs() == q8.Q8_ERR_LAUNCH                # the next validated call fails ...
+        if NO_GPU:                                      # ... once
+            assert qs() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+            assert inj(q8.Q8_ERR_WORKSPACE, 1) == q8.Q8_OK
+            assert lw4() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)   # skipped
+            assert lmoe() == q8.Q8_ERR_WORKSPACE
+        assert inj(q8.Q8_ERR_DEVICE_TIMEOUT, 0) == q8.Q8_OK
+        with pytest.raises(q8.Q8Error) as e:           # the binding raises the injected status
+            q8._check(lw4(), "q8_linear_w4a16")
+        assert e.value.status == q8.Q8_ERR_DEVICE_TIMEOUT
+        q8.q8_inject_failure(q8.Q8_ERR_LAUNCH, 3)
+        q8.q8_inject_failure(q8.Q8_OK)                 # disarm
+        if NO_GPU:
+            assert qs() in (q8.Q8_ERR_CUDA, q8.Q8_ERR_UNSUPPORTED_ARCH)
+    finally:
+        inj(q8.Q8_OK, 0)
