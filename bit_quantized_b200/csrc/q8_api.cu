@@ -3,6 +3,7 @@
 // memory or synchronizes, except q8_get_device_status.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cfloat>
 #include <cstdint>
 #include <cstring>
@@ -45,7 +46,7 @@ constexpr int64_t kMaxKInt8 = 32768;
 
 // Armed failure (q8_inject_failure): after `g_inject_skip` more validated
 // calls, the next one returns `g_inject_code` before anything is enqueued.
-int g_inject_code = 0;
+std::atomic<int> g_inject_code{0};   // written under g_mu; read without it when unarmed
 int g_inject_skip = 0;
 
 q8_status device_ready() {
@@ -70,15 +71,15 @@ q8_status device_ready() {
 // The last step of every launching entry point's checks: an armed injected
 // failure, then the device.
 q8_status check_device() {
-    {
+    if (g_inject_code.load(std::memory_order_acquire) != 0) {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (g_inject_code != 0) {
+        const int code = g_inject_code.load(std::memory_order_relaxed);
+        if (code != 0) {
             if (g_inject_skip > 0) {
                 --g_inject_skip;
             } else {
-                const q8_status code = static_cast<q8_status>(g_inject_code);
-                g_inject_code = 0;
-                return code;
+                g_inject_code.store(0, std::memory_order_release);
+                return static_cast<q8_status>(code);
             }
         }
     }
@@ -154,8 +155,8 @@ q8_status q8_inject_failure(q8_status code, int32_t skip) {
     if (code < Q8_OK || code > Q8_ERR_CUDA) return Q8_ERR_SCHEME;
     if (skip < 0) return Q8_ERR_SHAPE;
     std::lock_guard<std::mutex> lk(g_mu);
-    g_inject_code = code;
     g_inject_skip = code == Q8_OK ? 0 : skip;
+    g_inject_code.store(code, std::memory_order_release);
     return Q8_OK;
 }
 
