@@ -82,3 +82,19 @@ def test_grouped_fp8_llama4_like_sampled():
 def test_grouped_fp8_offsets_leave_rows_uncovered():
     # offsets cover rows 0..99 only: rows 100..149 are never written
     _moe_case((40, 60, 50), 128, 256, seed=9, offsets=[0, 40, 100, 100], what="moe uncovered")
+
+
+def test_grouped_fp8_strided_output_leaves_guard_bands():
+    counts, n, k = (70, 0, 140), 144, 256
+    E, m = len(counts), sum(counts)
+    X = workloads.random_matrix(m, k, torch.bfloat16, 51)
+    W = workloads.random_matrix(E * n, k, torch.bfloat16, 52, std=0.02)
+    off = torch.tensor(np.concatenate([[0], np.cumsum(counts)]), dtype=torch.int32, device=DEV)
+    qa = q8.q8_quantize_act(X.to(DEV), "fp8", clip_ub=1200.0)
+    qw = q8.q8_quantize_weight(W.to(DEV), "fp8", "e4m3")
+    big = torch.full((m + 3, n + 24), -5.0, dtype=torch.bfloat16, device=DEV)
+    q8.q8_linear_fp8_grouped(qa, qw, E, off, out=big[:m, :n])
+    ref = q8.q8_linear_fp8_grouped(qa, qw, E, off)
+    torch.cuda.synchronize()
+    assert torch.equal(big[:m, :n].view(torch.int16), ref.view(torch.int16))
+    assert (big[:m, n:] == -5.0).all() and (big[m:] == -5.0).all()

@@ -164,3 +164,19 @@ def test_q4k_linear():
     wd = O.widen16(O.dequant_group16(r["q"], r["S_eff"], 32, "bf16"), "bf16").astype(np.float64)
     extra = k * 2.0 ** -22 * (np.abs(x32.astype(np.float64)) @ np.abs(wd).T)
     P.assert_bf16_within(P.bf16_bits(Y), y_ref, extra, "q4k linear")
+
+
+def test_w4a16_strided_output_leaves_guard_bands():
+    # Y is a view into a larger buffer (row stride n + 40, two extra rows):
+    # the padding, filled with a sentinel, must stay untouched.
+    m, n, k, g = 37, 272, 512, 64
+    X = workloads.random_matrix(m, k, torch.bfloat16, 31)
+    W = workloads.random_matrix(n, k, torch.bfloat16, 32, std=0.02)
+    qw = q8.q8_quantize_weight_g4(W.to(DEV), g)
+    big = torch.full((m + 2, n + 40), -3.0, dtype=torch.bfloat16, device=DEV)
+    Y = q8.q8_linear_w4a16(X.to(DEV), qw, out=big[:m, :n])
+    ref = q8.q8_linear_w4a16(X.to(DEV), qw)
+    torch.cuda.synchronize()
+    assert Y.stride(0) == n + 40
+    assert torch.equal(big[:m, :n].view(torch.int16), ref.view(torch.int16))
+    assert (big[:m, n:] == -3.0).all() and (big[m:] == -3.0).all()
