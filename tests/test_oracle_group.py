@@ -196,3 +196,18 @@ def test_q4k_invariants_and_nearest_sub_codes():
     eff = r["S_eff"].reshape(12, 2, 8).astype(np.float64)
     assert np.all(np.abs(eff - ss) <= sup[..., None] * (0.5 + 2.0 ** -20))
     assert np.array_equal(eff, (sup[..., None] * qs.astype(np.float32)).astype(np.float64))
+
+
+def test_q4k_all_zero_super_block():
+    # Every sub-block at the eps floor: s_super = 1e-8 / 15, every sub-scale
+    # code 15, so the effective scale is the floor again; codes are 0.
+    w = np.zeros((2, 512), np.float32)
+    w[1, 300] = 0.5                               # second super block of row 1 is not empty
+    r = O.quant_weight_q4k(w)
+    assert np.all(r["q"][0] == 0)
+    assert np.all(r["s_super"][0] == np.float32(np.float32(1e-8) / np.float32(15)))
+    assert np.all(r["q_sub"][0] == 15)
+    assert np.all(np.abs(r["S_eff"][0] - np.float32(1e-8)) <= np.float32(1e-8) * 2.0 ** -22)
+    # row 1: block 0 empty as above; block 1 holds 0.5 in sub-block 1 (values 288..319)
+    assert r["q"][1, 300] == 7 and r["q_sub"][1, 9] == 15
+    assert np.all(r["q_sub"][1, 8:16][[0, 2, 3, 4, 5, 6, 7]] == 0)
