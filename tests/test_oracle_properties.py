@@ -1,0 +1,105 @@
+"""Property-based pins of the oracle's quantizers (hypothesis).
+
+Random rows of finite fp32 values are checked against what absmax / min-max
+quantization guarantees by construction ("大模型量化" (Xilyfe), symmetric and
+asymmetric sections; "大模型量化技术" overview 2.3): code ranges, the end
+points of a row landing on the end codes, half-step error bounds, odd
+symmetry, row sums, and the e4m3 rounding's monotonicity and saturation
+(OCP FP8 E4M3 definition).  Exact rational arithmetic decides the codes
+away from ties.
+"""
+from fractions import Fraction
+
+import numpy as np
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+from hypothesis.extra.numpy import arrays
+
+from oracle import oracle as O
+
+SETTINGS = settings(max_examples=60, deadline=None, derandomize=True,
+                    suppress_health_check=[HealthCheck.too_slow])
+
+finite = st.floats(min_value=-3.0e4, max_value=3.0e4, allow_nan=False, allow_infinity=False,
+                   width=32)
+rows = st.integers(1, 4).flatmap(
+    lambda r: st.integers(1, 8).flatmap(
+        lambda c: arrays(np.float32, (r, 32 * c), elements=finite)))
+
+
+def _near_tie(t: Fraction) -> bool:
+    f = t - (t.numerator // t.denominator)
+    return abs(f - Fraction(1, 2)) < Fraction(1, 2 ** 18)
+
+
+@SETTINGS
+@given(rows)
+def test_symmetric_int8_properties(x):
+    q, S, rs = O.quant_act_int8(x)
+    assert np.abs(q.astype(np.int32)).max() <= 127
+    assert np.array_equal(rs, q.astype(np.int32).sum(axis=1))
+    for r in range(x.shape[0]):
+        a = float(np.abs(x[r]).max())
+        s = float(S[r])
+        if a == 0.0:
+            assert s == np.float32(1e-8) and not q[r].any()
+            continue
+        raw = np.float32(np.float32(a) / np.float32(127))
+        assert s == float(max(raw, np.float32(1e-8)))               # eps floor
+        if raw >= np.float32(1e-8):
+            j = int(np.abs(x[r]).argmax())
+            assert abs(int(q[r, j])) == 127
+        for jj in range(0, x.shape[1], 7):
+            t = Fraction(float(x[r, jj])) / Fraction(s)
+            if not _near_tie(t):
+                want = min(range(-127, 128), key=lambda c: abs(t - c))
+                assert q[r, jj] == want
+    qn, Sn, _ = O.quant_act_int8(-x)
+    assert np.array_equal(Sn, S) and np.array_equal(qn, -q)
+
+
+@SETTINGS
+@given(rows)
+def test_asymmetric_int8_properties(w):
+    q, S, Z = O.quant_weight(w, "asym")
+    assert q.min() >= -128 and q.max() <= 127
+    for r in range(w.shape[0]):
+        lo, hi = float(w[r].min()), float(w[r].max())
+        s = float(S[r])
+        if hi == lo:
+            continue
+        jlo = int(w[r].argmin())
+        if lo <= 0.0 <= hi:
+            assert q[r, jlo] == -128
+            # dequantized values sit within half a step (plus rounding slop of S)
+            deq = s * (q[r].astype(np.float64) - float(Z[r]))
+            assert np.all(np.abs(deq - w[r].astype(np.float64)) <= s * (0.5 + 2.0 ** -18) + 1e-30)
+
+
+@SETTINGS
+@given(rows)
+def test_group_quant_is_blockwise_symmetric(w):
+    g = 32
+    q, S = O.quant_weight_group(w, g)
+    n, k = w.shape
+    qb, Sb, _ = O.quant_weight(w.reshape(n * (k // g), g), "sym", bits=4)
+    assert np.array_equal(q.reshape(n * (k // g), g), qb)
+    assert np.array_equal(S.reshape(-1), Sb)
+
+
+@SETTINGS
+@given(arrays(np.float32, (64,), elements=st.floats(min_value=-2000.0, max_value=2000.0,
+                                                    allow_nan=False, width=32)))
+def test_e4m3_rounding_properties(v):
+    codes = O.round_e4m3(v)
+    back = O.widen_e4m3(codes).astype(np.float64)
+    x = v.astype(np.float64)
+    order = np.argsort(x, kind="stable")
+    assert np.all(np.diff(back[order]) >= 0)                      # monotone
+    assert np.all(np.abs(back) <= 448.0)                          # saturates
+    assert np.array_equal(O.round_e4m3(back.astype(np.float32)), codes)   # idempotent
+    inside = np.abs(x) <= 448.0
+    # nearest: no finite e4m3 value is strictly closer (spacing 2^(e-3), subnormals 2^-9)
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -6)))
+    half = np.exp2(e - 3) / 2
+    assert np.all(np.abs(back - x)[inside] <= half[inside] + 1e-12)
