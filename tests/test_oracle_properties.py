@@ -4,7 +4,8 @@ Random rows of finite fp32 values are checked against what absmax / min-max
 quantization guarantees by construction ("大模型量化" (Xilyfe), symmetric and
 asymmetric sections; "大模型量化技术" overview 2.3): code ranges, the end
 points of a row landing on the end codes, half-step error bounds, odd
-symmetry, row sums, and the e4m3 rounding's monotonicity and saturation
+symmetry, row sums, the e4m3 rounding's monotonicity and saturation, the
+LLM.int8 outlier rule by brute force, the FP8 clip and static scales
 (OCP FP8 E4M3 definition).  Exact rational arithmetic decides the codes
 away from ties.
 """
@@ -103,3 +104,50 @@ def test_e4m3_rounding_properties(v):
     e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -6)))
     half = np.exp2(e - 3) / 2
     assert np.all(np.abs(back - x)[inside] <= half[inside] + 1e-12)
+
+
+@SETTINGS
+@given(rows, st.floats(min_value=0.5, max_value=40.0, width=32))
+def test_outlier_columns_brute_force(x, T):
+    mask, idx, count = O.outlier_columns(x, T)
+    want = (np.abs(x.astype(np.float64)) > T).any(axis=0)
+    assert np.array_equal(mask.astype(bool), want)
+    assert idx.tolist() == np.nonzero(want)[0].tolist() and count == int(want.sum())
+    # the regular stream's per-token scale ignores those columns; their codes are 0
+    q, S, _ = O.quant_act_int8(x, skip=mask)
+    assert not q[:, want].any()
+    rest = np.where(want[None, :], 0.0, np.abs(x))
+    expect = np.maximum((rest.max(axis=1).astype(np.float32) / np.float32(127)).astype(np.float32),
+                        np.float32(1e-8))
+    assert np.array_equal(S, expect)
+
+
+@SETTINGS
+@given(rows, st.sampled_from([0.0, 1200.0, 50.0]))
+def test_fp8_activation_clip(x, ub):
+    q, S = O.quant_act_fp8(x, ub)
+    a = np.abs(x).max(axis=1)
+    if ub > 0:
+        a = np.minimum(a, np.float32(ub))
+    expect = np.maximum((a.astype(np.float32) / np.float32(448)).astype(np.float32), np.float32(1e-8))
+    assert np.array_equal(S, expect)
+    back = np.abs(O.widen_e4m3(q))
+    assert back.max() <= 448.0
+    over = np.abs(x) > (a[:, None] if ub > 0 else np.inf)
+    assert np.all(back[over] == 448.0)                 # values past the clip saturate
+
+
+@SETTINGS
+@given(rows, st.floats(min_value=0.0009765625, max_value=50.0, width=32))
+def test_static_scale_and_requant(x, S):
+    q, Sr, rs = O.quant_act_static(x, S)
+    assert np.all(Sr == np.float32(S)) and np.array_equal(rs, q.astype(np.int32).sum(axis=1))
+    assert np.abs(q.astype(np.int32)).max() <= 127
+    assert np.array_equal(O.requant(x, S), q)          # the same rule on a layer output
+    s = Fraction(float(np.float32(S)))
+    flat = x.reshape(-1)
+    for j in range(0, flat.size, 5):
+        t = Fraction(float(flat[j])) / s
+        if not _near_tie(t):
+            want = max(-127, min(127, min(range(-128, 129), key=lambda c: abs(t - c))))
+            assert q.reshape(-1)[j] == want
