@@ -4,10 +4,10 @@ Random rows of finite fp32 values are checked against what absmax / min-max
 quantization guarantees by construction ("大模型量化" (Xilyfe), symmetric and
 asymmetric sections; "大模型量化技术" overview 2.3): code ranges, the end
 points of a row landing on the end codes, half-step error bounds, odd
-symmetry, row sums, the e4m3 rounding's monotonicity and saturation, the
-LLM.int8 outlier rule by brute force, the FP8 clip and static scales
-(OCP FP8 E4M3 definition).  Exact rational arithmetic decides the codes
-away from ties.
+symmetry, row sums, the e4m3 rounding's monotonicity and saturation (OCP
+FP8 E4M3 definition), the LLM.int8 outlier rule by brute force, the FP8
+clip and static scales.  Exact rational arithmetic decides the codes away
+from ties.
 """
 from fractions import Fraction
 
