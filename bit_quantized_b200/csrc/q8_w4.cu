@@ -21,14 +21,17 @@
 // lane each) and NT tokens (the MMA's N side).  For small token counts the K
 // range is split across the CTAs of a cluster and the fp32 partials are summed
 // through distributed shared memory in rank order, as in the int8 decode GEMM.
-//   warp 0     one lane streams the packed codes and the scales of each
-//              64-deep K slice into a ring of staging slots (TMA, no swizzle);
-//   warp 1     TMEM allocation; one lane issues tcgen05.mma kind::f16;
+//   warp 0     one lane streams, per 64-deep K slice, the packed codes and
+//              scales (no swizzle) and the activation tile (128-byte swizzle)
+//              into one slot of a staging ring by TMA; the first ring of codes
+//              and scales goes out before the programmatic-launch wait;
+//   warp 1     TMEM allocation; one lane issues tcgen05.mma kind::f16 with the
+//              dequantized weight slice as A and the staged activation tile
+//              as B, then frees both rings' slots;
 //   warps 2-5  dequantize: thread r expands row r's 64 codes of a slice into
 //              16-bit values written directly in the 128-byte-swizzled K-major
-//              layout the MMA reads (thread 0 also starts the activation
-//              tile's TMA into the same stage); then the same warps run the
-//              epilogue.
+//              layout the MMA reads (a separate, shorter ring); then the same
+//              warps run the epilogue.
 // No TMA multicast is used.
 #include <cuda.h>
 #include <cuda_bf16.h>
