@@ -88,6 +88,7 @@ def _linear_case(m, n, k, g, dt, seed, bias=False, what=""):
     (40, 272, 512, 64, torch.float16),       # token tile 64, ragged channels
     (100, 256, 512, 32, torch.bfloat16),     # token tile 128, no split
     (300, 384, 256, 128, torch.float16),     # two token tiles of 256, ragged
+    (260, 256, 2048, 32, torch.bfloat16),    # tile 256 with 32 K slices: staging rings wrap
 ])
 def test_linear_w4a16_shapes(m, n, k, g, dt):
     _linear_case(m, n, k, g, dt, seed=m * 7 + n, bias=(m % 2 == 0), what=f"{m}x{n}x{k} g{g}")
