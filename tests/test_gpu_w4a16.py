@@ -89,6 +89,7 @@ def _linear_case(m, n, k, g, dt, seed, bias=False, what=""):
     (100, 256, 512, 32, torch.bfloat16),     # token tile 128, no split
     (300, 384, 256, 128, torch.float16),     # two token tiles of 256, ragged
     (260, 256, 2048, 32, torch.bfloat16),    # tile 256 with 32 K slices: staging rings wrap
+    (16, 128, 8192, 128, torch.bfloat16),    # K split over 8 CTAs of 16 slices each: rings wrap
 ])
 def test_linear_w4a16_shapes(m, n, k, g, dt):
     _linear_case(m, n, k, g, dt, seed=m * 7 + n, bias=(m % 2 == 0), what=f"{m}x{n}x{k} g{g}")
