@@ -340,8 +340,8 @@ q8_status q8_quantize_weight_g4(const void *W, q8_dtype w_dtype, int64_t n, int6
  *   sub_codes    device output, (k / 64) x n bytes: byte [j][r] holds the codes
  *                of sub-blocks 2j (low nibble) and 2j+1 (high nibble) of row r.
  *   super_scale  device output, (k / 256) x n fp32.
- * sub_codes and super_scale are the compact stored form (0.53 bytes per 32
- * weights instead of 4); q8_expand_q4k_scales rebuilds `scale` from them.
+ * sub_codes and super_scale are the compact stored form (1 byte of scale per
+ * 32 weights instead of 4); q8_expand_q4k_scales rebuilds `scale` from them.
  */
 q8_status q8_quantize_weight_q4k(const void *W, q8_dtype w_dtype, int64_t n, int64_t k,
                                  int64_t ldw, void *codes, int64_t ldc, float *scale,
