@@ -12,6 +12,9 @@ and chains the steps in the order the pages give them:
   int8 linear        : int64 dot products -> zero-point correction -> S_x -> S_w
   fp8 linear         : double dot products -> fp32 -> S_x -> S_w
   LLM.int8 merge     : fp32(y_int8 + y16), y16 from the fp16 outlier columns
+  group-wise 4-bit   : per-group absmax / 7 codes; Q4_K second-level scales
+  W4A16 linear       : 16-bit dequantized weight, double dot products -> fp32
+  grouped FP8 (MoE)  : the FP8 linear over each expert's token rows and weight block
   output             : bf16 round-to-nearest-even of the fp32 result
 
 All inputs are numpy arrays on the host.  16-bit float tensors are passed as
