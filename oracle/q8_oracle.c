@@ -11,7 +11,8 @@
  *   [CSDN]     "大模型量化技术" overview (devpress.csdn.net), sections 2.1-2.3
  *   [FBGEMM]   "Transformers FP8 (W8A8) 量化实战：基于 FBGEMM", sections 5.1-5.3, 6
  *   [LLM.int8] "Transformers 单 GPU 高效推理：bitsandbytes LLM.int8 8-bit 混合精度量化"
- *   [Xilyfe]   "大模型量化" blog (xilyfe.github.io), symmetric / asymmetric / INT32 sections
+ *   [Xilyfe]   "大模型量化" blog (xilyfe.github.io), symmetric / asymmetric / INT32 /
+ *              GGUF (block and Q4_K) sections
  *
  * Arithmetic rules (no fused multiply-add, no fast-math; build flags
  * -O2 -ffp-contract=off):
