@@ -151,3 +151,39 @@ def test_static_scale_and_requant(x, S):
         if not _near_tie(t):
             want = max(-127, min(127, min(range(-128, 129), key=lambda c: abs(t - c))))
             assert q.reshape(-1)[j] == want
+
+
+blocks256 = st.integers(1, 3).flatmap(
+    lambda r: st.integers(1, 2).flatmap(
+        lambda c: arrays(np.float32, (r, 256 * c),
+                         elements=st.floats(min_value=-100.0, max_value=100.0, width=32))))
+
+
+@SETTINGS
+@given(blocks256)
+def test_q4k_scale_properties(w):
+    r = O.quant_weight_q4k(w)
+    n, k = w.shape
+    ss = r["s_sub"].reshape(n, k // 256, 8)
+    qs = r["q_sub"].reshape(n, k // 256, 8)
+    sup = r["s_super"]
+    assert qs.max() <= 15
+    assert np.array_equal(sup, (ss.max(axis=2) / np.float32(15)).astype(np.float32))
+    top = np.take_along_axis(qs, ss.argmax(axis=2)[..., None], 2)[..., 0]
+    assert np.all(top == 15)
+    eff = r["S_eff"].reshape(n, k // 256, 8).astype(np.float64)
+    assert np.all(np.abs(eff - ss) <= sup[..., None].astype(np.float64) * (0.5 + 2.0 ** -18))
+
+
+@SETTINGS
+@given(st.integers(1, 5), st.integers(1, 3), st.sampled_from([32, 64]), st.integers(0, 2 ** 31 - 1))
+def test_w4a16_product_matches_fp64(m, nk, g, seed):
+    rng = np.random.default_rng(seed)
+    n, k = 16, 64 * nk
+    x = O.widen16(O.round16(rng.standard_normal((m, k)).astype(np.float32), "bf16"), "bf16")
+    w = (rng.standard_normal((n, k)) * 0.05).astype(np.float32)
+    q, S = O.quant_weight_group(w, g)
+    y, _ = O.linear_w4a16(x, q, S, g, "bf16")
+    wd = O.widen16(O.dequant_group16(q, S, g, "bf16"), "bf16").astype(np.float64)
+    ref = x.astype(np.float64) @ wd.T
+    assert np.all(np.abs(y.astype(np.float64) - ref) <= np.spacing(np.abs(ref.astype(np.float32))))
