@@ -7,10 +7,18 @@
 A step is one forward of the quantized linear layer on one batch of synthetic
 input: dynamic per-token activation quantization followed by the W8A8 GEMM
 with its dequant epilogue (weights are quantized once, offline, before the
-timed region, as the pages do on load).  The default workload is the
-q_proj-shaped decode layer: 16 tokens x 4096 -> 4096, bf16 in, asymmetric
-uint8 weights, INT32 accumulation, bf16 out; --workload picks another of the
-seeded workloads in workloads.py (prefill FFN-up INT8, FP8 rowwise, LLM.int8).
+timed region, as the pages do on load).  The default workload is the largest
+one, the FBGEMM-style FP8 rowwise linear: 4096 tokens x 8192 -> 8192, bf16 in,
+per-token e4m3 activations with the 1200 upper bound, per-channel e4m3
+weights, fp32 accumulation, bf16 out; --workload picks another of the seeded
+workloads in workloads.py (decode and prefill INT8, LLM.int8), and the
+per_config extras time every workload's kernels one launch at a time.
+
+The roofline entry divides by the dense tensor peak for the GEMM's own dtype:
+the measured bf16 peak (MEASURED_PEAKS.json) times the nominal INT8/FP8 : bf16
+ratio of 2, burst or sustained according to the length of the timed region,
+and also by the INT8 and FP8 throughput of the library GEMMs
+(torch._int_mm, torch._scaled_mm) measured at 8192^3 in the same run.
 
 Timing: W warm-up steps, then exactly K steps replayed from CUDA graphs,
 bracketed by a barrier and a device synchronize, timed with CUDA events on the
@@ -231,7 +239,12 @@ def step_functions(q8, w):
     return step, gemm, 2
 
 
-def dominant_kernel(w, gemm_ms: float, pk: dict):
+# A timed region shorter than this runs at the burst clocks of a GPU that has
+# not yet settled under its power cap; longer ones at the sustained clocks.
+SUSTAINED_REGION_MS = 1000.0
+
+
+def dominant_kernel(w, gemm_ms: float, region_ms: float, pk: dict, lib_peaks: dict):
     """Roofline entry of the step's dominant kernel (the GEMM)."""
     ops = 2.0 * w.m * w.n * w.k
     t = gemm_ms * 1e-3
@@ -242,13 +255,96 @@ def dominant_kernel(w, gemm_ms: float, pk: dict):
                 "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4), "algorithmic_bytes": algo_bytes,
                 "peak_source": pk["source"] + " hbm_gbs (MEASURED_PEAKS.json, copy)"}
-    peak = pk["bf16_tflops_sustained"] * NOMINAL_INT8_OVER_BF16
+    sustained = region_ms >= SUSTAINED_REGION_MS
+    bf16 = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
+    peak = bf16 * NOMINAL_INT8_OVER_BF16
     achieved = ops / t / 1e12
-    return {"bound": "tensor", "kernel": "gemm_tile_kernel" + (" (LLM.int8)" if w.kind == "int8_mixed" else ""),
-            "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4), "algorithmic_ops": ops,
-            "peak_source": f"{pk['source']} bf16 sustained {pk['bf16_tflops_sustained']} x 2 "
-                           "(nominal dense INT8/FP8 : bf16 = 4.5 : 2.25); kernel timed in a long loop"}
+    out = {"bound": "tensor",
+           "kernel": "gemm_tile_kernel" + (" (LLM.int8)" if w.kind == "int8_mixed" else ""),
+           "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
+           "frac": round(achieved / peak, 4), "algorithmic_ops": ops,
+           "peak_source": (f"{pk['source']} bf16 {'sustained' if sustained else 'burst'} {bf16} x 2 "
+                           "(nominal dense INT8/FP8 : bf16 = 4.5 : 2.25); the kernel's timed region "
+                           f"lasted {region_ms:.1f} ms ({'>=' if sustained else '<'} "
+                           f"{SUSTAINED_REGION_MS:.0f} ms)")}
+    lib_key = "fp8_tops" if w.kind == "w8a8_fp8" else "int8_tops"
+    lp = lib_peaks.get(lib_key)
+    if lp:
+        out["peak_library"] = lp
+        out["frac_of_library"] = round(achieved / lp, 4)
+        out["library_source"] = lib_peaks.get(lib_key.replace("_tops", "_how"))
+    return out
+
+
+def library_peaks(dev) -> dict:
+    """Dense INT8 and FP8 GEMM throughput of the library kernels at 8192^3 on
+    this GPU: torch._int_mm (int8 x int8 -> int32) and torch._scaled_mm (e4m3 x
+    e4m3 -> bf16, rowwise fp32 scales where supported, else per-tensor).  Best
+    of 10 launches after 3 warm-ups, CUDA events.  Reported next to the
+    derived peak; a call the installed torch does not support is left out."""
+    n = 8192
+    out = {"shape": f"{n}^3", "how": "best of 10 launches, CUDA events"}
+    g = torch.Generator(device=dev).manual_seed(0)
+
+    def best(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(10):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return 2.0 * n ** 3 / (min(ts) * 1e-3) / 1e12
+
+    try:
+        A = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+        B = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+        out["int8_tops"] = round(best(lambda: torch._int_mm(A, B.t())), 1)
+        out["int8_how"] = "torch._int_mm int8 8192^3 (B column-major)"
+        del A, B
+    except Exception as e:  # noqa: BLE001 - report, do not fail the bench
+        out["int8_error"] = f"{type(e).__name__}: {str(e)[:120]}"
+    try:
+        A = (torch.randn(n, n, device=dev, generator=g) * 4).to(torch.float8_e4m3fn)
+        B = (torch.randn(n, n, device=dev, generator=g) * 4).to(torch.float8_e4m3fn)
+        sa = torch.ones((n, 1), dtype=torch.float32, device=dev)
+        sb = torch.ones((1, n), dtype=torch.float32, device=dev)
+        try:
+            fn = lambda: torch._scaled_mm(A, B.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
+            fn()
+            out["fp8_how"] = "torch._scaled_mm e4m3 8192^3, rowwise scales, bf16 out"
+        except Exception:  # noqa: BLE001 - rowwise scaling unsupported: per-tensor
+            one = torch.ones((), dtype=torch.float32, device=dev)
+            fn = lambda: torch._scaled_mm(A, B.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            out["fp8_how"] = "torch._scaled_mm e4m3 8192^3, per-tensor scales, bf16 out"
+        out["fp8_tops"] = round(best(fn), 1)
+        del A, B
+    except Exception as e:  # noqa: BLE001
+        out["fp8_error"] = f"{type(e).__name__}: {str(e)[:120]}"
+    torch.cuda.synchronize()
+    return out
+
+
+def launch_spread(fn, layers, R, n: int) -> dict:
+    """Median, p10 and p90 of n single launches of fn (CUDA events around each,
+    layers rotated as in the timed region)."""
+    for i in range(3):
+        fn(layers[i % R])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    for i in range(n):
+        ev[i][0].record()
+        fn(layers[i % R])
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ts = np.array([a.elapsed_time(b) * 1e3 for a, b in ev])
+    return {"median_us": round(float(np.median(ts)), 3), "p10_us": round(float(np.percentile(ts, 10)), 3),
+            "p90_us": round(float(np.percentile(ts, 90)), 3), "launches": n,
+            "how": "one launch between CUDA events, eager, layers rotated"}
 
 
 def describe(w):
@@ -334,8 +430,11 @@ def run_q8(args, world, rank, local):
     kernel_avg_ms = kernel_ms / args.steps
     del kernel_graphs
 
+    spread = launch_spread(kernel_fn, layers, R, n=min(max(args.steps, 20), 200))
     e2e = run_e2e(q8, layers, R, step_fn, args, world, ops_per_step, wl)
-    roof = dominant_kernel(wl, kernel_avg_ms, pk)
+    lib_peaks = library_peaks(dev) if (world == 1 and not args.no_library_peaks) else {}
+    roof = dominant_kernel(wl, kernel_avg_ms, kernel_ms, pk, lib_peaks)
+    roof["launch_spread"] = spread
     roof["traffic"] = load_profile_traffic(args.workload)
     roof["avg_launch_us"] = round(kernel_avg_ms * 1e3, 3)
     roof["duration_from"] = ("K launches of the kernel replayed alone right after the timed steps"
@@ -351,12 +450,13 @@ def run_q8(args, world, rank, local):
                    **describe(wl), "parallelism": f"dp{world} (independent batches per GPU)",
                    "l2": (f"steps rotate over {R} layers ({ws_bytes / 1e6:.0f} MB > 126 MB L2)"
                           if ws_bytes > L2_BYTES else
-                          f"{R} layers ({ws_bytes / 1e6:.1f} MB) stay L2-resident"),
-                   "timing": f"CUDA graphs of {R} steps, CUDA events, max over ranks"},
+                          f"{R} layers ({ws_bytes / 1e6:.1f} MB) stay L2-resident")},
+        "timing": f"CUDA graphs of {R} steps, CUDA events, max over ranks",
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": launches * args.steps,
         "clocks": clocks,
+        "library_peaks": lib_peaks,
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, seconds=args.cpu_seconds)
@@ -490,6 +590,41 @@ def _time_kernel(fn, flush, reps=20):
     return statistics.median(ts[3:])
 
 
+def _time_graph(fn, count: int, reps: int = 5) -> float:
+    """Average time (ms) of one fn(i) call, i = 0..count-1 captured back to
+    back in a CUDA graph and replayed `reps` times (no host launch overhead
+    between the calls; the rotated inputs keep them reading from HBM)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(count):
+            fn(i)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(count):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (reps * count)
+    del g
+    return ms
+
+
+def _rotated_copies(X, min_bytes: int):
+    """Independent copies of X whose total exceeds min_bytes (at least 2)."""
+    per = X.numel() * X.element_size()
+    n = int(max(2, min(16, -(-min_bytes // per))))
+    return [X.clone() for _ in range(n)]
+
+
 def extras(q8, dev, pk):
     """Kernel-level numbers for every workload (single GPU, L2 flushed per launch)."""
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
@@ -522,6 +657,16 @@ def extras(q8, dev, pk):
             r["act_quant_us"] = round(t_act * 1e3, 2)
             r["act_quant_gbs"] = round(act_bytes / (t_act * 1e-3) / 1e9, 1)
             r["act_quant_frac_hbm"] = round(act_bytes / (t_act * 1e-3) / 1e9 / pk["hbm_gbs"], 3)
+            # The same quantizer back to back over rotated inputs (> 2 x L2) in a
+            # CUDA graph: the kernel's own bandwidth, without launch overhead.
+            xs = _rotated_copies(Xd, 2 * L2_BYTES)
+            qas = [q8.q8_quantize_act(x, scheme, clip_ub=w.clip_ub) for x in xs]
+            t_g = _time_graph(lambda i: q8.q8_quantize_act(xs[i], scheme, clip_ub=w.clip_ub, out=qas[i]),
+                              len(xs))
+            r["act_quant_graph_us"] = round(t_g * 1e3, 2)
+            r["act_quant_graph_gbs"] = round(act_bytes / (t_g * 1e-3) / 1e9, 1)
+            r["act_quant_graph_frac_hbm"] = round(act_bytes / (t_g * 1e-3) / 1e9 / pk["hbm_gbs"], 3)
+            del xs, qas
             qw = q8.q8_quantize_weight(Wd, w.weight_scheme, w.weight_codes)
             Y = torch.empty((w.m, w.n), dtype=torch.bfloat16, device=dev)
             t = _time_kernel(lambda: q8.q8_linear_w8a8(qa, qw, out=Y), flush)
@@ -532,11 +677,12 @@ def extras(q8, dev, pk):
             r["gemm_frac_tensor_peak"] = round(tops / int8_peak, 4)
             r["gemm_gbs"] = round(gbytes, 1)
             r["gemm_frac_hbm"] = round(gbytes / pk["hbm_gbs"], 4)
-            if name == "prefill_ffn_up":
+            if name in ("prefill_ffn_up", "fp8_rowwise"):
                 wq_bytes = w.n * w.k * 3 + 8 * w.n
                 t_w = _time_kernel(lambda: q8.q8_quantize_weight(Wd, w.weight_scheme, w.weight_codes), flush, reps=5)
                 r["weight_quant_us"] = round(t_w * 1e3, 1)
                 r["weight_quant_gbs"] = round(wq_bytes / (t_w * 1e-3) / 1e9, 1)
+                r["weight_quant_frac_hbm"] = round(wq_bytes / (t_w * 1e-3) / 1e9 / pk["hbm_gbs"], 3)
             if w.kind == "w8a8_int8":
                 # Static scales (calibrated once; here 1.1 x the batch absmax / 127) and the
                 # linear that re-quantizes its output to INT8 for the next layer.
@@ -634,10 +780,14 @@ def cpu_baseline(name: str, seconds: float = 10.0):
     full steps when one takes under a second, else steps on a row sample."""
     O, w, x32, q = oracle_inputs(name)
     cols = np.arange(w.n)
+    threads = O.threads()
+    # The oracle runs its rows on parallel threads: time a step of one row per
+    # thread, then size the sample so one step takes about a second.
     t0 = time.perf_counter()
-    oracle_step(O, w, x32, q, np.arange(1), cols)
-    per_row = time.perf_counter() - t0
-    rows_n = int(max(1, min(w.m, 1.0 / max(per_row, 1e-9))))
+    oracle_step(O, w, x32, q, np.arange(min(w.m, threads)), cols)
+    per_round = time.perf_counter() - t0
+    rounds = int(max(1, 1.0 / max(per_round, 1e-9)))
+    rows_n = int(min(w.m, threads * rounds))
     rows = np.arange(rows_n)
     ops = 2.0 * rows_n * w.n * w.k
     done, t0 = 0, time.perf_counter()
@@ -648,25 +798,30 @@ def cpu_baseline(name: str, seconds: float = 10.0):
             break
     dt = time.perf_counter() - t0
     what = "full steps" if rows_n == w.m else f"steps on {rows_n} of {w.m} token rows"
-    cores = O.threads()
-    # The same step on one host thread, for a quarter of the time.
+    cores = min(threads, rows_n)
+    # The same work on one host thread, for a quarter of the time, on a row
+    # sample a thread's share of the step (so that one step stays short).
+    rows1 = rows[:max(1, rows_n // max(cores, 1))]
+    ops1 = 2.0 * len(rows1) * w.n * w.k
     O.set_threads(1)
     try:
         done1, t1 = 0, time.perf_counter()
         while True:
-            oracle_step(O, w, x32, q, rows, cols)
+            oracle_step(O, w, x32, q, rows1, cols)
             done1 += 1
             if time.perf_counter() - t1 >= seconds / 4:
                 break
         dt1 = time.perf_counter() - t1
     finally:
-        O.set_threads(cores)
+        O.set_threads(threads)
     return {"value": round(done * ops / dt / 1e12, 6), "unit": UNIT, "cores": cores,
             "kind": "oracle",
             "sample": f"{done} {what} of {name} ({w.m}x{w.n}x{w.k}: activation quantization + "
-                      f"GEMM + epilogue) in {dt:.1f} s; weight quantization excluded as on the GPU",
-            "one_thread": {"value": round(done1 * ops / dt1 / 1e12, 6), "unit": UNIT,
-                           "sample": f"{done1} {what} in {dt1:.1f} s on 1 thread"}}
+                      f"GEMM + epilogue) in {dt:.1f} s on {cores} threads; weight quantization "
+                      "excluded as on the GPU",
+            "one_thread": {"value": round(done1 * ops1 / dt1 / 1e12, 6), "unit": UNIT,
+                           "sample": f"{done1} steps on {len(rows1)} token rows in {dt1:.1f} s "
+                                     "on 1 thread"}}
 
 
 def run_reference(args, world, rank):
@@ -674,17 +829,20 @@ def run_reference(args, world, rank):
         return
     O, w, x32, q = oracle_inputs(args.workload)
     cols_all = np.arange(w.n)
-    # Size each step's sample (one token row x some output columns) so that
-    # warm-up + K steps take about a minute.
+    # Each step's sample: one token row per host thread (the oracle runs rows
+    # on parallel threads) x as many output columns as keep warm-up + K steps
+    # within about a minute.
+    threads = O.threads()
+    nrows = min(w.m, threads)
     t0 = time.perf_counter()
-    oracle_step(O, w, x32, q, np.arange(1), cols_all)
+    oracle_step(O, w, x32, q, np.arange(nrows), cols_all)
     per_col = (time.perf_counter() - t0) / w.n
     budget = 60.0 / max(1, args.steps + args.warmup)
     ncols = int(max(16, min(w.n, budget / max(per_col, 1e-9))))
     cols = cols_all[:ncols]
 
     def step(i):
-        oracle_step(O, w, x32, q, np.array([i % w.m]), cols)
+        oracle_step(O, w, x32, q, (np.arange(nrows) + i * nrows) % w.m, cols)
 
     for i in range(args.warmup):
         step(i)
@@ -692,22 +850,78 @@ def run_reference(args, world, rank):
     for i in range(args.steps):
         step(i)
     dt = time.perf_counter() - t0
-    value = 2.0 * ncols * w.k * args.steps / dt / 1e12
-    sample = (f"each step: 1 token row of the {w.m}x{w.k} {args.workload} input (activation "
-              f"quantization) x {ncols} of {w.n} output columns (GEMM + epilogue)")
+    value = 2.0 * nrows * ncols * w.k * args.steps / dt / 1e12
+    sample = (f"each step: {nrows} token rows of the {w.m}x{w.k} {args.workload} input (activation "
+              f"quantization) x {ncols} of {w.n} output columns (GEMM + epilogue), one row per "
+              "host thread")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3" if w.kind == "w8a8_fp8" else "s8",
             "data": "synthetic",
             "config": {"workload": args.workload, "m_tokens": w.m, "n_out": w.n, "k_in": w.k,
-                       **describe(w), "parallelism": f"dp{world} (independent batches per GPU)",
-                       "timing": "host wall clock of the oracle on the host cores, bounded sample per step"},
-            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": O.threads(),
+                       **describe(w), "parallelism": f"dp{world} (independent batches per GPU)"},
+            "timing": "host wall clock of the oracle on the host cores, bounded sample per step",
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": nrows,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def run_profile(args):
+    """One kernel of a workload, a few launches, for an ncu capture of a
+    small case: 3 warm-up launches, then --steps launches; prints one line
+    with the median launch time (CUDA events)."""
+    from bit_quantized_b200 import q8
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workloads.WORKLOADS[args.workload]
+    X, W, _ = workloads.make_inputs(args.workload)
+    Xd, Wd = X.to(dev), W.to(dev)
+    scheme = "fp8" if w.kind == "w8a8_fp8" else "int8"
+    fn = None
+    if args.profile == "moe":
+        E, n, k, m = 16, 2048, 4096, 4096
+        g = torch.Generator().manual_seed(5)
+        counts = torch.bincount(torch.randint(0, E, (m,), generator=g), minlength=E)
+        off = torch.zeros(E + 1, dtype=torch.int32)
+        off[1:] = torch.cumsum(counts, 0).to(torch.int32)
+        qa = q8.q8_quantize_act(workloads.random_matrix(m, k, torch.bfloat16, 6).to(dev), "fp8", clip_ub=1200.0)
+        qw = q8.q8_quantize_weight(workloads.random_matrix(E * n, k, torch.bfloat16, 7, 0.02).to(dev), "fp8", "e4m3")
+        offd, Y = off.to(dev), torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        fn = lambda: q8.q8_linear_fp8_grouped(qa, qw, E, offd, out=Y)
+    elif args.profile == "weight_quant":
+        fn = lambda: q8.q8_quantize_weight(Wd, w.weight_scheme, w.weight_codes)
+    elif w.kind == "int8_mixed":
+        qw = q8.q8_quantize_weight(Wd, w.weight_scheme, w.weight_codes)
+        Y = torch.empty((w.m, w.n), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, w.m, w.n, w.k),
+                         dtype=torch.uint8, device=dev)
+        fn = lambda: q8.q8_linear_int8_mixed(Xd, qw, w.threshold, out=Y, workspace=ws)
+    else:
+        qw = q8.q8_quantize_weight(Wd, w.weight_scheme, w.weight_codes)
+        qa = q8.q8_quantize_act(Xd, scheme, clip_ub=w.clip_ub)
+        Y = torch.empty((w.m, w.n), dtype=torch.bfloat16, device=dev)
+        if args.profile == "act_quant":
+            fn = lambda: q8.q8_quantize_act(Xd, scheme, clip_ub=w.clip_ub, out=qa)
+        elif args.profile == "gemm":
+            fn = lambda: q8.q8_linear_w8a8(qa, qw, out=Y)
+        else:
+            fn = lambda: q8.q8_linear_w8a8_dynamic(Xd, qw, scheme, clip_ub=w.clip_ub, out=Y, act=qa)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    print(json.dumps({"profile": args.profile, "workload": args.workload, "launches": args.steps,
+                      "median_us": round(float(np.median(ts)), 2)}), flush=True)
 
 
 def main():
@@ -716,12 +930,19 @@ def main():
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=32)
     ap.add_argument("--impl", choices=["q8", "reference"], default="q8")
-    ap.add_argument("--workload", choices=workloads.ORDER, default="decode_q_proj")
+    ap.add_argument("--workload", choices=workloads.ORDER, default="fp8_rowwise")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-library-peaks", action="store_true")
+    ap.add_argument("--profile", choices=["gemm", "step", "act_quant", "weight_quant", "moe"],
+                    default=None, help="run one kernel of the workload a few times (for ncu)")
     args = ap.parse_args()
+    if args.profile is not None:
+        args.steps = 3 if args.steps is None else args.steps
+        run_profile(args)
+        return
     if args.steps is None:
         args.steps = DEFAULT_STEPS[args.workload]
     if args.e2e_steps is None:

@@ -162,6 +162,9 @@ q8_status q8_inject_failure(q8_status code, int32_t skip) {
 
 size_t q8_workspace_size(int op, int64_t m, int64_t n, int64_t k) {
     if (op != Q8_OP_LINEAR_INT8_MIXED || m < 0 || n < 0 || k < 0) return 0;
+    // Beyond 2^31 - 1 no call is valid; the products below would also be
+    // able to overflow int64 there.
+    if (m > kMaxDim || n > kMaxDim || k > kMaxDim) return SIZE_MAX;
     auto up = [](int64_t v, int64_t a) { return (v + a - 1) / a * a; };
     const int64_t kp = up(k, 64);
     int64_t b = 0;
@@ -287,12 +290,18 @@ static q8_status validate_outlier_act(const void* X, q8_dtype x_dtype, int64_t m
     return Q8_OK;
 }
 
+// Two launches: the column absmax pass writes the outlier mask (every token
+// must be seen before any row is coded), then the row pass ranks the outlier
+// columns, codes the regular stream and gathers the fp16 outlier columns of X
+// and, when `w` is given, of the weight.
 static q8_status run_outlier_act(const void* X, int64_t m, int64_t k, int64_t ldx, float threshold,
                                  void* codes, float* scale, int32_t* rowsum, uint8_t* mask,
                                  int32_t* idx, int32_t* count, void* x_outlier, int64_t ldo,
+                                 const q8_weight* w, const void* W16, void* w_outlier,
                                  cudaStream_t s) {
-    cudaError_t e = launch_outlier_columns(X, Q8_F16, m, k, ldx, threshold, mask, idx, count, s);
+    cudaError_t e = launch_outlier_columns(X, Q8_F16, m, k, ldx, threshold, mask, s);
     if (e != cudaSuccess) return launch_status(e);
+    if (m == 0) return launch_status(cudaMemsetAsync(count, 0, sizeof(int32_t), s));   // no rows: no outliers
     RowQuantArgs a = {};
     a.src = X; a.src_dtype = Q8_F16; a.rows = m; a.k = k; a.ld = ldx;
     a.op = kOpActInt8;
@@ -301,6 +310,16 @@ static q8_status run_outlier_act(const void* X, int64_t m, int64_t k, int64_t ld
     a.outlier_idx = idx; a.outlier_count = count;
     a.x_outlier = static_cast<__half*>(x_outlier);
     a.ldo = ldo;
+    if (w != nullptr) {
+        a.w_rows = w->n;
+        a.w_codes = w->codes;
+        a.w_codes_u8 = w->code_dtype == Q8_U8;
+        a.w_ld = W16 ? k : w->ld;
+        a.w_scale = w->scale;
+        a.w_zero = w->zero_point;
+        a.w16 = static_cast<const __half*>(W16);
+        a.w_outlier = static_cast<__half*>(w_outlier);
+    }
     return launch_status(launch_row_quant(a, s));
 }
 
@@ -314,7 +333,8 @@ q8_status q8_outlier_quantize_act(const void* X, q8_dtype x_dtype, int64_t m, in
     st = check_device();
     if (st != Q8_OK) return st;
     return run_outlier_act(X, m, k, ldx, threshold, codes, scale, rowsum, mask, idx, count,
-                           x_outlier, ldo, reinterpret_cast<cudaStream_t>(stream));
+                           x_outlier, ldo, nullptr, nullptr, nullptr,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 q8_status q8_linear_w8a8(const q8_act* x, const q8_weight* w, const float* bias, void* Y,
@@ -461,10 +481,8 @@ q8_status q8_linear_int8_mixed(const void* X, q8_dtype x_dtype, int64_t m, int64
     __half* wo = reinterpret_cast<__half*>(p);
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    st = run_outlier_act(X, m, k, ldx, threshold, codes, sx, rowsum, mask, idx, count, xo, kp, s);
-    if (st != Q8_OK) return st;
-    st = launch_status(launch_gather_weight_outliers(*w, static_cast<const __half*>(W16), idx,
-                                                     count, wo, kp, s));
+    st = run_outlier_act(X, m, k, ldx, threshold, codes, sx, rowsum, mask, idx, count, xo, kp, w,
+                         W16, wo, s);
     if (st != Q8_OK) return st;
     LinearArgs a = {};
     a.m = m; a.n = w->n; a.k = k;

@@ -99,12 +99,17 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Dequant of one accumulator value (int32 path).
+// Dequant of one accumulator value (int32 path): fl32(fl32(acc - Z rowsum) *
+// Sx) * Sw, rounded once per step.  The zero-point correction is exact in
+// 32-bit integers: Z (an integer in [-128, 255] held in fp32), Z rowsum,
+// acc and their difference (= sum_k xq (wq - Z), at most 127 * 255 * K in
+// magnitude) all stay below 2^31 for K <= 32768, and two's-complement
+// subtraction gives the exact difference whenever that fits.
 __device__ __forceinline__ float dequant_int(int32_t acc, float zw, int32_t rs, float sx, float sw,
                                              bool has_zp) {
-    int64_t c = static_cast<int64_t>(acc);
-    if (has_zp) c -= static_cast<int64_t>(zw) * static_cast<int64_t>(rs);
-    float v = __ll2float_rn(c);
+    int32_t c = acc;
+    if (has_zp) c -= __float2int_rn(zw) * rs;
+    float v = __int2float_rn(c);
     v = __fmul_rn(v, sx);
     return __fmul_rn(v, sw);
 }
@@ -175,6 +180,111 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
     const __nv_bfloat16 lo = __float2bfloat16_rn(a), hi = __float2bfloat16_rn(b);
     return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
            (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
+// Dequant epilogue of one accumulator tile for the calling thread's output
+// row: BN columns from n_tile, read from TMEM at `tb` (the warp's 32-lane
+// quarter and the accumulator buffer); the LLM.int8 outlier accumulator sits
+// BN columns further.  Every thread of the warp calls it (tcgen05.ld is
+// warp-wide); rows and columns past the output are computed and not stored.
+template <int BN, int KIND, bool MIXED, bool QOUT>
+__device__ __forceinline__ void epilogue_tile(const EpiParams& p, uint32_t tb, int row, int n_tile,
+                                              int n16_kb) {
+    const bool has_zp = p.zw != nullptr;
+    const bool row_ok = row < p.m;
+    const float sx = row_ok ? p.sx[row] : 0.f;
+    const int32_t rs = (row_ok && has_zp) ? p.rowsum[row] : 0;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        __syncwarp();
+        uint32_t r[32];
+        tmem_ld32(tb + c * 32, r);
+        uint32_t r16[32];
+        if constexpr (MIXED) {
+            if (n16_kb > 0) tmem_ld32(tb + BN + c * 32, r16);
+        }
+        tmem_ld_wait();
+        const int n0 = n_tile + c * 32;
+        if (row_ok && n0 < p.n) {
+        const int nv = (p.n - n0) >= 32 ? 32 : (p.n - n0);   // 16 or 32
+        float out[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (4 * j >= nv) break;
+            const float4 sw4 = *reinterpret_cast<const float4*>(p.sw + n0 + 4 * j);
+            float4 zw4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = zw4;
+            if (has_zp) zw4 = *reinterpret_cast<const float4*>(p.zw + n0 + 4 * j);
+            if (p.bias) b4 = *reinterpret_cast<const float4*>(p.bias + n0 + 4 * j);
+            const float swv[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
+            const float zwv[4] = {zw4.x, zw4.y, zw4.z, zw4.w};
+            const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = 4 * j + e;
+                float v;
+                if constexpr (KIND == kE4M3) {
+                    v = __fmul_rn(__fmul_rn(__uint_as_float(r[i]), sx), swv[e]);
+                } else {
+                    v = dequant_int(static_cast<int32_t>(r[i]), zwv[e], rs, sx, swv[e], has_zp);
+                }
+                if constexpr (MIXED) {
+                    const float y16 = n16_kb > 0 ? __uint_as_float(r16[i]) : 0.0f;
+                    v = __fadd_rn(v, y16);
+                }
+                if (p.bias) v = __fadd_rn(v, bv[e]);
+                out[i] = v;
+            }
+        }
+        if constexpr (QOUT) {
+            const Requant rq = requant_consts(p.out_scale);
+            uint32_t w[8], diff = 0u;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w[j] = requant_codes4(&out[4 * j], rq, diff, 4 * j);
+            if (diff != 0u) {   // rare: outputs near a rounding boundary
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if ((diff >> i) & 1u)
+                        w[i / 4] = (w[i / 4] & ~(0xFFu << (8 * (i % 4)))) |
+                                   (requant_code_slow(out[i], rq.S) << (8 * (i % 4)));
+            }
+            uint4* qp = reinterpret_cast<uint4*>(p.yq + static_cast<int64_t>(row) * p.ldy + n0);
+            qp[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            if (nv > 16) qp[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        } else {
+            uint4* yp = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(row) * p.ldy + n0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (8 * j >= nv) break;
+                yp[j] = make_uint4(pack_bf16(out[8 * j], out[8 * j + 1]),
+                                   pack_bf16(out[8 * j + 2], out[8 * j + 3]),
+                                   pack_bf16(out[8 * j + 4], out[8 * j + 5]),
+                                   pack_bf16(out[8 * j + 6], out[8 * j + 7]));
+            }
+        }
+        if (p.acc_debug) {
+            uint4* ap = reinterpret_cast<uint4*>(static_cast<uint32_t*>(p.acc_debug) +
+                                                 static_cast<int64_t>(row) * p.n + n0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (4 * j >= nv) break;
+                ap[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+            }
+        }
+        if constexpr (MIXED) {
+            if (p.y16_debug) {
+                uint4* dp = reinterpret_cast<uint4*>(p.y16_debug + static_cast<int64_t>(row) * p.n + n0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (4 * j >= nv) break;
+                    if (n16_kb > 0)
+                        dp[j] = make_uint4(r16[4 * j], r16[4 * j + 1], r16[4 * j + 2], r16[4 * j + 3]);
+                    else
+                        dp[j] = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+        }
+        }  // row_ok && n0 < p.n
+    }
 }
 
 // ============================================================================
@@ -343,109 +453,14 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // ------------------------------------------------ epilogue
         pdl_wait();   // scales and row sums may come from the previous kernel
         const int q = warp & 3;  // this warp's TMEM lane quarter
-        const bool has_zp = p.zw != nullptr;
         int buf = 0;
         uint32_t bphase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const int tm = tile % tiles_m, tn = tile / tiles_m;
             if (!mbar_wait(&tfull_bar[buf], bphase, &abort_sh, p.status)) break;
             tc_fence_after();
-            const int row = tm * kBM + q * 32 + lane;
-            const bool row_ok = row < p.m;
-            const float sx = row_ok ? p.sx[row] : 0.f;
-            const int32_t rs = (row_ok && has_zp) ? p.rowsum[row] : 0;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::BUF_COLS;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                __syncwarp();
-                uint32_t r[32];
-                tmem_ld32(tb + c * 32, r);
-                uint32_t r16[32];
-                if constexpr (MIXED) {
-                    if (n16_kb > 0) tmem_ld32(tb + BN + c * 32, r16);
-                }
-                tmem_ld_wait();
-                const int n0 = tn * BN + c * 32;
-                if (row_ok && n0 < p.n) {
-                const int nv = (p.n - n0) >= 32 ? 32 : (p.n - n0);   // 16 or 32
-                float out[32];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    if (4 * j >= nv) break;
-                    const float4 sw4 = *reinterpret_cast<const float4*>(p.sw + n0 + 4 * j);
-                    float4 zw4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = zw4;
-                    if (has_zp) zw4 = *reinterpret_cast<const float4*>(p.zw + n0 + 4 * j);
-                    if (p.bias) b4 = *reinterpret_cast<const float4*>(p.bias + n0 + 4 * j);
-                    const float swv[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
-                    const float zwv[4] = {zw4.x, zw4.y, zw4.z, zw4.w};
-                    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 4 * j + e;
-                        float v;
-                        if constexpr (KIND == kE4M3) {
-                            v = __fmul_rn(__fmul_rn(__uint_as_float(r[i]), sx), swv[e]);
-                        } else {
-                            v = dequant_int(static_cast<int32_t>(r[i]), zwv[e], rs, sx, swv[e], has_zp);
-                        }
-                        if constexpr (MIXED) {
-                            const float y16 = n16_kb > 0 ? __uint_as_float(r16[i]) : 0.0f;
-                            v = __fadd_rn(v, y16);
-                        }
-                        if (p.bias) v = __fadd_rn(v, bv[e]);
-                        out[i] = v;
-                    }
-                }
-                if constexpr (QOUT) {
-                    const Requant rq = requant_consts(p.out_scale);
-                    uint32_t w[8], diff = 0u;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) w[j] = requant_codes4(&out[4 * j], rq, diff, 4 * j);
-                    if (diff != 0u) {   // rare: outputs near a rounding boundary
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if ((diff >> i) & 1u)
-                                w[i / 4] = (w[i / 4] & ~(0xFFu << (8 * (i % 4)))) |
-                                           (requant_code_slow(out[i], rq.S) << (8 * (i % 4)));
-                    }
-                    uint4* qp = reinterpret_cast<uint4*>(p.yq + static_cast<int64_t>(row) * p.ldy + n0);
-                    qp[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    if (nv > 16) qp[1] = make_uint4(w[4], w[5], w[6], w[7]);
-                } else {
-                    uint4* yp = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(row) * p.ldy + n0);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        if (8 * j >= nv) break;
-                        yp[j] = make_uint4(pack_bf16(out[8 * j], out[8 * j + 1]),
-                                           pack_bf16(out[8 * j + 2], out[8 * j + 3]),
-                                           pack_bf16(out[8 * j + 4], out[8 * j + 5]),
-                                           pack_bf16(out[8 * j + 6], out[8 * j + 7]));
-                    }
-                }
-                if (p.acc_debug) {
-                    uint4* ap = reinterpret_cast<uint4*>(static_cast<uint32_t*>(p.acc_debug) +
-                                                         static_cast<int64_t>(row) * p.n + n0);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        if (4 * j >= nv) break;
-                        ap[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-                    }
-                }
-                if constexpr (MIXED) {
-                    if (p.y16_debug) {
-                        uint4* dp = reinterpret_cast<uint4*>(p.y16_debug + static_cast<int64_t>(row) * p.n + n0);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            if (4 * j >= nv) break;
-                            if (n16_kb > 0)
-                                dp[j] = make_uint4(r16[4 * j], r16[4 * j + 1], r16[4 * j + 2], r16[4 * j + 3]);
-                            else
-                                dp[j] = make_uint4(0u, 0u, 0u, 0u);
-                        }
-                    }
-                }
-                }  // row_ok && n0 < p.n
-            }
+            epilogue_tile<BN, KIND, MIXED, QOUT>(p, tb, tm * kBM + q * 32 + lane, tn * BN, n16_kb);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[buf]);
@@ -459,6 +474,199 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ============================================================================
+// Persistent pair kernel: 256 x BN tiles on the two SMs of a CTA pair
+// ============================================================================
+//
+// Clusters of two CTAs.  Each CTA stages its own 128 rows of the activation
+// tile and its own BN/2 rows of the weight tile, so a pair reads 256 + BN
+// operand rows per K slice for a 256 x BN output tile: per SM that is half the
+// weight rows of gemm_tile_kernel's 128 x BN tile for the same MMA work.  The
+// even CTA's MMA warp issues tcgen05.mma.cta_group::2 (M = 256); each CTA's
+// TMEM holds its own 128 accumulator rows, and each CTA's epilogue warps
+// finish their own rows exactly as in gemm_tile_kernel.
+//
+// Barriers: the stage-full barriers of the even CTA count the transaction
+// bytes of both CTAs' loads (each CTA's loads complete on them through
+// cta_group::2 TMA); the MMA's commits arrive on the stage-empty and
+// accumulator-full barriers of both CTAs; the accumulator-empty barriers of
+// the even CTA take one arrival from each epilogue warp of both CTAs.
+template <int BN>
+struct PairCfg {
+    static constexpr int A_BYTES = kBM * kBKB;            // this CTA's 128 activation rows
+    static constexpr int B_BYTES = (BN / 2) * kBKB;       // this CTA's BN/2 weight rows
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int STAGES_RAW = kSmemBudget / STAGE;
+    static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+    static constexpr int BUF_COLS = BN;
+    static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+    static constexpr int SMEM = STAGES * STAGE + 1024;
+    static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "BN");
+    static_assert((BN / 2) % 8 == 0, "weight half-tile rows: whole 8-row swizzle atoms");
+};
+
+template <int BN, int KIND, bool QOUT>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const EpiParams p, int num_kb, int tiles_m, int tiles_n) {
+    using C = PairCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    __shared__ __align__(8) uint64_t full_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_sh;
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_ctarank();          // 0: issues the pair's MMAs
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int npairs = static_cast<int>(gridDim.x >> 1);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], 8);   // 4 epilogue warps x 2 CTAs
+        }
+        mbar_init(&drain_bar, 1);
+        abort_sh = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tmem_base_sh, C::TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    __syncthreads();
+    // Both CTAs' barriers are initialized before either touches the other's.
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+    pdl_launch_dependents();
+
+    const int num_tiles = tiles_m * tiles_n;
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (elect_one()) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            const uint32_t full0 = map_shared_rank(smem_addr(&full_bar[0]), 0);
+            pdl_wait();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+                const int tm = tile % tiles_m, tn = tile / tiles_m;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + stage * C::STAGE;
+                    uint8_t* sb = sa + C::A_BYTES;
+                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE);
+                    const uint32_t fb = full0 + 8u * static_cast<uint32_t>(stage);
+                    tma_load_2d_pair(sa, &tmA, fb, kb * kBKB, tm * (2 * kBM) + static_cast<int>(rank) * kBM);
+                    tma_load_2d_pair(sb, &tmB, fb, kb * kBKB, tn * BN + static_cast<int>(rank) * (BN / 2));
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (even CTA)
+        if (rank == 0 && elect_one()) {
+            const uint32_t idesc = KIND == kE4M3 ? make_idesc(1, 0, 0, 2 * kBM, BN)
+                                                 : make_idesc(2, 1, KIND == kS8U8 ? 0 : 1, 2 * kBM, BN);
+            int stage = 0;
+            uint32_t phase = 0;
+            int buf = 0;
+            uint32_t bphase = 0;
+            bool ok = true;
+            for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+                if (!mbar_wait(&tempty_bar[buf], bphase ^ 1, &abort_sh, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem_base + buf * C::BUF_COLS;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&full_bar[stage], phase, &abort_sh, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_addr(smem + stage * C::STAGE);
+                    const uint64_t ad = sdesc_kmajor_sw128(sa);
+                    const uint64_t bd = sdesc_kmajor_sw128(sa + C::A_BYTES);
+#pragma unroll
+                    for (int ks = 0; ks < kBKB / 32; ++ks) {
+                        if constexpr (KIND == kE4M3)
+                            mma_issue_pair<kKindF8>(d, ad + 2 * ks, bd + 2 * ks, idesc, (kb | ks) != 0);
+                        else
+                            mma_issue_pair<kKindI8>(d, ad + 2 * ks, bd + 2 * ks, idesc, (kb | ks) != 0);
+                    }
+                    tc_commit_pair(&empty_bar[stage], 0x3);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair(&tfull_bar[buf], 0x3);
+                buf ^= 1;
+                if (buf == 0) bphase ^= 1;
+            }
+            if (!ok) {
+                // Abort: wait for the MMAs already issued before TMEM is freed.
+                tc_commit_pair_local(&drain_bar);
+                mbar_wait(&drain_bar, 0, nullptr, nullptr);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue (both CTAs)
+        pdl_wait();
+        const int q = warp & 3;
+        const uint32_t tempty0 = map_shared_rank(smem_addr(&tempty_bar[0]), 0);
+        int buf = 0;
+        uint32_t bphase = 0;
+        for (int tile = pair; tile < num_tiles; tile += npairs) {
+            const int tm = tile % tiles_m, tn = tile / tiles_m;
+            if (!mbar_wait(&tfull_bar[buf], bphase, &abort_sh, p.status)) break;
+            tc_fence_after();
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::BUF_COLS;
+            const int row = tm * (2 * kBM) + static_cast<int>(rank) * kBM + q * 32 + lane;
+            epilogue_tile<BN, KIND, false, QOUT>(p, tb, row, tn * BN, 0);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(buf));
+            buf ^= 1;
+            if (buf == 0) bphase ^= 1;
+        }
+        __syncwarp();
+    }
+
+    __syncthreads();
+    // No CTA leaves while its partner may still signal one of its barriers or
+    // read its shared memory.
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
     }
 }
 
@@ -788,6 +996,70 @@ q8_status run_tile(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     return Q8_OK;
 }
 
+// Pairs that fit on the device at once (clusters of two 1-CTA-per-SM CTAs),
+// cached per kernel instantiation and device.
+template <typename K>
+int max_pairs(K kernel, int smem) {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sm_count() / 2;
+    if (cached[dev] > 0) return cached[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = sm_count() / 2;
+    }
+    cached[dev] = n;
+    return n;
+}
+
+template <int BN, int KIND, bool QOUT = false>
+q8_status run_pair(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
+    using C = PairCfg<BN>;
+    CUtensorMap tA, tB;
+    if (!make_map(&tA, a.a_codes, false, a.k, a.m, a.lda, kBKB, kBM) ||
+        !make_map(&tB, a.b_codes, false, a.k, a.n, a.ldb, kBKB, BN / 2))
+        return Q8_ERR_CUDA;
+    auto kern = gemm_pair_kernel<BN, KIND, QOUT>;
+    if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
+    const int tiles_m = static_cast<int>((a.m + 2 * kBM - 1) / (2 * kBM));
+    const int tiles_n = static_cast<int>((a.n + BN - 1) / BN);
+    const int tiles = tiles_m * tiles_n;
+    const int num_kb = static_cast<int>((a.k + kBKB - 1) / kBKB);
+    const int pairs_max = max_pairs(kern, C::SMEM);
+    const int pairs = tiles < pairs_max ? tiles : pairs_max;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, ep, num_kb, tiles_m, tiles_n) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    return Q8_OK;
+}
+
 template <int NT, int KIND, bool QOUT = false>
 q8_status run_decode(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     using C = DecodeCfg<NT, KIND>;
@@ -845,6 +1117,33 @@ q8_status dispatch_kind(const LinearArgs& a, const EpiParams& ep, cudaStream_t s
     if (a.m <= 16) return run_decode<16, KIND>(a, ep, s);
     if (a.m <= 32) return run_decode<32, KIND>(a, ep, s);
     if (a.m <= 64) return run_decode<64, KIND>(a, ep, s);
+    if (a.m > 2 * kBM) {
+        // 256-row tiles on CTA pairs.  Tile width: the persistent grid's
+        // makespan is ceil(tiles / pairs) tiles of time proportional to BN,
+        // so pick the BN with the smallest waves x BN (the wider on ties).
+        const int64_t pairs = sm_count() / 2;
+        const int cand[3] = {256, 224, 192};
+        int best = 256;
+        int64_t best_cost = INT64_MAX;
+        for (int bn : cand) {
+            const int64_t tiles = ((a.m + 255) / 256) * ((a.n + bn - 1) / bn);
+            const int64_t cost = ((tiles + pairs - 1) / pairs) * bn;
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = bn;
+            }
+        }
+        if constexpr (KIND != kE4M3) {
+            if (a.yq != nullptr) {   // INT8 output codes
+                if (best == 256) return run_pair<256, KIND, true>(a, ep, s);
+                if (best == 224) return run_pair<224, KIND, true>(a, ep, s);
+                return run_pair<192, KIND, true>(a, ep, s);
+            }
+        }
+        if (best == 256) return run_pair<256, KIND>(a, ep, s);
+        if (best == 224) return run_pair<224, KIND>(a, ep, s);
+        return run_pair<192, KIND>(a, ep, s);
+    }
     // Output tile width: the persistent grid's makespan is
     // ceil(tiles / SMs) tiles of time proportional to BN, so pick the BN with
     // the smallest waves x BN (the wider tile on ties).

@@ -31,24 +31,31 @@ struct RowQuantArgs {
     float* scale;          // [rows]
     float* zero_point;     // [rows] or null
     int32_t* rowsum;       // [rows] or null
-    // LLM.int8 gather of the outlier columns (only with skip)
-    const int32_t* outlier_idx;
-    const int32_t* outlier_count;
-    __half* x_outlier;     // rows x ldo, or null
+    // LLM.int8 (only with skip): the kernel ranks the outlier columns itself
+    // (a block-wide scan of the mask) and writes the ascending column list and
+    // the count (outputs), then gathers the outlier columns of X (rows x ldo
+    // fp16, zero-padded to a multiple of 64) and, when w_rows > 0, of the
+    // weight (w_rows x ldo fp16: W16's columns, or S (q - Z) rounded to fp16).
+    int32_t* outlier_idx;
+    int32_t* outlier_count;
+    __half* x_outlier;     // or null
     int64_t ldo;
+    int64_t w_rows;        // 0: no weight gather
+    const void* w_codes;   // w_rows x w_ld int8 / uint8 codes
+    bool w_codes_u8;
+    int64_t w_ld;          // codes' (or W16's) leading dimension
+    const float* w_scale;
+    const float* w_zero;   // or null
+    const __half* w16;     // original fp16 weight (has_fp16_weight), or null
+    __half* w_outlier;     // w_rows x ldo
 };
 
 cudaError_t launch_row_quant(const RowQuantArgs& a, cudaStream_t s);
 
+// Outlier mask of an LLM.int8 call: mask[c] = 1 for the columns c where some
+// row has |x| > threshold (none when threshold <= 0).
 cudaError_t launch_outlier_columns(const void* X, q8_dtype dt, int64_t m, int64_t k, int64_t ldx,
-                                   float threshold, uint8_t* mask, int32_t* idx, int32_t* count,
-                                   cudaStream_t s);
-
-// W16o[n, j] for j < round_up(count, 64): the fp16 outlier columns of the weight
-// (from W16 when given, else dequantized from the codes); zeros past count.
-cudaError_t launch_gather_weight_outliers(const q8_weight& w, const __half* W16,
-                                          const int32_t* idx, const int32_t* count,
-                                          __half* W16o, int64_t ldo, cudaStream_t s);
+                                   float threshold, uint8_t* mask, cudaStream_t s);
 
 cudaError_t launch_dequant(const q8_weight& w, q8_dtype out_dtype, void* out, cudaStream_t s);
 

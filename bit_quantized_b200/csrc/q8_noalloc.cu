@@ -27,6 +27,10 @@ namespace {
 // enough for, e.g., m = 512 tokens with n = k = 4096, since the workspace
 // holds every column as a potential outlier.
 constexpr size_t kScratchBytes = Q8_NOALLOC_SCRATCH_BYTES;
+// Size limits of q8_linear_int8_mixed (M, N <= 2^31 - 1; K <= 32768 for the
+// INT32 accumulator).
+constexpr int64_t kMaxDimNoalloc = (int64_t(1) << 31) - 1;
+constexpr int64_t kMaxKInt8Noalloc = 32768;
 
 // Shared by every call on a device and kept until the process exits.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
@@ -36,7 +40,9 @@ void* g_scratch_addr[kMaxDevices];
 std::mutex g_scratch_mu;
 
 // Device address of this device's scratch; looked up on the first call made
-// on the device (with that device current) and cached for later calls.
+// on the device (with that device current) and cached for later calls.  A
+// cudaDeviceReset destroys the array with the context, so the cached address
+// is only valid until the device is reset (documented in include/q8.h).
 q8_status scratch_address(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -68,8 +74,11 @@ q8_status q8_linear_int8_mixed_noalloc(const void* X, q8_dtype x_dtype, int64_t 
                                        int32_t* acc_debug, float* y16_debug,
                                        q8_stream_t stream) {
     if (!w) return Q8_ERR_NULL;
-    if (m < 0 || w->n < 0 || k <= 0) return Q8_ERR_SHAPE;
-    // Reject, before anything else, sizes whose scratch does not fit.
+    // The sizes the scratch is computed from must be valid ones first (the
+    // same limits q8_linear_int8_mixed applies), then the scratch must fit.
+    if (m < 0 || m > kMaxDimNoalloc || w->n < 0 || w->n > kMaxDimNoalloc || k <= 0 ||
+        k != w->k || k > kMaxKInt8Noalloc)
+        return Q8_ERR_SHAPE;
     if (q8_workspace_size(Q8_OP_LINEAR_INT8_MIXED, m, w->n, k) > kScratchBytes) return Q8_ERR_SHAPE;
     void* scratch = nullptr;
     const q8_status st = scratch_address(&scratch);

@@ -42,6 +42,8 @@ using qm::kFastLimit;
 using qm::kMagic;
 constexpr int kBlock = 256;
 constexpr int kMaxVec = 16;   // 16-byte vectors a thread keeps in registers
+constexpr int kRingMaxStages = 24;        // ring barriers per block (all groups)
+constexpr int kRingBytes = 192 * 1024;    // ring per block (one block per SM)
 
 template <typename T> struct VecOf;
 template <> struct VecOf<__half> { static constexpr int N = 8; };
@@ -97,6 +99,26 @@ __device__ __forceinline__ void group_sync() {
         __syncthreads();
     } else {
         asm volatile("bar.sync %0, %1;" ::"r"(1 + static_cast<int>(threadIdx.x) / TPR), "n"(TPR) : "memory");
+    }
+}
+
+// True when `v` holds on every thread of the TPR-thread row group (a
+// barrier of the group).
+template <int TPR>
+__device__ __forceinline__ bool group_all(bool v) {
+    if constexpr (TPR == 32) {
+        return __all_sync(0xffffffffu, v);
+    } else if constexpr (TPR >= kBlock) {
+        return __syncthreads_and(v) != 0;
+    } else {
+        uint32_t r;
+        asm volatile(
+            "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+            "bar.red.and.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(r)
+            : "r"(static_cast<uint32_t>(v)), "r"(1 + static_cast<int>(threadIdx.x) / TPR), "n"(TPR)
+            : "memory");
+        return r != 0;
     }
 }
 
@@ -461,13 +483,88 @@ __device__ __forceinline__ void accumulate_stats(const uint4 u, RowStats& st, co
     }
 }
 
+// The LLM.int8 outlier columns as one block sees them.  Thread i owns the
+// run of `per` consecutive mask bytes from `begin`, held as bits; `before`
+// outlier columns precede its run, `total` is the count.  A column's rank among
+// the outliers (its slot in the gathered fp16 columns and in the ascending
+// column list) is `before` plus the set bits below it in the run, so the
+// gathers below scatter by rank and need no column list.
+struct OutlierRuns {
+    uint32_t bits[4];   // k <= 32768: runs of at most 128 columns
+    int64_t begin;
+    int per, before, total;
+};
+
+__device__ __forceinline__ OutlierRuns scan_outlier_mask(const uint8_t* mask, int64_t k, int* sh) {
+    OutlierRuns r;
+    r.per = static_cast<int>((k + kBlock - 1) / kBlock);
+    r.begin = static_cast<int64_t>(threadIdx.x) * r.per;
+    int local = 0;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) r.bits[w] = 0u;
+    for (int j = 0; j < r.per; ++j) {
+        const int64_t c = r.begin + j;
+        if (c < k && mask[c] != 0) {
+            r.bits[j / 32] |= 1u << (j % 32);
+            ++local;
+        }
+    }
+    // exclusive scan of `local` over the block
+    const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) sh[warp] = incl;
+    __syncthreads();
+    int before_w = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kBlock / 32; ++w) {
+        const int v = sh[w];
+        if (w < warp) before_w += v;
+        total += v;
+    }
+    __syncthreads();
+    r.before = before_w + incl - local;
+    r.total = total;
+    return r;
+}
+
+// Calls f(column, rank) for every outlier column of this thread's run.
+template <typename F>
+__device__ __forceinline__ void for_each_outlier(const OutlierRuns& r, F&& f) {
+    int rank = r.before;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        uint32_t b = r.bits[w];
+        while (b != 0u) {
+            const int j = __ffs(b) - 1;
+            b &= b - 1u;
+            f(r.begin + 32 * w + j, rank++);
+        }
+    }
+}
+
 // One group of TPR (a multiple of 32) threads per row.  Thread t of a group
 // handles the row's 16-byte vectors t, t + TPR, t + 2 TPR, ...; up to MAXV of
 // them stay in registers between the two passes (longer rows are read twice,
 // the second time from L2).
-template <typename T, int OP, int TPR, int MAXV>
-__global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(RowQuantArgs a) {
+//
+// RING: each group of TPR (32 or 64) threads streams its rows into its own
+// ring of `nstages` shared-memory stages with 1-D bulk copies, issued by the
+// group's first thread as soon as a stage's row has been read into
+// registers.  A group codes one row while the next ones are in flight, and
+// no barrier spans more than the group, so the SM keeps 8 groups' rows of
+// HBM reads outstanding through their reductions and code passes (a
+// persistent grid, one block per SM).  Without RING each thread loads its
+// vectors straight from global memory.
+template <typename T, int OP, int TPR, int MAXV, bool RING = false>
+__global__ void __launch_bounds__(kBlock, RING ? 1 : (MAXV <= 4 ? 4 : 2))
+row_quant_kernel(RowQuantArgs a, int nstages, int64_t stage_bytes, int* status) {
     static_assert(TPR % 32 == 0, "a warp works on one row");
+    static_assert(!RING || TPR == 32 || TPR == 64, "ring groups are one or two warps");
     constexpr int V = VecOf<T>::N;
     constexpr int RPB = kBlock / TPR;
     constexpr bool kSkip = OP == kOpActInt8Skip;
@@ -478,10 +575,27 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
     __shared__ int redi[kBlock / 32];
     __shared__ FixQueue fixq[kBlock / 32];
     __shared__ float cshare[kBlock / TPR][8];
+    extern __shared__ __align__(128) uint8_t ring[];   // RING: RPB groups x nstages x stage_bytes
+    __shared__ __align__(8) uint64_t ring_full[RING ? kRingMaxStages : 1];
+    __shared__ int ring_abort[RING ? kBlock / TPR : 1];
     FixQueue* q = &fixq[threadIdx.x / 32];
+    const uint32_t row_bytes = static_cast<uint32_t>(a.k * static_cast<int64_t>(sizeof(T)));
+    if constexpr (RING) {
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < RPB * nstages; ++i) mbar_init(&ring_full[i], 1);
+            for (int i = 0; i < RPB; ++i) ring_abort[i] = 0;
+            fence_barrier_init();
+        }
+        __syncthreads();
+    }
 
     const int g = threadIdx.x / TPR;
     const int t = threadIdx.x % TPR;
+    // RING: this group's stages and barriers; its rows are gid, gid + G, ...
+    uint8_t* gring = ring + static_cast<int64_t>(g) * nstages * stage_bytes;
+    uint64_t* gfull = &ring_full[RING ? g * nstages : 0];
+    const int64_t gid = static_cast<int64_t>(blockIdx.x) * RPB + g;
+    const int64_t G = static_cast<int64_t>(gridDim.x) * RPB;
     const int64_t nvec = a.k / V;
     const bool cached = nvec <= static_cast<int64_t>(TPR) * MAXV;
     // Vectors this thread holds when the row is cached, and the most any
@@ -499,9 +613,37 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
                   OP == kOpActInt8Smooth)
         pdl_launch_dependents();
     pdl_wait();
+    // RING: the group's row of iteration i (gid + i G) goes to its stage i % nstages.
+    auto ring_issue = [&](int64_t it) {
+        const int64_t r = gid + it * G;
+        if (r < a.rows) {
+            const int st = static_cast<int>(it % nstages);
+            mbar_arrive_expect_tx(&gfull[st], row_bytes);
+            bulk_load(gring + st * stage_bytes, static_cast<const T*>(a.src) + r * a.ld, row_bytes,
+                      &gfull[st]);
+        }
+    };
+    if constexpr (RING) {
+        if (t == 0)
+            for (int i = 0; i < nstages; ++i) ring_issue(i);
+    }
 
+    // LLM.int8: rank the outlier columns; block 0 publishes the ascending
+    // column list and the count (read by the GEMM that follows).
+    OutlierRuns oruns;
+    int cpad = 0;
+    if constexpr (kSkip) {
+        oruns = scan_outlier_mask(a.skip, a.k, redi);
+        cpad = (oruns.total + 63) / 64 * 64;
+        if (blockIdx.x == 0) {
+            for_each_outlier(oruns, [&](int64_t c, int rank) { a.outlier_idx[rank] = static_cast<int32_t>(c); });
+            if (threadIdx.x == 0) *a.outlier_count = oruns.total;
+        }
+    }
+
+    int64_t it = 0;
     for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * RPB; row0 < a.rows;
-         row0 += static_cast<int64_t>(gridDim.x) * RPB) {
+         row0 += static_cast<int64_t>(gridDim.x) * RPB, ++it) {
         const int64_t row = row0 + g;
         const bool active = row < a.rows;   // the same for a whole warp
         const T* src_row = static_cast<const T*>(a.src) + (active ? row : 0) * a.ld;
@@ -527,11 +669,36 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
         // rows only count loaded vectors.  Left-out columns are zeroed.
         uint4 raw[MAXV];
         RowStats st{0.f, FLT_MAX, -FLT_MAX};
+        const uint8_t* srow = RING ? gring + (it % nstages) * stage_bytes : nullptr;
+        if constexpr (RING) {
+            // Every thread of the group waits for the row's bytes; the group
+            // decides together (a wait that ran out stops the group before any
+            // barrier of the row's reduction).
+            if (active) {   // uniform per group
+                const bool ok = mbar_wait(&gfull[it % nstages], static_cast<uint32_t>((it / nstages) & 1),
+                                          &ring_abort[g], status);
+                if (!group_all<TPR>(ok)) {
+                    if (t == 0) {
+                        // Let the copies still in flight land before the block exits.
+                        for (int64_t j = it; j < it + nstages; ++j)
+                            if (gid + j * G < a.rows)
+                                mbar_wait(&gfull[j % nstages], static_cast<uint32_t>((j / nstages) & 1),
+                                          nullptr, nullptr);
+                    }
+                    break;
+                }
+            }
+        }
         auto pass1 = [&](auto full_tag) {
             constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
-            for (int i = 0; i < MAXV; ++i)
-                raw[i] = (FULL || i < nv) ? ld_stream16(src + i * TPR * V) : make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < MAXV; ++i) {
+                if constexpr (RING)
+                    raw[i] = (FULL || i < nv) ? ld_shared16(srow + (static_cast<int64_t>(t) + i * TPR) * 16)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+                else
+                    raw[i] = (FULL || i < nv) ? ld_stream16(src + i * TPR * V) : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
             for (int i = 0; i < MAXV; ++i) {
                 if (FULL || i < nv) {
@@ -569,6 +736,15 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
         }
         st.amax = fmaxf(st.hi, -st.lo);
         st = group_reduce<TPR, OP == kOpWeightAsym>(st, red);
+        if constexpr (RING) {
+            // Every thread of the group has read its vectors of this stage
+            // (they fed the reduction): it can take the row nstages further on.
+            __syncwarp();
+            if (t == 0) {
+                fence_proxy_async_smem();
+                ring_issue(it + nstages);
+            }
+        }
         if constexpr (OP != kOpWeightAsym) st.amax = fmaxf(st.amax, 0.0f);
 
         RowConsts c;
@@ -678,19 +854,47 @@ __global__ void __launch_bounds__(kBlock, MAXV <= 4 ? 4 : 2) row_quant_kernel(Ro
                 if (a.zero_point) a.zero_point[row] = 0.0f;
             }
         }
-        // LLM.int8: gather the outlier columns of this row into fp16, zero-padded
-        // to a multiple of 64 columns for the tensor-core outlier GEMM.
+        // LLM.int8: gather the outlier columns of this iteration's rows into
+        // fp16 by rank, zero-padded to a multiple of 64 columns for the
+        // tensor-core outlier GEMM (the whole block works on each row).
         if constexpr (kSkip) {
-            if (active && a.x_outlier != nullptr) {
-                const int cnt = *a.outlier_count;
-                const int cpad = (cnt + 63) / 64 * 64;
-                __half* xo = a.x_outlier + row * a.ldo;
-                for (int j = t; j < cpad; j += TPR) {
-                    __half h = __float2half_rn(0.0f);
-                    if (j < cnt) h = src_row[a.outlier_idx[j]];
-                    xo[j] = h;
+            if (a.x_outlier != nullptr) {
+                for (int i = 0; i < RPB; ++i) {
+                    const int64_t r = row0 + i;
+                    if (r >= a.rows) break;
+                    const T* xs = static_cast<const T*>(a.src) + r * a.ld;
+                    __half* xo = a.x_outlier + r * a.ldo;
+                    for_each_outlier(oruns, [&](int64_t c, int rank) { xo[rank] = xs[c]; });
+                    for (int j = oruns.total + static_cast<int>(threadIdx.x); j < cpad; j += kBlock)
+                        xo[j] = __float2half_rn(0.0f);
                 }
             }
+        }
+    }
+
+    // LLM.int8: the fp16 outlier columns of the weight, by rank and
+    // zero-padded like X's: W16's own columns, or the dequantized codes
+    // fp16(fl32(S (q - Z))) when only the 8-bit weight is kept.
+    if constexpr (kSkip) {
+        for (int64_t r = blockIdx.x; r < a.w_rows; r += gridDim.x) {
+            __half* wo = a.w_outlier + r * a.ldo;
+            const float S = a.w_scale[r];
+            const float Zr = a.w_zero ? a.w_zero[r] : 0.0f;
+            for_each_outlier(oruns, [&](int64_t c, int rank) {
+                __half h;
+                if (a.w16 != nullptr) {
+                    h = a.w16[r * a.w_ld + c];
+                } else {
+                    const float q = a.w_codes_u8
+                                        ? static_cast<float>(static_cast<const uint8_t*>(a.w_codes)[r * a.w_ld + c])
+                                        : static_cast<float>(static_cast<const int8_t*>(a.w_codes)[r * a.w_ld + c]);
+                    const float d = a.w_zero ? __fsub_rn(q, Zr) : q;
+                    h = __float2half_rn(__fmul_rn(S, d));
+                }
+                wo[rank] = h;
+            });
+            for (int j = oruns.total + static_cast<int>(threadIdx.x); j < cpad; j += kBlock)
+                wo[j] = __float2half_rn(0.0f);
         }
     }
 }
@@ -699,6 +903,7 @@ template <typename T, int OP>
 cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
     constexpr int V = VecOf<T>::N;
     const int64_t nvec = a.k / V;
+    int* status = device_status_ptr();
     auto go = [&](auto tpr_tag, auto maxv_tag) -> cudaError_t {
         constexpr int TPR = decltype(tpr_tag)::value;
         constexpr int MAXV = decltype(maxv_tag)::value;
@@ -715,8 +920,55 @@ cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, row_quant_kernel<T, OP, TPR, MAXV>, a);
+        return cudaLaunchKernelEx(&cfg, row_quant_kernel<T, OP, TPR, MAXV>, a, 0, int64_t(0), status);
     };
+    // Ring configuration (large matrices): one persistent block per SM whose
+    // row groups of 32 or 64 threads stream their rows through at least two
+    // stages each, when a row fits the group's registers (16 vectors a thread).
+    auto go_ring = [&](auto tpr_tag, auto maxv_tag) -> cudaError_t {
+        constexpr int TPR = decltype(tpr_tag)::value;
+        constexpr int MAXV = decltype(maxv_tag)::value;
+        constexpr int RPB = kBlock / TPR;
+        const int64_t row_bytes = a.k * static_cast<int64_t>(sizeof(T));
+        const int64_t stage_bytes = (row_bytes + 127) / 128 * 128;
+        int nstages = static_cast<int>(kRingBytes / (RPB * stage_bytes));
+        if (nstages > kRingMaxStages / RPB) nstages = kRingMaxStages / RPB;
+        int sms = 148, dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        int64_t blocks = (a.rows + RPB - 1) / RPB;
+        if (blocks > sms) blocks = sms;
+        auto kern = row_quant_kernel<T, OP, TPR, MAXV, true>;
+        const int dyn = static_cast<int>(RPB * nstages * stage_bytes);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
+        cfg.blockDim = dim3(kBlock, 1, 1);
+        cfg.dynamicSmemBytes = static_cast<size_t>(dyn);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kern, a, nstages, stage_bytes, status);
+    };
+    {
+        const int64_t row_bytes = a.k * static_cast<int64_t>(sizeof(T));
+        const int64_t stage_bytes = (row_bytes + 127) / 128 * 128;
+        const bool aligned = (a.ld * static_cast<int64_t>(sizeof(T))) % 16 == 0 &&
+                             (reinterpret_cast<uintptr_t>(a.src) & 15u) == 0;
+        if (aligned && a.rows >= 4 * 148) {
+            using W1 = std::integral_constant<int, 32>;
+            using W2 = std::integral_constant<int, 64>;
+            if (nvec <= 32 * 4) return go_ring(W1{}, std::integral_constant<int, 4>{});
+            if (nvec <= 32 * 8) return go_ring(W1{}, std::integral_constant<int, 8>{});
+            if (nvec <= 32 * 16 && 2 * 8 * stage_bytes <= kRingBytes)
+                return go_ring(W1{}, std::integral_constant<int, 16>{});
+            if (nvec <= 64 * 16 && 2 * 4 * stage_bytes <= kRingBytes)
+                return go_ring(W2{}, std::integral_constant<int, 16>{});
+        }
+    }
     using T128 = std::integral_constant<int, 128>;
     using T256 = std::integral_constant<int, 256>;
     using C2 = std::integral_constant<int, 2>;
@@ -803,70 +1055,6 @@ __global__ void __launch_bounds__(kBlock) outlier_colmax_kernel(const T* __restr
     }
 }
 
-// Ordered compaction of the mask into idx[0..count): one block of 1024 threads,
-// each owning a contiguous run of columns.
-__global__ void __launch_bounds__(1024) outlier_scan_kernel(const uint8_t* __restrict__ mask,
-                                                            int64_t k, int32_t* __restrict__ idx,
-                                                            int32_t* __restrict__ count) {
-    __shared__ int warp_tot[32];
-    const int tid = threadIdx.x;
-    const int64_t per = (k + 1023) / 1024;
-    const int64_t b = tid * per, e = (b + per < k) ? b + per : k;
-    int local = 0;
-    for (int64_t c = b; c < e; ++c) local += mask[c] ? 1 : 0;
-    // block exclusive scan of `local`
-    const int lane = tid % 32, warp = tid / 32;
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int w = warp_tot[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += y;
-        }
-        warp_tot[lane] = w;  // inclusive over warps
-    }
-    __syncthreads();
-    int pos = incl - local + (warp > 0 ? warp_tot[warp - 1] : 0);
-    for (int64_t c = b; c < e; ++c)
-        if (mask[c]) idx[pos++] = static_cast<int32_t>(c);
-    if (tid == 1023) *count = warp_tot[31];
-}
-
-// fp16 outlier columns of the weight: 256 threads per row, rows by blocks.
-__global__ void __launch_bounds__(kBlock) gather_weight_outliers_kernel(
-    const void* __restrict__ codes, int code_u8, int64_t ldq, const float* __restrict__ S,
-    const float* __restrict__ Z, const __half* __restrict__ W16, int64_t n,
-    const int32_t* __restrict__ idx, const int32_t* __restrict__ count, __half* __restrict__ out,
-    int64_t ldo) {
-    const int cnt = *count;
-    const int cpad = (cnt + 63) / 64 * 64;
-    for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
-        for (int j = threadIdx.x; j < cpad; j += blockDim.x) {
-            __half h = __float2half_rn(0.0f);
-            if (j < cnt) {
-                const int64_t c = idx[j];
-                if (W16 != nullptr) {
-                    h = W16[r * ldq + c];
-                } else {
-                    const float q = code_u8 ? static_cast<float>(static_cast<const uint8_t*>(codes)[r * ldq + c])
-                                            : static_cast<float>(static_cast<const int8_t*>(codes)[r * ldq + c]);
-                    const float d = Z ? __fsub_rn(q, Z[r]) : q;
-                    h = __float2half_rn(__fmul_rn(S[r], d));
-                }
-            }
-            out[r * ldo + j] = h;
-        }
-    }
-}
-
 __global__ void dequant_kernel(const void* __restrict__ codes, int code_dtype, int64_t n, int64_t k,
                                int64_t ldq, const float* __restrict__ S,
                                const float* __restrict__ Z, int out_dtype, void* __restrict__ out) {
@@ -903,8 +1091,7 @@ cudaError_t launch_row_quant(const RowQuantArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_outlier_columns(const void* X, q8_dtype dt, int64_t m, int64_t k, int64_t ldx,
-                                   float threshold, uint8_t* mask, int32_t* idx, int32_t* count,
-                                   cudaStream_t s) {
+                                   float threshold, uint8_t* mask, cudaStream_t s) {
     const unsigned blocks = static_cast<unsigned>((k + 31) / 32);
     if (dt == Q8_F16)
         outlier_colmax_kernel<__half><<<blocks, kBlock, 0, s>>>(static_cast<const __half*>(X), m, k,
@@ -912,19 +1099,6 @@ cudaError_t launch_outlier_columns(const void* X, q8_dtype dt, int64_t m, int64_
     else
         outlier_colmax_kernel<__nv_bfloat16><<<blocks, kBlock, 0, s>>>(
             static_cast<const __nv_bfloat16*>(X), m, k, ldx, threshold, mask);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    outlier_scan_kernel<<<1, 1024, 0, s>>>(mask, k, idx, count);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_gather_weight_outliers(const q8_weight& w, const __half* W16,
-                                          const int32_t* idx, const int32_t* count, __half* W16o,
-                                          int64_t ldo, cudaStream_t s) {
-    int64_t blocks = w.n < 65535 ? w.n : 65535;
-    gather_weight_outliers_kernel<<<static_cast<unsigned>(blocks), kBlock, 0, s>>>(
-        w.codes, w.code_dtype == Q8_U8 ? 1 : 0, W16 ? w.k : w.ld, w.scale, w.zero_point, W16, w.n,
-        idx, count, W16o, ldo);
     return cudaGetLastError();
 }
 

@@ -45,7 +45,7 @@ EXPORTED = [
     "q8_linear_fp8_grouped",
     "q8_workspace_size", "q8_status_string",
     "q8_get_device_status", "q8_clear_device_status", "q8_device_check", "q8_version",
-    "q8_inject_failure",
+    "q8_inject_failure", "q8_selftest_wait_timeout",
 ]
 
 
@@ -100,6 +100,7 @@ _SIG = {
     "q8_clear_device_status": ([_vp], _int),
     "q8_device_check": ([], _int),
     "q8_inject_failure": ([_int, ctypes.c_int32], _int),
+    "q8_selftest_wait_timeout": ([ctypes.c_int32, _vp], _int),
     "q8_version": ([], _int),
 }
 for _name, (_args, _res) in _SIG.items():
@@ -494,3 +495,11 @@ def q8_get_device_status(stream=None) -> int:
 
 def q8_clear_device_status(stream=None) -> None:
     _check(_lib.q8_clear_device_status(_stream(stream)), "q8_clear_device_status")
+
+
+def q8_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Enqueue the failure-detection self-test: a kernel whose bounded barrier
+    wait runs out after `limit_us` microseconds and records
+    Q8_ERR_DEVICE_TIMEOUT in the device status word (q8_get_device_status)."""
+    _check(_lib.q8_selftest_wait_timeout(int(limit_us), _stream(stream)),
+           "q8_selftest_wait_timeout")

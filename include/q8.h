@@ -66,7 +66,7 @@
 extern "C" {
 #endif
 
-#define Q8_VERSION 7
+#define Q8_VERSION 8
 
 /* Same object as cudaStream_t. */
 typedef struct CUstream_st *q8_stream_t;
@@ -482,6 +482,9 @@ q8_status q8_linear_int8_mixed(const void *X, q8_dtype x_dtype, int64_t m, int64
  *   Set-up    the first call on each device looks up the array's device
  *             address (cudaGetSymbolAddress, with that device current) and
  *             caches it; make that first call before any stream capture.
+ *             cudaDeviceReset destroys the array with the context, and the
+ *             cached address with it: do not call this entry point on a
+ *             device after resetting it in the same process.
  *   Sharing   every call on a device uses the same scratch, which keeps the
  *             last call's contents (nothing in it needs to start at zero).
  *             Calls whose executions overlap on the GPU (other streams, other
@@ -500,7 +503,9 @@ enum { Q8_OP_LINEAR_W8A8 = 0, Q8_OP_LINEAR_INT8_MIXED = 1 };
 
 /* Bytes of device workspace an operation needs for these sizes (host function,
  * no device access).  The mixed operation sizes its outlier buffers for every
- * column being an outlier, so no call can overflow them. */
+ * column being an outlier, so no call can overflow them.  Returns 0 for an
+ * operation that needs none or for negative sizes, and SIZE_MAX when a size
+ * exceeds 2^31 - 1 (no such call is valid). */
 size_t q8_workspace_size(int op, int64_t m, int64_t n, int64_t k);
 
 /* Static, NUL-terminated description of a status code (host). */
@@ -513,6 +518,23 @@ q8_status q8_get_device_status(int32_t *out, q8_stream_t stream);
 
 /* Resets the current device's status word to Q8_OK (enqueued on `stream`). */
 q8_status q8_clear_device_status(q8_stream_t stream);
+
+/*
+ * Self-test of the device-side failure detection described under "Errors"
+ * above (the pages have no counterpart: it tests this library's own
+ * bounded waits).  Enqueues on `stream` one CTA with the GEMM kernels' roles
+ * (a TMA producer warp, an MMA warp and four epilogue warps sharing an abort
+ * flag, with tensor memory allocated) whose producer waits on a barrier that
+ * nothing ever arrives on, bounded by `limit_us` microseconds instead of the
+ * usual second.  When the wait runs out the kernel records
+ * Q8_ERR_DEVICE_TIMEOUT in the current device's status word, the other roles
+ * leave their waits on the abort flag, the CTA frees its tensor memory and
+ * returns: nothing faults or hangs and the context stays usable.  Read the
+ * result with q8_get_device_status and reset it with q8_clear_device_status.
+ * Returns Q8_ERR_SHAPE unless 1 <= limit_us <= 1000000, else Q8_OK once the
+ * kernel is enqueued (or the q8_device_check status).
+ */
+q8_status q8_selftest_wait_timeout(int32_t limit_us, q8_stream_t stream);
 
 /* Q8_OK when the current device can run this library, else
  * Q8_ERR_UNSUPPORTED_ARCH or Q8_ERR_CUDA (host). */

@@ -62,6 +62,46 @@ def test_workspace_size():
     assert q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, 1, 16, 32) > 0
 
 
+def test_workspace_size_out_of_range_sizes():
+    # Sizes beyond 2^31 - 1 are never valid: the size function answers
+    # SIZE_MAX instead of a product that could overflow into a small number.
+    size_max = 2**64 - 1
+    big = 2**31
+    assert q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, big, 16, 32) == size_max
+    assert q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, 16, 2**62, 32) == size_max
+    assert q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, 16, 16, 2**62) == size_max
+    assert q8.q8_workspace_size(q8.Q8_OP_LINEAR_INT8_MIXED, -1, 16, 32) == 0
+
+
+def test_noalloc_validation_before_sizing():
+    # The allocation-free entry point checks K against the weight and the
+    # INT32 bound, and M against 2^31 - 1, before it sizes its scratch; all of
+    # these fail without touching the device.
+    f = L.q8_linear_int8_mixed_noalloc
+    w = _weight(k=128, ld=128)
+
+    def call(m=16, k=128, w=w):
+        return f(FAKE, q8.Q8_F16, m, k, k, ctypes.byref(w), None, 6.0, None, FAKE, w.n, None, None,
+                 None, None, _ns)
+    assert f(FAKE, q8.Q8_F16, 16, 128, 128, None, None, 6.0, None, FAKE, 64, None, None, None,
+             None, _ns) == q8.Q8_ERR_NULL
+    assert call(k=256) == q8.Q8_ERR_SHAPE                       # k != w->k
+    assert call(m=-1) == q8.Q8_ERR_SHAPE
+    assert call(m=2**40) == q8.Q8_ERR_SHAPE                     # beyond 2^31 - 1
+    wk = _weight(k=65536, ld=65536)
+    assert call(k=65536, w=wk) == q8.Q8_ERR_SHAPE               # beyond the INT32 bound
+    assert call(m=2**20, k=128) == q8.Q8_ERR_SHAPE              # scratch does not fit
+
+
+def test_selftest_wait_timeout_validation():
+    assert L.q8_selftest_wait_timeout(0, _ns) == q8.Q8_ERR_SHAPE
+    assert L.q8_selftest_wait_timeout(-5, _ns) == q8.Q8_ERR_SHAPE
+    assert L.q8_selftest_wait_timeout(1000001, _ns) == q8.Q8_ERR_SHAPE
+    if NO_GPU:
+        assert L.q8_selftest_wait_timeout(1000, _ns) in (q8.Q8_ERR_CUDA,
+                                                         q8.Q8_ERR_UNSUPPORTED_ARCH)
+
+
 L = q8.lib()
 _ns = None
 

@@ -3,7 +3,9 @@ allocate device memory, against q8_linear_int8_mixed with a caller workspace.
 
 The allocation-free entry point runs the same kernels on a scratch array the
 library owns, so on the same inputs its output must equal the workspace entry
-point's.  The calls go straight through the C ABI.  Two different problems are
+point's: the output and the debug copies (outlier mask and count, INT32
+accumulators, fp32 outlier stream) that come out of the library's scratch.
+The calls go straight through the C ABI.  Two different problems are
 run back to back (the scratch keeps the previous call's contents), then the
 first one again.  This file is collected last on purpose.
 """
@@ -27,13 +29,16 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _noalloc(X, qw, threshold, Y, bias=None):
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _noalloc(X, qw, threshold, Y, bias=None, mask=None, count=None, acc=None, y16=None):
     cw = qw.c()
     m, k = X.shape
     return q8.lib().q8_linear_int8_mixed_noalloc(
-        ctypes.c_void_p(X.data_ptr()), q8.Q8_F16, m, k, X.stride(0), ctypes.byref(cw), None,
-        float(threshold), None if bias is None else ctypes.c_void_p(bias.data_ptr()),
-        ctypes.c_void_p(Y.data_ptr()), Y.stride(0), None, None, None, None, _stream())
+        _ptr(X), q8.Q8_F16, m, k, X.stride(0), ctypes.byref(cw), None, float(threshold),
+        _ptr(bias), _ptr(Y), Y.stride(0), _ptr(mask), _ptr(count), _ptr(acc), _ptr(y16), _stream())
 
 
 def _case(seed, m, n, k, outlier_cols):
@@ -44,15 +49,28 @@ def _case(seed, m, n, k, outlier_cols):
 
 
 def _check(X, qw, threshold, what, bias=None):
-    m, n = X.shape[0], qw.codes.shape[0]
-    Y_ref = q8.q8_linear_int8_mixed(X, qw, threshold, bias=bias)
+    """The allocation-free call against the workspace entry point: output,
+    outlier mask and count, INT32 accumulators and the fp32 outlier stream,
+    all copied out of the library's scratch, must be bit-identical."""
+    m, k = X.shape
+    n = qw.codes.shape[0]
+    Y_ref, dbg = q8.q8_linear_int8_mixed(X, qw, threshold, bias=bias, debug=True)
     Y = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device=DEV)
-    assert _noalloc(X, qw, threshold, Y, bias) == q8.Q8_OK, what
+    mask = torch.full((k,), 0xAB, dtype=torch.uint8, device=DEV)
+    count = torch.full((1,), -1, dtype=torch.int32, device=DEV)
+    acc = torch.full((m, n), 0x7EADBEEF, dtype=torch.int32, device=DEV)
+    y16 = torch.full((m, n), float("nan"), dtype=torch.float32, device=DEV)
+    assert _noalloc(X, qw, threshold, Y, bias, mask, count, acc, y16) == q8.Q8_OK, what
     torch.cuda.synchronize()
     ref_bits = P.bf16_bits(Y_ref)
     got_bits = P.bf16_bits(Y)
     P.assert_bf16_within(got_bits, P.bf16_values(ref_bits), 0.0, what)
-    P.assert_equal(got_bits, ref_bits, what)
+    P.assert_equal(got_bits, ref_bits, what + " Y")
+    P.assert_equal(mask.cpu().numpy(), dbg["mask"].cpu().numpy(), what + " mask")
+    assert int(count.item()) == int(dbg["count"].item()), what + " count"
+    P.assert_equal(acc.cpu().numpy(), dbg["acc"].cpu().numpy(), what + " acc")
+    P.assert_equal(y16.cpu().numpy().view(np.uint32), dbg["y16"].cpu().numpy().view(np.uint32),
+                   what + " y16")
 
 
 def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():

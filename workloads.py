@@ -116,3 +116,49 @@ def bits16(t: torch.Tensor):
     import numpy as np
     assert t.dtype in (torch.float16, torch.bfloat16)
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------- exact-arithmetic inputs
+#
+# Inputs whose products and partial sums are all exactly representable in
+# fp32, so that any summation order gives the same accumulator.  They carry
+# no quantization arithmetic: small integers, powers of two, and weights laid
+# on a grid whose per-row (or per-group) range is fixed by construction.
+
+def small_int_matrix(rows: int, cols: int, seed: int, lim: int) -> torch.Tensor:
+    """Seeded fp32 matrix of integers drawn uniformly from [-lim, lim]."""
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(-lim, lim + 1, (rows, cols), generator=g).float()
+
+
+def pow2_vector(n: int, seed: int, lo: int, hi: int) -> torch.Tensor:
+    """Seeded fp32 vector of powers of two 2^e, e drawn uniformly from [lo, hi)."""
+    g = torch.Generator().manual_seed(seed)
+    return torch.exp2(torch.randint(lo, hi, (n,), generator=g).float())
+
+
+def grid_rows(rows: int, cols: int, seed: int, step_exp: int) -> torch.Tensor:
+    """Rows of integers in [-128, 127] times 2^step_exp, each row holding both
+    -128 and 127 (at seeded positions), so every row spans exactly 255 grid
+    steps."""
+    g = torch.Generator().manual_seed(seed)
+    v = torch.randint(-128, 128, (rows, cols), generator=g)
+    perm = torch.argsort(torch.rand(rows, cols, generator=g), dim=1)
+    r = torch.arange(rows)
+    v[r, perm[:, 0]] = -128
+    v[r, perm[:, 1]] = 127
+    return v.float() * 2.0 ** step_exp
+
+
+def group_grid(rows: int, cols: int, group: int, seed: int, lo: int, hi: int) -> torch.Tensor:
+    """Each run of `group` consecutive values along a row is 2^e times integers
+    in [-7, 7] (e drawn from [lo, hi) per run), and holds +-7 * 2^e at a seeded
+    position, so the run's absolute maximum is exactly 7 * 2^e."""
+    assert cols % group == 0
+    g = torch.Generator().manual_seed(seed)
+    v = torch.randint(-7, 8, (rows, cols // group, group), generator=g).float()
+    e = torch.randint(lo, hi, (rows, cols // group, 1), generator=g).float()
+    pos = torch.randint(0, group, (rows, cols // group), generator=g)
+    sign = torch.randint(0, 2, (rows, cols // group), generator=g).float() * 2 - 1
+    v.scatter_(2, pos.unsqueeze(2), (7 * sign).unsqueeze(2))
+    return (v * torch.exp2(e)).reshape(rows, cols)
