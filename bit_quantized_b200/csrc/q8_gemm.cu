@@ -51,6 +51,8 @@ constexpr int kBM = 128;        // MMA M (TMEM lanes)
 constexpr int kBKB = 128;       // bytes of K per pipeline stage (one 128-byte swizzle row)
 constexpr int kThreads = 192;
 constexpr int kSmemBudget = 200 * 1024;
+constexpr int kEpiStageBytes = 4 * 2 * 2048;   // output staging per CTA: 4 epilogue warps x 2 buffers
+constexpr int kEpiConstBytes = 4 * 3 * 256 * 4; // column constants per CTA: 4 warps x 3 x BN (<= 256) floats
 
 enum GemmKind { kS8S8 = 0, kS8U8 = 1, kE4M3 = 2 };
 
@@ -82,7 +84,7 @@ struct TileCfg {
     static constexpr int USED_COLS = 2 * BUF_COLS;
     static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64
                                    : USED_COLS <= 128 ? 128 : USED_COLS <= 256 ? 256 : 512;
-    static constexpr int SMEM = STAGES * STAGE + 1024;
+    static constexpr int SMEM = STAGES * STAGE + kEpiStageBytes + kEpiConstBytes + 1024;
     static_assert(USED_COLS <= 512, "TMEM holds 512 columns");
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
 };
@@ -176,10 +178,75 @@ __device__ __forceinline__ uint32_t requant_code_fast(float y, const Requant& c)
     return requant_code_slow(y, c.S);
 }
 
+// bf16_rne(a) in the low half, bf16_rne(b) in the high half (one conversion).
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-    const __nv_bfloat16 lo = __float2bfloat16_rn(a), hi = __float2bfloat16_rn(b);
-    return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
-           (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Output path of the bf16 epilogue.  With a tensor map, each warp stages its
+// 32 x 32 output chunk (rows of 64 bytes, 16-byte chunks swizzled by
+// (row / 2) % 4, which is TMA's 64-byte swizzle and keeps the 32 lanes' writes
+// free of bank conflicts) in one of two 2 KB buffers of its own, and one lane
+// stores it with a TMA tensor store that clips rows and columns past the
+// output.  The store runs asynchronously, so it overlaps the next chunk and the
+// next tile, and writes whole sectors, where 32 lanes storing 16 bytes of 32
+// different rows would each leave a partial one.  Without a tensor map (the
+// INT8-output epilogue, or no map) every thread stores its own row directly.
+struct EpiStore {
+    const CUtensorMap* tmY;   // null: direct stores
+    uint8_t* stage;           // this warp's 2 x 2048 bytes (1024-aligned)
+    int row0;                 // first output row of this warp's 32
+    uint32_t* sbuf;           // which of the two buffers is next
+    const float* colc;        // this tile's weight scales, zero points, bias: 3 x BN (shared)
+    float sx;                 // this thread's row: token scale
+    int32_t rs;               //                    and row sum
+};
+
+// The column and row constants of a tile, fetched into registers a tile
+// ahead: every lane holds BN / 32 columns of each constant.  The epilogue of
+// the current tile then reads them from warp-private shared memory (one
+// broadcast load per four columns) instead of waiting on global loads.
+template <int BN>
+struct EpiConsts {
+    float c[3][BN / 32];
+    float sx;
+    int32_t rs;
+
+    __device__ __forceinline__ void fetch(const EpiParams& p, int n_tile, int row) {
+        const int lane = threadIdx.x % 32;
+#pragma unroll
+        for (int i = 0; i < BN / 32; ++i) {
+            const int col = n_tile + i * 32 + lane;
+            const bool ok = col < p.n;
+            c[0][i] = ok ? p.sw[col] : 0.f;
+            c[1][i] = (ok && p.zw) ? p.zw[col] : 0.f;
+            c[2][i] = (ok && p.bias) ? p.bias[col] : 0.f;
+        }
+        const bool rok = row < p.m;
+        sx = rok ? p.sx[row] : 0.f;
+        rs = (rok && p.zw && p.rowsum) ? p.rowsum[row] : 0;
+    }
+
+    // Publishes the column constants to the warp's shared array (3 x BN).
+    __device__ __forceinline__ void publish(float* colc) const {
+        const int lane = threadIdx.x % 32;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < BN / 32; ++i) {
+            colc[i * 32 + lane] = c[0][i];
+            colc[BN + i * 32 + lane] = c[1][i];
+            colc[2 * BN + i * 32 + lane] = c[2][i];
+        }
+        __syncwarp();
+    }
+};
+
+
+__device__ __forceinline__ void st_shared_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_addr(p)), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
 }
 
 // Dequant epilogue of one accumulator tile for the calling thread's output
@@ -189,32 +256,45 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // warp-wide); rows and columns past the output are computed and not stored.
 template <int BN, int KIND, bool MIXED, bool QOUT>
 __device__ __forceinline__ void epilogue_tile(const EpiParams& p, uint32_t tb, int row, int n_tile,
-                                              int n16_kb) {
+                                              int n16_kb, const EpiStore& es) {
+    const int lane = threadIdx.x % 32;
     const bool has_zp = p.zw != nullptr;
     const bool row_ok = row < p.m;
-    const float sx = row_ok ? p.sx[row] : 0.f;
-    const int32_t rs = (row_ok && has_zp) ? p.rowsum[row] : 0;
+    const float sx = es.sx;
+    const int32_t rs = es.rs;
+    const bool tma = !QOUT && es.tmY != nullptr && es.row0 < p.m;
+    // Accumulator columns are read from TMEM G chunks of 32 at a time.
+    constexpr int NCH = BN / 32;
+    constexpr int G = 1;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c0 = 0; c0 < NCH; c0 += G) {
         __syncwarp();
-        uint32_t r[32];
-        tmem_ld32(tb + c * 32, r);
+        uint32_t rg[G][32];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            if (c0 + g < NCH) tmem_ld32(tb + (c0 + g) * 32, rg[g]);
         uint32_t r16[32];
         if constexpr (MIXED) {
-            if (n16_kb > 0) tmem_ld32(tb + BN + c * 32, r16);
+            if (n16_kb > 0) tmem_ld32(tb + BN + c0 * 32, r16);
         }
         tmem_ld_wait();
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        const int c = c0 + g;
+        if (c >= NCH) break;
+        const uint32_t (&r)[32] = rg[g];
         const int n0 = n_tile + c * 32;
-        if (row_ok && n0 < p.n) {
+        if (n0 >= p.n) continue;                               // uniform over the warp
         const int nv = (p.n - n0) >= 32 ? 32 : (p.n - n0);   // 16 or 32
         float out[32];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             if (4 * j >= nv) break;
-            const float4 sw4 = *reinterpret_cast<const float4*>(p.sw + n0 + 4 * j);
+            const float* cc = es.colc + c * 32 + 4 * j;
+            const float4 sw4 = *reinterpret_cast<const float4*>(cc);
             float4 zw4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = zw4;
-            if (has_zp) zw4 = *reinterpret_cast<const float4*>(p.zw + n0 + 4 * j);
-            if (p.bias) b4 = *reinterpret_cast<const float4*>(p.bias + n0 + 4 * j);
+            if (has_zp) zw4 = *reinterpret_cast<const float4*>(cc + BN);
+            if (p.bias) b4 = *reinterpret_cast<const float4*>(cc + 2 * BN);
             const float swv[4] = {sw4.x, sw4.y, sw4.z, sw4.w};
             const float zwv[4] = {zw4.x, zw4.y, zw4.z, zw4.w};
             const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
@@ -235,33 +315,56 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, uint32_t tb, i
                 out[i] = v;
             }
         }
-        if constexpr (QOUT) {
-            const Requant rq = requant_consts(p.out_scale);
-            uint32_t w[8], diff = 0u;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) w[j] = requant_codes4(&out[4 * j], rq, diff, 4 * j);
-            if (diff != 0u) {   // rare: outputs near a rounding boundary
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if ((diff >> i) & 1u)
-                        w[i / 4] = (w[i / 4] & ~(0xFFu << (8 * (i % 4)))) |
-                                   (requant_code_slow(out[i], rq.S) << (8 * (i % 4)));
-            }
-            uint4* qp = reinterpret_cast<uint4*>(p.yq + static_cast<int64_t>(row) * p.ldy + n0);
-            qp[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            if (nv > 16) qp[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        } else {
-            uint4* yp = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(row) * p.ldy + n0);
+        if (tma) {
+            uint8_t* buf = es.stage + *es.sbuf * 2048;
+            if (lane == 0) bulk_wait_read<1>();   // the buffer's previous store has read it
+            __syncwarp();
+            const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                if (8 * j >= nv) break;
-                yp[j] = make_uint4(pack_bf16(out[8 * j], out[8 * j + 1]),
-                                   pack_bf16(out[8 * j + 2], out[8 * j + 3]),
-                                   pack_bf16(out[8 * j + 4], out[8 * j + 5]),
-                                   pack_bf16(out[8 * j + 6], out[8 * j + 7]));
+                if (8 * j < nv)
+                    st_shared_v4(buf + lane * 64 + ((static_cast<uint32_t>(j) ^ sw) << 4),
+                                 pack_bf16(out[8 * j], out[8 * j + 1]),
+                                 pack_bf16(out[8 * j + 2], out[8 * j + 3]),
+                                 pack_bf16(out[8 * j + 4], out[8 * j + 5]),
+                                 pack_bf16(out[8 * j + 6], out[8 * j + 7]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(es.tmY, buf, n0, es.row0);
+                bulk_commit();
+            }
+            *es.sbuf ^= 1u;
+        } else if (row_ok) {
+            if constexpr (QOUT) {
+                const Requant rq = requant_consts(p.out_scale);
+                uint32_t w[8], diff = 0u;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[j] = requant_codes4(&out[4 * j], rq, diff, 4 * j);
+                if (diff != 0u) {   // rare: outputs near a rounding boundary
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if ((diff >> i) & 1u)
+                            w[i / 4] = (w[i / 4] & ~(0xFFu << (8 * (i % 4)))) |
+                                       (requant_code_slow(out[i], rq.S) << (8 * (i % 4)));
+                }
+                uint4* qp = reinterpret_cast<uint4*>(p.yq + static_cast<int64_t>(row) * p.ldy + n0);
+                qp[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                if (nv > 16) qp[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            } else {
+                uint4* yp = reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(row) * p.ldy + n0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (8 * j >= nv) break;
+                    yp[j] = make_uint4(pack_bf16(out[8 * j], out[8 * j + 1]),
+                                       pack_bf16(out[8 * j + 2], out[8 * j + 3]),
+                                       pack_bf16(out[8 * j + 4], out[8 * j + 5]),
+                                       pack_bf16(out[8 * j + 6], out[8 * j + 7]));
+                }
             }
         }
-        if (p.acc_debug) {
+        if (row_ok && p.acc_debug) {
             uint4* ap = reinterpret_cast<uint4*>(static_cast<uint32_t*>(p.acc_debug) +
                                                  static_cast<int64_t>(row) * p.n + n0);
 #pragma unroll
@@ -271,7 +374,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, uint32_t tb, i
             }
         }
         if constexpr (MIXED) {
-            if (p.y16_debug) {
+            if (row_ok && p.y16_debug) {
                 uint4* dp = reinterpret_cast<uint4*>(p.y16_debug + static_cast<int64_t>(row) * p.n + n0);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -283,7 +386,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, uint32_t tb, i
                 }
             }
         }
-        }  // row_ok && n0 < p.n
+    }
     }
 }
 
@@ -294,8 +397,8 @@ template <int BN, int KIND, bool MIXED, bool QOUT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmA16,
-                 const __grid_constant__ CUtensorMap tmB16, const EpiParams p, int num_kb,
-                 int tiles_m, int tiles_n) {
+                 const __grid_constant__ CUtensorMap tmB16, const __grid_constant__ CUtensorMap tmY,
+                 int use_tmy, const EpiParams p, int num_kb, int tiles_m, int tiles_n) {
     using C = TileCfg<BN, MIXED>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -453,6 +556,15 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         // ------------------------------------------------ epilogue
         pdl_wait();   // scales and row sums may come from the previous kernel
         const int q = warp & 3;  // this warp's TMEM lane quarter
+        uint32_t sbuf = 0;
+        uint8_t* epi_smem = smem + C::STAGES * C::STAGE;
+        float* colc = reinterpret_cast<float*>(epi_smem + kEpiStageBytes) + (warp - 2) * 3 * BN;
+        EpiStore es{use_tmy ? &tmY : nullptr, epi_smem + (warp - 2) * 4096, 0, &sbuf, colc, 0.f, 0};
+        EpiConsts<BN> pf;
+        if (static_cast<int>(blockIdx.x) < num_tiles) {
+            const int t0 = static_cast<int>(blockIdx.x);
+            pf.fetch(p, (t0 / tiles_m) * BN, (t0 % tiles_m) * kBM + q * 32 + lane);
+        }
         int buf = 0;
         uint32_t bphase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -460,13 +572,20 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (!mbar_wait(&tfull_bar[buf], bphase, &abort_sh, p.status)) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::BUF_COLS;
-            epilogue_tile<BN, KIND, MIXED, QOUT>(p, tb, tm * kBM + q * 32 + lane, tn * BN, n16_kb);
+            es.row0 = tm * kBM + q * 32;
+            pf.publish(colc);
+            es.sx = pf.sx;
+            es.rs = pf.rs;
+            const int nt = tile + static_cast<int>(gridDim.x);
+            if (nt < num_tiles) pf.fetch(p, (nt / tiles_m) * BN, (nt % tiles_m) * kBM + q * 32 + lane);
+            epilogue_tile<BN, KIND, MIXED, QOUT>(p, tb, es.row0 + lane, tn * BN, n16_kb, es);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[buf]);
             buf ^= 1;
             if (buf == 0) bphase ^= 1;
         }
+        if (lane == 0) bulk_wait_all();   // staged output stores done before the CTA ends
         __syncwarp();
     }
 
@@ -503,7 +622,7 @@ struct PairCfg {
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
     static constexpr int BUF_COLS = BN;
     static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
-    static constexpr int SMEM = STAGES * STAGE + 1024;
+    static constexpr int SMEM = STAGES * STAGE + kEpiStageBytes + kEpiConstBytes + 1024;
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "BN");
     static_assert((BN / 2) % 8 == 0, "weight half-tile rows: whole 8-row swizzle atoms");
 };
@@ -511,7 +630,8 @@ struct PairCfg {
 template <int BN, int KIND, bool QOUT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const EpiParams p, int num_kb, int tiles_m, int tiles_n) {
+                 const __grid_constant__ CUtensorMap tmY, int use_tmy, const EpiParams p, int num_kb,
+                 int tiles_m, int tiles_n) {
     using C = PairCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -642,6 +762,13 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         pdl_wait();
         const int q = warp & 3;
         const uint32_t tempty0 = map_shared_rank(smem_addr(&tempty_bar[0]), 0);
+        uint32_t sbuf = 0;
+        uint8_t* epi_smem = smem + C::STAGES * C::STAGE;
+        float* colc = reinterpret_cast<float*>(epi_smem + kEpiStageBytes) + (warp - 2) * 3 * BN;
+        EpiStore es{use_tmy ? &tmY : nullptr, epi_smem + (warp - 2) * 4096, 0, &sbuf, colc, 0.f, 0};
+        const int rbase = static_cast<int>(rank) * kBM + q * 32 + lane;   // this thread's row in a tile
+        EpiConsts<BN> pf;
+        if (pair < num_tiles) pf.fetch(p, (pair / tiles_m) * BN, (pair % tiles_m) * (2 * kBM) + rbase);
         int buf = 0;
         uint32_t bphase = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs) {
@@ -649,14 +776,20 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (!mbar_wait(&tfull_bar[buf], bphase, &abort_sh, p.status)) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::BUF_COLS;
-            const int row = tm * (2 * kBM) + static_cast<int>(rank) * kBM + q * 32 + lane;
-            epilogue_tile<BN, KIND, false, QOUT>(p, tb, row, tn * BN, 0);
+            es.row0 = tm * (2 * kBM) + static_cast<int>(rank) * kBM + q * 32;
+            pf.publish(colc);
+            es.sx = pf.sx;
+            es.rs = pf.rs;
+            const int nt = tile + npairs;
+            if (nt < num_tiles) pf.fetch(p, (nt / tiles_m) * BN, (nt % tiles_m) * (2 * kBM) + rbase);
+            epilogue_tile<BN, KIND, false, QOUT>(p, tb, es.row0 + lane, tn * BN, 0, es);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(buf));
             buf ^= 1;
             if (buf == 0) bphase ^= 1;
         }
+        if (lane == 0) bulk_wait_all();   // staged output stores done before the CTA ends
         __syncwarp();
     }
 
@@ -946,6 +1079,20 @@ bool make_map(CUtensorMap* m, const void* base, bool fp16, uint64_t inner, uint6
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map of the bf16 output for the epilogue's staged stores: boxes of
+// 32 columns x 32 rows with the 64-byte swizzle of the staging buffers.
+bool make_map_y(CUtensorMap* m, const void* y, uint64_t n, uint64_t rows, uint64_t ldy_elems) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {n, rows};
+    const cuuint64_t strides[1] = {ldy_elems * 2};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(y), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -972,6 +1119,8 @@ q8_status run_tile(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
         tA16 = tA;
         tB16 = tB;
     }
+    CUtensorMap tY = tA;
+    const int use_tmy = (!QOUT && a.y != nullptr && make_map_y(&tY, a.y, a.n, a.m, a.ldy)) ? 1 : 0;
     auto kern = gemm_tile_kernel<BN, KIND, MIXED, QOUT>;
     if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
     const int tiles_m = static_cast<int>((a.m + kBM - 1) / kBM);
@@ -989,7 +1138,8 @@ q8_status run_tile(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tA16, tB16, ep, num_kb, tiles_m, tiles_n) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tA16, tB16, tY, use_tmy, ep, num_kb, tiles_m, tiles_n) !=
+        cudaSuccess) {
         cudaGetLastError();
         return Q8_ERR_LAUNCH;
     }
@@ -1031,6 +1181,8 @@ q8_status run_pair(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     if (!make_map(&tA, a.a_codes, false, a.k, a.m, a.lda, kBKB, kBM) ||
         !make_map(&tB, a.b_codes, false, a.k, a.n, a.ldb, kBKB, BN / 2))
         return Q8_ERR_CUDA;
+    CUtensorMap tY = tA;
+    const int use_tmy = (!QOUT && a.y != nullptr && make_map_y(&tY, a.y, a.n, a.m, a.ldy)) ? 1 : 0;
     auto kern = gemm_pair_kernel<BN, KIND, QOUT>;
     if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
     const int tiles_m = static_cast<int>((a.m + 2 * kBM - 1) / (2 * kBM));
@@ -1053,7 +1205,7 @@ q8_status run_pair(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, ep, num_kb, tiles_m, tiles_n) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tY, use_tmy, ep, num_kb, tiles_m, tiles_n) != cudaSuccess) {
         cudaGetLastError();
         return Q8_ERR_LAUNCH;
     }

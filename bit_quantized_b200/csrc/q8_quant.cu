@@ -42,8 +42,6 @@ using qm::kFastLimit;
 using qm::kMagic;
 constexpr int kBlock = 256;
 constexpr int kMaxVec = 16;   // 16-byte vectors a thread keeps in registers
-constexpr int kRingMaxStages = 24;        // ring barriers per block (all groups)
-constexpr int kRingBytes = 192 * 1024;    // ring per block (one block per SM)
 
 template <typename T> struct VecOf;
 template <> struct VecOf<__half> { static constexpr int N = 8; };
@@ -99,26 +97,6 @@ __device__ __forceinline__ void group_sync() {
         __syncthreads();
     } else {
         asm volatile("bar.sync %0, %1;" ::"r"(1 + static_cast<int>(threadIdx.x) / TPR), "n"(TPR) : "memory");
-    }
-}
-
-// True when `v` holds on every thread of the TPR-thread row group (a
-// barrier of the group).
-template <int TPR>
-__device__ __forceinline__ bool group_all(bool v) {
-    if constexpr (TPR == 32) {
-        return __all_sync(0xffffffffu, v);
-    } else if constexpr (TPR >= kBlock) {
-        return __syncthreads_and(v) != 0;
-    } else {
-        uint32_t r;
-        asm volatile(
-            "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
-            "bar.red.and.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(r)
-            : "r"(static_cast<uint32_t>(v)), "r"(1 + static_cast<int>(threadIdx.x) / TPR), "n"(TPR)
-            : "memory");
-        return r != 0;
     }
 }
 
@@ -552,19 +530,14 @@ __device__ __forceinline__ void for_each_outlier(const OutlierRuns& r, F&& f) {
 // them stay in registers between the two passes (longer rows are read twice,
 // the second time from L2).
 //
-// RING: each group of TPR (32 or 64) threads streams its rows into its own
-// ring of `nstages` shared-memory stages with 1-D bulk copies, issued by the
-// group's first thread as soon as a stage's row has been read into
-// registers.  A group codes one row while the next ones are in flight, and
-// no barrier spans more than the group, so the SM keeps 8 groups' rows of
-// HBM reads outstanding through their reductions and code passes (a
-// persistent grid, one block per SM).  Without RING each thread loads its
-// vectors straight from global memory.
-template <typename T, int OP, int TPR, int MAXV, bool RING = false>
-__global__ void __launch_bounds__(kBlock, RING ? 1 : (MAXV <= 4 ? 4 : 2))
-row_quant_kernel(RowQuantArgs a, int nstages, int64_t stage_bytes, int* status) {
+// PF (multi-wave matrices whose rows fit the register cache): the block
+// walks its rows with a stride of the grid, and every thread issues the loads
+// of its next row's vectors before it reduces and codes the current one, so
+// HBM reads stay in flight through the reductions and the code pass.
+template <typename T, int OP, int TPR, int MAXV, bool PF = false>
+__global__ void __launch_bounds__(kBlock, PF ? (MAXV <= 4 ? 3 : 2) : (MAXV <= 4 ? 4 : 2))
+row_quant_kernel(RowQuantArgs a) {
     static_assert(TPR % 32 == 0, "a warp works on one row");
-    static_assert(!RING || TPR == 32 || TPR == 64, "ring groups are one or two warps");
     constexpr int V = VecOf<T>::N;
     constexpr int RPB = kBlock / TPR;
     constexpr bool kSkip = OP == kOpActInt8Skip;
@@ -575,27 +548,10 @@ row_quant_kernel(RowQuantArgs a, int nstages, int64_t stage_bytes, int* status) 
     __shared__ int redi[kBlock / 32];
     __shared__ FixQueue fixq[kBlock / 32];
     __shared__ float cshare[kBlock / TPR][8];
-    extern __shared__ __align__(128) uint8_t ring[];   // RING: RPB groups x nstages x stage_bytes
-    __shared__ __align__(8) uint64_t ring_full[RING ? kRingMaxStages : 1];
-    __shared__ int ring_abort[RING ? kBlock / TPR : 1];
     FixQueue* q = &fixq[threadIdx.x / 32];
-    const uint32_t row_bytes = static_cast<uint32_t>(a.k * static_cast<int64_t>(sizeof(T)));
-    if constexpr (RING) {
-        if (threadIdx.x == 0) {
-            for (int i = 0; i < RPB * nstages; ++i) mbar_init(&ring_full[i], 1);
-            for (int i = 0; i < RPB; ++i) ring_abort[i] = 0;
-            fence_barrier_init();
-        }
-        __syncthreads();
-    }
 
     const int g = threadIdx.x / TPR;
     const int t = threadIdx.x % TPR;
-    // RING: this group's stages and barriers; its rows are gid, gid + G, ...
-    uint8_t* gring = ring + static_cast<int64_t>(g) * nstages * stage_bytes;
-    uint64_t* gfull = &ring_full[RING ? g * nstages : 0];
-    const int64_t gid = static_cast<int64_t>(blockIdx.x) * RPB + g;
-    const int64_t G = static_cast<int64_t>(gridDim.x) * RPB;
     const int64_t nvec = a.k / V;
     const bool cached = nvec <= static_cast<int64_t>(TPR) * MAXV;
     // Vectors this thread holds when the row is cached, and the most any
@@ -613,19 +569,17 @@ row_quant_kernel(RowQuantArgs a, int nstages, int64_t stage_bytes, int* status) 
                   OP == kOpActInt8Smooth)
         pdl_launch_dependents();
     pdl_wait();
-    // RING: the group's row of iteration i (gid + i G) goes to its stage i % nstages.
-    auto ring_issue = [&](int64_t it) {
-        const int64_t r = gid + it * G;
-        if (r < a.rows) {
-            const int st = static_cast<int>(it % nstages);
-            mbar_arrive_expect_tx(&gfull[st], row_bytes);
-            bulk_load(gring + st * stage_bytes, static_cast<const T*>(a.src) + r * a.ld, row_bytes,
-                      &gfull[st]);
-        }
+    // PF: this thread's vectors of its group's next row (all rows are cached).
+    uint4 nxt[PF ? MAXV : 1] = {};
+    auto load_row = [&](int64_t r) {
+        const T* p = static_cast<const T*>(a.src) + r * a.ld + static_cast<int64_t>(t) * V;
+#pragma unroll
+        for (int i = 0; i < MAXV; ++i)
+            nxt[i] = i < nvl ? ld_stream16(p + i * TPR * V) : make_uint4(0u, 0u, 0u, 0u);
     };
-    if constexpr (RING) {
-        if (t == 0)
-            for (int i = 0; i < nstages; ++i) ring_issue(i);
+    if constexpr (PF) {
+        const int64_t r = static_cast<int64_t>(blockIdx.x) * RPB + g;
+        if (r < a.rows) load_row(r);
     }
 
     // LLM.int8: rank the outlier columns; block 0 publishes the ascending
@@ -641,9 +595,8 @@ row_quant_kernel(RowQuantArgs a, int nstages, int64_t stage_bytes, int* status) 
         }
     }
 
-    int64_t it = 0;
     for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * RPB; row0 < a.rows;
-         row0 += static_cast<int64_t>(gridDim.x) * RPB, ++it) {
+         row0 += static_cast<int64_t>(gridDim.x) * RPB) {
         const int64_t row = row0 + g;
         const bool active = row < a.rows;   // the same for a whole warp
         const T* src_row = static_cast<const T*>(a.src) + (active ? row : 0) * a.ld;
@@ -669,34 +622,19 @@ row_quant_kernel(RowQuantArgs a, int nstages, int64_t stage_bytes, int* status) 
         // rows only count loaded vectors.  Left-out columns are zeroed.
         uint4 raw[MAXV];
         RowStats st{0.f, FLT_MAX, -FLT_MAX};
-        const uint8_t* srow = RING ? gring + (it % nstages) * stage_bytes : nullptr;
-        if constexpr (RING) {
-            // Every thread of the group waits for the row's bytes; the group
-            // decides together (a wait that ran out stops the group before any
-            // barrier of the row's reduction).
-            if (active) {   // uniform per group
-                const bool ok = mbar_wait(&gfull[it % nstages], static_cast<uint32_t>((it / nstages) & 1),
-                                          &ring_abort[g], status);
-                if (!group_all<TPR>(ok)) {
-                    if (t == 0) {
-                        // Let the copies still in flight land before the block exits.
-                        for (int64_t j = it; j < it + nstages; ++j)
-                            if (gid + j * G < a.rows)
-                                mbar_wait(&gfull[j % nstages], static_cast<uint32_t>((j / nstages) & 1),
-                                          nullptr, nullptr);
-                    }
-                    break;
-                }
-            }
+        if constexpr (PF) {
+            // This row's vectors were loaded during the previous row; the next
+            // row's loads go out now.
+#pragma unroll
+            for (int i = 0; i < MAXV; ++i) raw[i] = nxt[i];
+            const int64_t rn = row + static_cast<int64_t>(gridDim.x) * RPB;
+            if (rn < a.rows) load_row(rn);
         }
         auto pass1 = [&](auto full_tag) {
             constexpr bool FULL = decltype(full_tag)::value;
+            if constexpr (!PF) {
 #pragma unroll
-            for (int i = 0; i < MAXV; ++i) {
-                if constexpr (RING)
-                    raw[i] = (FULL || i < nv) ? ld_shared16(srow + (static_cast<int64_t>(t) + i * TPR) * 16)
-                                              : make_uint4(0u, 0u, 0u, 0u);
-                else
+                for (int i = 0; i < MAXV; ++i)
                     raw[i] = (FULL || i < nv) ? ld_stream16(src + i * TPR * V) : make_uint4(0u, 0u, 0u, 0u);
             }
 #pragma unroll
@@ -736,15 +674,6 @@ row_quant_kernel(RowQuantArgs a, int nstages, int64_t stage_bytes, int* status) 
         }
         st.amax = fmaxf(st.hi, -st.lo);
         st = group_reduce<TPR, OP == kOpWeightAsym>(st, red);
-        if constexpr (RING) {
-            // Every thread of the group has read its vectors of this stage
-            // (they fed the reduction): it can take the row nstages further on.
-            __syncwarp();
-            if (t == 0) {
-                fence_proxy_async_smem();
-                ring_issue(it + nstages);
-            }
-        }
         if constexpr (OP != kOpWeightAsym) st.amax = fmaxf(st.amax, 0.0f);
 
         RowConsts c;
@@ -903,13 +832,20 @@ template <typename T, int OP>
 cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
     constexpr int V = VecOf<T>::N;
     const int64_t nvec = a.k / V;
-    int* status = device_status_ptr();
-    auto go = [&](auto tpr_tag, auto maxv_tag) -> cudaError_t {
+    // PF launches a grid of at most 3 blocks per SM that strides over the rows.
+    auto go = [&](auto tpr_tag, auto maxv_tag, auto pf_tag) -> cudaError_t {
         constexpr int TPR = decltype(tpr_tag)::value;
         constexpr int MAXV = decltype(maxv_tag)::value;
+        constexpr bool PF = decltype(pf_tag)::value;
         constexpr int RPB = kBlock / TPR;
         int64_t blocks = (a.rows + RPB - 1) / RPB;
         if (blocks > 65535 * 4) blocks = 65535 * 4;
+        if (PF) {
+            int sms = 148, dev = 0;
+            if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            const int per_sm = MAXV <= 4 ? 3 : 2;
+            if (blocks > per_sm * sms) blocks = per_sm * sms;
+        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
         cfg.blockDim = dim3(kBlock, 1, 1);
@@ -920,55 +856,8 @@ cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, row_quant_kernel<T, OP, TPR, MAXV>, a, 0, int64_t(0), status);
+        return cudaLaunchKernelEx(&cfg, row_quant_kernel<T, OP, TPR, MAXV, PF>, a);
     };
-    // Ring configuration (large matrices): one persistent block per SM whose
-    // row groups of 32 or 64 threads stream their rows through at least two
-    // stages each, when a row fits the group's registers (16 vectors a thread).
-    auto go_ring = [&](auto tpr_tag, auto maxv_tag) -> cudaError_t {
-        constexpr int TPR = decltype(tpr_tag)::value;
-        constexpr int MAXV = decltype(maxv_tag)::value;
-        constexpr int RPB = kBlock / TPR;
-        const int64_t row_bytes = a.k * static_cast<int64_t>(sizeof(T));
-        const int64_t stage_bytes = (row_bytes + 127) / 128 * 128;
-        int nstages = static_cast<int>(kRingBytes / (RPB * stage_bytes));
-        if (nstages > kRingMaxStages / RPB) nstages = kRingMaxStages / RPB;
-        int sms = 148, dev = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        int64_t blocks = (a.rows + RPB - 1) / RPB;
-        if (blocks > sms) blocks = sms;
-        auto kern = row_quant_kernel<T, OP, TPR, MAXV, true>;
-        const int dyn = static_cast<int>(RPB * nstages * stage_bytes);
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-        if (e != cudaSuccess) return e;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(blocks), 1, 1);
-        cfg.blockDim = dim3(kBlock, 1, 1);
-        cfg.dynamicSmemBytes = static_cast<size_t>(dyn);
-        cfg.stream = s;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, kern, a, nstages, stage_bytes, status);
-    };
-    {
-        const int64_t row_bytes = a.k * static_cast<int64_t>(sizeof(T));
-        const int64_t stage_bytes = (row_bytes + 127) / 128 * 128;
-        const bool aligned = (a.ld * static_cast<int64_t>(sizeof(T))) % 16 == 0 &&
-                             (reinterpret_cast<uintptr_t>(a.src) & 15u) == 0;
-        if (aligned && a.rows >= 4 * 148) {
-            using W1 = std::integral_constant<int, 32>;
-            using W2 = std::integral_constant<int, 64>;
-            if (nvec <= 32 * 4) return go_ring(W1{}, std::integral_constant<int, 4>{});
-            if (nvec <= 32 * 8) return go_ring(W1{}, std::integral_constant<int, 8>{});
-            if (nvec <= 32 * 16 && 2 * 8 * stage_bytes <= kRingBytes)
-                return go_ring(W1{}, std::integral_constant<int, 16>{});
-            if (nvec <= 64 * 16 && 2 * 4 * stage_bytes <= kRingBytes)
-                return go_ring(W2{}, std::integral_constant<int, 16>{});
-        }
-    }
     using T128 = std::integral_constant<int, 128>;
     using T256 = std::integral_constant<int, 256>;
     using C2 = std::integral_constant<int, 2>;
@@ -986,20 +875,27 @@ cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
     // thread instead (rows of up to 1024 vectors): fewer registers, twice the
     // resident warps, so loads of some rows overlap the arithmetic of others.
     const int64_t warps16 = a.rows * (tpr / 32);
-    if (warps16 > 2 * 148 * (kBlock / 32) && nvec <= 256 * 4) {
-        if (nvec <= 128 * 4) return go(T128{}, C4{});
-        return go(T256{}, C4{});
+    using Y = std::true_type;
+    using N = std::false_type;
+    // Multi-wave matrices: 8 vectors a thread (the per-row reductions and
+    // constants are shared by twice the work of 4), the next row prefetched.
+    if (warps16 > 2 * 148 * (kBlock / 32) && nvec <= 256 * 8) {
+        using C8 = std::integral_constant<int, 8>;
+        if (nvec <= 32 * 8) return go(std::integral_constant<int, 32>{}, C8{}, Y{});
+        if (nvec <= 64 * 8) return go(std::integral_constant<int, 64>{}, C8{}, Y{});
+        if (nvec <= 128 * 8) return go(T128{}, C8{}, Y{});
+        return go(T256{}, C8{}, Y{});
     }
     // Rows spread over 128 or 256 threads hold a few vectors each: a kernel
     // unrolled for just those keeps the code short, which matters when each
     // SM runs it once (small batches: the instructions are fetched cold).
-    if (tpr == 256 && nvec <= 256 * 2) return go(T256{}, C2{});
-    if (tpr >= 128 && nvec <= 128 * 4) return go(T128{}, C4{});
-    if (tpr == 256 && nvec <= 256 * 4) return go(T256{}, C4{});
-    if (tpr == 32) return go(std::integral_constant<int, 32>{}, C16{});
-    if (tpr == 64) return go(std::integral_constant<int, 64>{}, C16{});
-    if (tpr == 128) return go(T128{}, C16{});
-    return go(T256{}, C16{});
+    if (tpr == 256 && nvec <= 256 * 2) return go(T256{}, C2{}, N{});
+    if (tpr >= 128 && nvec <= 128 * 4) return go(T128{}, C4{}, N{});
+    if (tpr == 256 && nvec <= 256 * 4) return go(T256{}, C4{}, N{});
+    if (tpr == 32) return go(std::integral_constant<int, 32>{}, C16{}, N{});
+    if (tpr == 64) return go(std::integral_constant<int, 64>{}, C16{}, N{});
+    if (tpr == 128) return go(T128{}, C16{}, N{});
+    return go(T256{}, C16{}, N{});
 }
 
 template <typename T>
