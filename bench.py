@@ -259,8 +259,13 @@ def dominant_kernel(w, gemm_ms: float, region_ms: float, pk: dict, lib_peaks: di
     bf16 = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
     peak = bf16 * NOMINAL_INT8_OVER_BF16
     achieved = ops / t / 1e12
-    out = {"bound": "tensor",
-           "kernel": "gemm_tile_kernel" + (" (LLM.int8)" if w.kind == "int8_mixed" else ""),
+    if w.kind == "int8_mixed":
+        kernel = "gemm_tile_kernel (LLM.int8, int32 + fp32 accumulators)"
+    elif w.m > 256:
+        kernel = "gemm_pair_kernel (cta_group::2, 256-row tiles on SM pairs)"
+    else:
+        kernel = "gemm_tile_kernel (128-row tiles)"
+    out = {"bound": "tensor", "kernel": kernel,
            "achieved": round(achieved, 1), "peak": round(peak, 1), "unit": "TFLOP/s",
            "frac": round(achieved / peak, 4), "algorithmic_ops": ops,
            "peak_source": (f"{pk['source']} bf16 {'sustained' if sustained else 'burst'} {bf16} x 2 "

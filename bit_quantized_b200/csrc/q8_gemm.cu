@@ -50,9 +50,12 @@ namespace {
 constexpr int kBM = 128;        // MMA M (TMEM lanes)
 constexpr int kBKB = 128;       // bytes of K per pipeline stage (one 128-byte swizzle row)
 constexpr int kThreads = 192;
-constexpr int kSmemBudget = 200 * 1024;
 constexpr int kEpiStageBytes = 4 * 2 * 2048;   // output staging per CTA: 4 epilogue warps x 2 buffers
 constexpr int kEpiConstBytes = 4 * 3 * 256 * 4; // column constants per CTA: 4 warps x 3 x BN (<= 256) floats
+// Operand stages get what is left of the 227 KB a CTA may use once the
+// epilogue's buffers, the 1 KB alignment slack and up to 5 KB of static
+// shared memory (barriers, the grouped tile map) are set aside.
+constexpr int kSmemBudget = 227 * 1024 - kEpiStageBytes - kEpiConstBytes - 1024 - 5 * 1024;
 
 enum GemmKind { kS8S8 = 0, kS8U8 = 1, kE4M3 = 2 };
 
@@ -201,6 +204,8 @@ struct EpiStore {
     const float* colc;        // this tile's weight scales, zero points, bias: 3 x BN (shared)
     float sx;                 // this thread's row: token scale
     int32_t rs;               //                    and row sum
+    int row_end;              // rows >= row_end are not stored
+    bool tma_tile;            // this warp's 32 rows may go through the tensor store
 };
 
 // The column and row constants of a tile, fetched into registers a tile
@@ -213,17 +218,20 @@ struct EpiConsts {
     float sx;
     int32_t rs;
 
-    __device__ __forceinline__ void fetch(const EpiParams& p, int n_tile, int row) {
+    // Columns n_tile.. of the output (col_off + column in the scale and bias
+    // arrays), and this thread's row (stored only below row_end).
+    __device__ __forceinline__ void fetch(const EpiParams& p, int n_tile, int col_off, int row,
+                                          int row_end) {
         const int lane = threadIdx.x % 32;
 #pragma unroll
         for (int i = 0; i < BN / 32; ++i) {
             const int col = n_tile + i * 32 + lane;
             const bool ok = col < p.n;
-            c[0][i] = ok ? p.sw[col] : 0.f;
-            c[1][i] = (ok && p.zw) ? p.zw[col] : 0.f;
-            c[2][i] = (ok && p.bias) ? p.bias[col] : 0.f;
+            c[0][i] = ok ? p.sw[col_off + col] : 0.f;
+            c[1][i] = (ok && p.zw) ? p.zw[col_off + col] : 0.f;
+            c[2][i] = (ok && p.bias) ? p.bias[col_off + col] : 0.f;
         }
-        const bool rok = row < p.m;
+        const bool rok = row < row_end;
         sx = rok ? p.sx[row] : 0.f;
         rs = (rok && p.zw && p.rowsum) ? p.rowsum[row] : 0;
     }
@@ -259,10 +267,10 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, uint32_t tb, i
                                               int n16_kb, const EpiStore& es) {
     const int lane = threadIdx.x % 32;
     const bool has_zp = p.zw != nullptr;
-    const bool row_ok = row < p.m;
+    const bool row_ok = row < es.row_end;
     const float sx = es.sx;
     const int32_t rs = es.rs;
-    const bool tma = !QOUT && es.tmY != nullptr && es.row0 < p.m;
+    const bool tma = !QOUT && es.tmY != nullptr && es.tma_tile;
     // Accumulator columns are read from TMEM G chunks of 32 at a time.
     constexpr int NCH = BN / 32;
     constexpr int G = 1;
@@ -390,16 +398,91 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, uint32_t tb, i
     }
 }
 
+// Where one output tile of a persistent schedule lies.
+struct TileRef {
+    int a_row;     // first activation row the tile reads
+    int row_end;   // rows at or past row_end are computed and not stored
+    int b_row;     // first weight row
+    int n_tile;    // first output column
+    int col_off;   // offset of the output columns in the scale and bias arrays
+};
+
+// Dense schedule: tiles_m x tiles_n tiles, the M index fastest.
+__device__ __forceinline__ TileRef dense_tile(int tile, int tiles_m, int rows, int bn, int m) {
+    const int tm = tile % tiles_m, tn = tile / tiles_m;
+    return TileRef{tm * rows, m, tn * bn, tn * bn, 0};
+}
+
+// Grouped schedule of a mixture-of-experts layer (the grouped FP8 linear of
+// the FBGEMM FP8 page, section 5.4): tokens sorted by expert, rows
+// off[e] .. off[e+1]-1 meet expert e's weight rows e*n .. e*n+n-1.  Expert e
+// has ceil((off[e+1] - off[e]) / rows) row tiles; mt[e] counts those of the
+// experts before it, so the layer has mt[E] x tiles_n tiles, the row-tile index
+// fastest.  A tile starts at any token row (TMA has no alignment rule for the
+// outer coordinate); rows past the expert's end are computed and not stored.
+constexpr int kMaxGroupedExperts = 512;
+
+__device__ __forceinline__ TileRef grouped_tile(int tile, const int* off, const int* mt, int experts,
+                                                int rows, int bn, int n) {
+    const int G = mt[experts];
+    const int g = tile % G, tn = tile / G;
+    // the expert e with mt[e] <= g < mt[e + 1] (empty experts have none)
+    int lo = 0, hi = experts;   // mt[lo] <= g < mt[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (mt[mid] <= g) lo = mid; else hi = mid;
+    }
+    return TileRef{off[lo] + (g - mt[lo]) * rows, off[lo + 1], lo * n + tn * bn, tn * bn, lo * n};
+}
+
+// off[0..E]: the offsets clamped to [0, m] and made non-decreasing; mt[0..E]:
+// the row-tile prefix.  One warp, 32 experts at a time.
+__device__ __forceinline__ void build_group_map(const int32_t* offsets, int experts, int m, int rows,
+                                                int* off, int* mt) {
+    const int lane = threadIdx.x % 32;
+    int carry_off = 0, carry_mt = 0;
+    for (int base = 0; base <= experts; base += 32) {
+        const int e = base + lane;
+        int v = e <= experts ? offsets[e] : m;
+        v = v < 0 ? 0 : (v > m ? m : v);
+        v = v > carry_off ? v : carry_off;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {   // running maximum
+            const int y = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v = v > y ? v : y;
+        }
+        // expert e - 1 spans [off[e - 1], off[e]): its row tiles, counted at index e
+        const int prev = __shfl_up_sync(0xffffffffu, v, 1);
+        const int lo_e = lane == 0 ? carry_off : prev;
+        int t = (e >= 1 && e <= experts) ? (v - lo_e + rows - 1) / rows : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {   // inclusive sum
+            const int y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        if (e <= experts) {
+            off[e] = v;
+            mt[e] = carry_mt + t;
+        }
+        carry_off = __shfl_sync(0xffffffffu, v, 31);
+        carry_mt += __shfl_sync(0xffffffffu, t, 31);
+    }
+}
+
 // ============================================================================
 // Persistent tile kernel
 // ============================================================================
-template <int BN, int KIND, bool MIXED, bool QOUT>
+template <int BN, int KIND, bool MIXED, bool QOUT, bool GROUPED = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmA16,
                  const __grid_constant__ CUtensorMap tmB16, const __grid_constant__ CUtensorMap tmY,
-                 int use_tmy, const EpiParams p, int num_kb, int tiles_m, int tiles_n) {
+                 int use_tmy, const EpiParams p, int num_kb, int tiles_m, int tiles_n,
+                 const int32_t* group_offsets, int experts) {
     using C = TileCfg<BN, MIXED>;
+    static_assert(!(GROUPED && MIXED), "grouped tiles carry no outlier stream");
+    __shared__ int g_off[GROUPED ? kMaxGroupedExperts + 1 : 1];
+    __shared__ int g_mt[GROUPED ? kMaxGroupedExperts + 1 : 1];
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     __shared__ __align__(8) uint64_t full_bar[C::STAGES];
@@ -430,6 +513,11 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
         tmem_relinquish();
     }
+    if constexpr (GROUPED) {
+        // The routing offsets come from the previous kernels.
+        pdl_wait();
+        if (warp == 2) build_group_map(group_offsets, experts, p.m, kBM, g_off, g_mt);
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -444,7 +532,11 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         n16_kb = (*p.outlier_count + 63) / 64;
     }
     const int total_kb = num_kb + n16_kb;
-    const int num_tiles = tiles_m * tiles_n;
+    const int num_tiles = GROUPED ? g_mt[GROUPED ? experts : 0] * tiles_n : tiles_m * tiles_n;
+    auto tile_ref = [&](int tile) -> TileRef {
+        if constexpr (GROUPED) return grouped_tile(tile, g_off, g_mt, experts, kBM, BN, p.n);
+        else return dense_tile(tile, tiles_m, kBM, BN, p.m);
+    };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -462,7 +554,7 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int tm = tile % tiles_m, tn = tile / tiles_m;
+                const TileRef tr = tile_ref(tile);
                 for (int kb = 0; kb < total_kb; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
                         ok = false;
@@ -472,12 +564,12 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     uint8_t* sb = sa + C::A_BYTES;
                     mbar_arrive_expect_tx(&full_bar[stage], C::STAGE);
                     if (!MIXED || kb < num_kb) {
-                        tma_load_2d(sa, &tmA, &full_bar[stage], kb * kBKB, tm * kBM);
-                        tma_load_2d(sb, &tmB, &full_bar[stage], kb * kBKB, tn * BN);
+                        tma_load_2d(sa, &tmA, &full_bar[stage], kb * kBKB, tr.a_row);
+                        tma_load_2d(sb, &tmB, &full_bar[stage], kb * kBKB, tr.b_row);
                     } else {
                         const int k16 = (kb - num_kb) * 64;
-                        tma_load_2d(sa, &tmA16, &full_bar[stage], k16, tm * kBM);
-                        tma_load_2d(sb, &tmB16, &full_bar[stage], k16, tn * BN);
+                        tma_load_2d(sa, &tmA16, &full_bar[stage], k16, tr.a_row);
+                        tma_load_2d(sb, &tmB16, &full_bar[stage], k16, tr.b_row);
                     }
                     issued |= 1u << stage;
                     last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -559,26 +651,34 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         uint32_t sbuf = 0;
         uint8_t* epi_smem = smem + C::STAGES * C::STAGE;
         float* colc = reinterpret_cast<float*>(epi_smem + kEpiStageBytes) + (warp - 2) * 3 * BN;
-        EpiStore es{use_tmy ? &tmY : nullptr, epi_smem + (warp - 2) * 4096, 0, &sbuf, colc, 0.f, 0};
+        EpiStore es{use_tmy ? &tmY : nullptr, epi_smem + (warp - 2) * 4096, 0, &sbuf, colc, 0.f, 0, 0,
+                    false};
         EpiConsts<BN> pf;
         if (static_cast<int>(blockIdx.x) < num_tiles) {
-            const int t0 = static_cast<int>(blockIdx.x);
-            pf.fetch(p, (t0 / tiles_m) * BN, (t0 % tiles_m) * kBM + q * 32 + lane);
+            const TileRef t0 = tile_ref(static_cast<int>(blockIdx.x));
+            pf.fetch(p, t0.n_tile, t0.col_off, t0.a_row + q * 32 + lane, t0.row_end);
         }
         int buf = 0;
         uint32_t bphase = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            const int tm = tile % tiles_m, tn = tile / tiles_m;
+            const TileRef tr = tile_ref(tile);
             if (!mbar_wait(&tfull_bar[buf], bphase, &abort_sh, p.status)) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::BUF_COLS;
-            es.row0 = tm * kBM + q * 32;
+            es.row0 = tr.a_row + q * 32;
+            es.row_end = tr.row_end;
+            // A tensor store clips at the output's last row only: chunks that
+            // cross an expert's end are stored row by row.
+            es.tma_tile = GROUPED ? es.row0 + 32 <= tr.row_end : es.row0 < tr.row_end;
             pf.publish(colc);
             es.sx = pf.sx;
             es.rs = pf.rs;
             const int nt = tile + static_cast<int>(gridDim.x);
-            if (nt < num_tiles) pf.fetch(p, (nt / tiles_m) * BN, (nt % tiles_m) * kBM + q * 32 + lane);
-            epilogue_tile<BN, KIND, MIXED, QOUT>(p, tb, es.row0 + lane, tn * BN, n16_kb, es);
+            if (nt < num_tiles) {
+                const TileRef tn = tile_ref(nt);
+                pf.fetch(p, tn.n_tile, tn.col_off, tn.a_row + q * 32 + lane, tn.row_end);
+            }
+            epilogue_tile<BN, KIND, MIXED, QOUT>(p, tb, es.row0 + lane, tr.n_tile, n16_kb, es);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[buf]);
@@ -627,12 +727,14 @@ struct PairCfg {
     static_assert((BN / 2) % 8 == 0, "weight half-tile rows: whole 8-row swizzle atoms");
 };
 
-template <int BN, int KIND, bool QOUT>
+template <int BN, int KIND, bool QOUT, bool GROUPED = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  const __grid_constant__ CUtensorMap tmY, int use_tmy, const EpiParams p, int num_kb,
-                 int tiles_m, int tiles_n) {
+                 int tiles_m, int tiles_n, const int32_t* group_offsets, int experts) {
     using C = PairCfg<BN>;
+    __shared__ int g_off[GROUPED ? kMaxGroupedExperts + 1 : 1];
+    __shared__ int g_mt[GROUPED ? kMaxGroupedExperts + 1 : 1];
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     __shared__ __align__(8) uint64_t full_bar[C::STAGES];
@@ -666,6 +768,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         tmem_alloc_pair(&tmem_base_sh, C::TMEM_COLS);
         tmem_relinquish_pair();
     }
+    if constexpr (GROUPED) {
+        // The routing offsets come from the previous kernels.
+        pdl_wait();
+        if (warp == 2) build_group_map(group_offsets, experts, p.m, 2 * kBM, g_off, g_mt);
+    }
     tc_fence_before();
     __syncthreads();
     // Both CTAs' barriers are initialized before either touches the other's.
@@ -674,7 +781,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     const uint32_t tmem_base = tmem_base_sh;
     pdl_launch_dependents();
 
-    const int num_tiles = tiles_m * tiles_n;
+    const int num_tiles = GROUPED ? g_mt[GROUPED ? experts : 0] * tiles_n : tiles_m * tiles_n;
+    // A pair tile is 256 activation rows (128 from each CTA) x BN columns.
+    auto tile_ref = [&](int tile) -> TileRef {
+        if constexpr (GROUPED) return grouped_tile(tile, g_off, g_mt, experts, 2 * kBM, BN, p.n);
+        else return dense_tile(tile, tiles_m, 2 * kBM, BN, p.m);
+    };
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
         if (elect_one()) {
@@ -686,7 +798,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
-                const int tm = tile % tiles_m, tn = tile / tiles_m;
+                const TileRef tr = tile_ref(tile);
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
                         ok = false;
@@ -696,8 +808,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     uint8_t* sb = sa + C::A_BYTES;
                     if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE);
                     const uint32_t fb = full0 + 8u * static_cast<uint32_t>(stage);
-                    tma_load_2d_pair(sa, &tmA, fb, kb * kBKB, tm * (2 * kBM) + static_cast<int>(rank) * kBM);
-                    tma_load_2d_pair(sb, &tmB, fb, kb * kBKB, tn * BN + static_cast<int>(rank) * (BN / 2));
+                    tma_load_2d_pair(sa, &tmA, fb, kb * kBKB, tr.a_row + static_cast<int>(rank) * kBM);
+                    tma_load_2d_pair(sb, &tmB, fb, kb * kBKB, tr.b_row + static_cast<int>(rank) * (BN / 2));
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -765,24 +877,35 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         uint32_t sbuf = 0;
         uint8_t* epi_smem = smem + C::STAGES * C::STAGE;
         float* colc = reinterpret_cast<float*>(epi_smem + kEpiStageBytes) + (warp - 2) * 3 * BN;
-        EpiStore es{use_tmy ? &tmY : nullptr, epi_smem + (warp - 2) * 4096, 0, &sbuf, colc, 0.f, 0};
+        EpiStore es{use_tmy ? &tmY : nullptr, epi_smem + (warp - 2) * 4096, 0, &sbuf, colc, 0.f, 0, p.m,
+                    false};
         const int rbase = static_cast<int>(rank) * kBM + q * 32 + lane;   // this thread's row in a tile
         EpiConsts<BN> pf;
-        if (pair < num_tiles) pf.fetch(p, (pair / tiles_m) * BN, (pair % tiles_m) * (2 * kBM) + rbase);
+        if (pair < num_tiles) {
+            const TileRef t0 = tile_ref(pair);
+            pf.fetch(p, t0.n_tile, t0.col_off, t0.a_row + rbase, t0.row_end);
+        }
         int buf = 0;
         uint32_t bphase = 0;
         for (int tile = pair; tile < num_tiles; tile += npairs) {
-            const int tm = tile % tiles_m, tn = tile / tiles_m;
+            const TileRef tr = tile_ref(tile);
             if (!mbar_wait(&tfull_bar[buf], bphase, &abort_sh, p.status)) break;
             tc_fence_after();
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::BUF_COLS;
-            es.row0 = tm * (2 * kBM) + static_cast<int>(rank) * kBM + q * 32;
+            es.row0 = tr.a_row + static_cast<int>(rank) * kBM + q * 32;
+            es.row_end = tr.row_end;
+            // A tensor store clips at the output's last row only: chunks that
+            // cross an expert's end are stored row by row.
+            es.tma_tile = GROUPED ? es.row0 + 32 <= tr.row_end : es.row0 < tr.row_end;
             pf.publish(colc);
             es.sx = pf.sx;
             es.rs = pf.rs;
             const int nt = tile + npairs;
-            if (nt < num_tiles) pf.fetch(p, (nt / tiles_m) * BN, (nt % tiles_m) * (2 * kBM) + rbase);
-            epilogue_tile<BN, KIND, false, QOUT>(p, tb, es.row0 + lane, tn * BN, 0, es);
+            if (nt < num_tiles) {
+                const TileRef tn = tile_ref(nt);
+                pf.fetch(p, tn.n_tile, tn.col_off, tn.a_row + rbase, tn.row_end);
+            }
+            epilogue_tile<BN, KIND, false, QOUT>(p, tb, es.row0 + lane, tr.n_tile, 0, es);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(buf));
@@ -1138,8 +1261,8 @@ q8_status run_tile(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tA16, tB16, tY, use_tmy, ep, num_kb, tiles_m, tiles_n) !=
-        cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tA16, tB16, tY, use_tmy, ep, num_kb, tiles_m, tiles_n,
+                           static_cast<const int32_t*>(nullptr), 0) != cudaSuccess) {
         cudaGetLastError();
         return Q8_ERR_LAUNCH;
     }
@@ -1205,7 +1328,8 @@ q8_status run_pair(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tY, use_tmy, ep, num_kb, tiles_m, tiles_n) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tY, use_tmy, ep, num_kb, tiles_m, tiles_n,
+                           static_cast<const int32_t*>(nullptr), 0) != cudaSuccess) {
         cudaGetLastError();
         return Q8_ERR_LAUNCH;
     }
@@ -1256,6 +1380,42 @@ q8_status run_decode(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     return Q8_OK;
 }
 
+
+template <int BN>
+q8_status run_grouped(const MoeArgs& a, const EpiParams& ep, cudaStream_t s) {
+    using C = TileCfg<BN, false>;
+    CUtensorMap tA, tB, tY;
+    if (!make_map(&tA, a.x_codes, false, a.k, a.m, a.ldx, kBKB, kBM) ||
+        !make_map(&tB, a.w_codes, false, a.k, a.experts * a.n, a.ldw, kBKB, BN))
+        return Q8_ERR_CUDA;
+    const int use_tmy = make_map_y(&tY, a.y, a.n, a.m, a.ldy) ? 1 : 0;
+    if (!use_tmy) tY = tA;
+    auto kern = gemm_tile_kernel<BN, kE4M3, false, false, true>;
+    if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
+    const int tiles_n = static_cast<int>((a.n + BN - 1) / BN);
+    // Upper bound of the tiles (each expert adds at most one partial row tile);
+    // the kernel reads the offsets and walks the actual ones.
+    const int64_t upper = ((a.m + kBM - 1) / kBM + a.experts) * tiles_n;
+    const int sms = sm_count();
+    const int grid = static_cast<int>(upper < sms ? upper : sms);
+    const int num_kb = static_cast<int>((a.k + kBKB - 1) / kBKB);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tA, tB, tY, use_tmy, ep, num_kb, 0, tiles_n, a.offsets,
+                           static_cast<int>(a.experts)) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    return Q8_OK;
+}
 
 template <int KIND>
 q8_status dispatch_kind(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
@@ -1325,6 +1485,88 @@ q8_status dispatch_kind(const LinearArgs& a, const EpiParams& ep, cudaStream_t s
 
 }  // namespace
 
+
+template <int BN>
+q8_status run_grouped_pair(const MoeArgs& a, const EpiParams& ep, cudaStream_t s) {
+    using C = PairCfg<BN>;
+    CUtensorMap tA, tB, tY;
+    if (!make_map(&tA, a.x_codes, false, a.k, a.m, a.ldx, kBKB, kBM) ||
+        !make_map(&tB, a.w_codes, false, a.k, a.experts * a.n, a.ldw, kBKB, BN / 2))
+        return Q8_ERR_CUDA;
+    const int use_tmy = make_map_y(&tY, a.y, a.n, a.m, a.ldy) ? 1 : 0;
+    if (!use_tmy) tY = tA;
+    auto kern = gemm_pair_kernel<BN, kE4M3, false, true>;
+    if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
+    const int tiles_n = static_cast<int>((a.n + BN - 1) / BN);
+    const int64_t upper = ((a.m + 2 * kBM - 1) / (2 * kBM) + a.experts) * tiles_n;
+    const int pairs_max = max_pairs(kern, C::SMEM);
+    const int pairs = static_cast<int>(upper < pairs_max ? upper : pairs_max);
+    const int num_kb = static_cast<int>((a.k + kBKB - 1) / kBKB);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tY, use_tmy, ep, num_kb, 0, tiles_n, a.offsets,
+                           static_cast<int>(a.experts)) != cudaSuccess) {
+        cudaGetLastError();
+        return Q8_ERR_LAUNCH;
+    }
+    return Q8_OK;
+}
+
+// Grouped FP8 rowwise linear on the persistent kernels with the expert-aware
+// tile map (at most kMaxGroupedExperts experts); Q8_ERR_SHAPE tells the
+// caller to use the one-tile-per-CTA kernel instead.
+q8_status launch_grouped_fp8(const MoeArgs& a, cudaStream_t s) {
+    if (a.experts > kMaxGroupedExperts) return Q8_ERR_SHAPE;
+    if (a.m == 0 || a.n == 0) return Q8_OK;
+    EpiParams ep = {};
+    ep.m = static_cast<int>(a.m);
+    ep.n = static_cast<int>(a.n);
+    ep.sx = a.sx;
+    ep.sw = a.sw;
+    ep.bias = a.bias;
+    ep.y = a.y;
+    ep.ldy = a.ldy;
+    ep.status = device_status_ptr();
+    // With 256 or more tokens per expert on average, 256-row tiles on CTA
+    // pairs: half the operand traffic per SM of 128-row tiles, which is what
+    // bounds these GEMMs, for at most half a tile of padding per expert.
+    if (a.m >= 256 * a.experts) {
+        if (a.n % 256 == 0 || a.n > 2048) return run_grouped_pair<256>(a, ep, s);
+        return run_grouped_pair<128>(a, ep, s);
+    }
+    // Output tile width: the persistent grid's makespan, waves x (BN + a
+    // tile's fixed cost of about 64 columns' worth), over an estimate of the
+    // row tiles (each expert adds about half a partial tile).
+    const int64_t sms = sm_count();
+    const int64_t rows_est = (a.m + kBM - 1) / kBM + a.experts / 2;
+    const int cand[4] = {256, 224, 192, 128};
+    int best = 256;
+    int64_t best_cost = INT64_MAX;
+    for (int bn : cand) {
+        const int64_t tiles = rows_est * ((a.n + bn - 1) / bn);
+        const int64_t cost = ((tiles + sms - 1) / sms) * (bn + 64);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    if (best == 256) return run_grouped<256>(a, ep, s);
+    if (best == 224) return run_grouped<224>(a, ep, s);
+    if (best == 192) return run_grouped<192>(a, ep, s);
+    return run_grouped<128>(a, ep, s);
+}
 
 q8_status launch_linear(const LinearArgs& a, cudaStream_t s) {
     if (a.m == 0 || a.n == 0) return Q8_OK;

@@ -121,6 +121,9 @@ struct MoeArgs {
 };
 
 q8_status launch_moe_fp8(const MoeArgs& a, cudaStream_t s);
+// The grouped linear on the persistent tile kernel (q8_gemm.cu); returns
+// Q8_ERR_SHAPE for more experts than its tile map holds.
+q8_status launch_grouped_fp8(const MoeArgs& a, cudaStream_t s);
 
 
 }  // namespace q8

@@ -273,6 +273,10 @@ bool make_map_u8(CUtensorMap* m, const void* base, uint64_t k, uint64_t rows, ui
 
 q8_status launch_moe_fp8(const MoeArgs& a, cudaStream_t s) {
     if (a.m == 0 || a.n == 0 || a.experts == 0) return Q8_OK;
+    // Persistent tile kernel with the expert-aware tile map when its map holds
+    // the experts; else one CTA per 128 x 128 tile below.
+    const q8_status st = launch_grouped_fp8(a, s);
+    if (st != Q8_ERR_SHAPE) return st;
     CUtensorMap tA, tB;
     if (!make_map_u8(&tA, a.x_codes, a.k, a.m, a.ldx, kBM) ||
         !make_map_u8(&tB, a.w_codes, a.k, a.experts * a.n, a.ldw, kBN))

@@ -510,6 +510,10 @@ __device__ __forceinline__ OutlierRuns scan_outlier_mask(const uint8_t* mask, in
     return r;
 }
 
+// Outlier columns a block lists in shared memory (by rank) for its gathers;
+// calls with more fall back to scattering from the mask runs.
+constexpr int kSmemOutliers = 1024;
+
 // Calls f(column, rank) for every outlier column of this thread's run.
 template <typename F>
 __device__ __forceinline__ void for_each_outlier(const OutlierRuns& r, F&& f) {
@@ -548,6 +552,7 @@ row_quant_kernel(RowQuantArgs a) {
     __shared__ int redi[kBlock / 32];
     __shared__ FixQueue fixq[kBlock / 32];
     __shared__ float cshare[kBlock / TPR][8];
+    __shared__ int s_oidx[kSkip ? kSmemOutliers : 1];   // LLM.int8: outlier column of each rank
     FixQueue* q = &fixq[threadIdx.x / 32];
 
     const int g = threadIdx.x / TPR;
@@ -586,13 +591,17 @@ row_quant_kernel(RowQuantArgs a) {
     // column list and the count (read by the GEMM that follows).
     OutlierRuns oruns;
     int cpad = 0;
+    bool olist = false;   // the block's outlier columns are listed in s_oidx
     if constexpr (kSkip) {
         oruns = scan_outlier_mask(a.skip, a.k, redi);
         cpad = (oruns.total + 63) / 64 * 64;
+        olist = oruns.total <= kSmemOutliers;
+        if (olist) for_each_outlier(oruns, [&](int64_t c, int rank) { s_oidx[rank] = static_cast<int>(c); });
         if (blockIdx.x == 0) {
             for_each_outlier(oruns, [&](int64_t c, int rank) { a.outlier_idx[rank] = static_cast<int32_t>(c); });
             if (threadIdx.x == 0) *a.outlier_count = oruns.total;
         }
+        __syncthreads();
     }
 
     for (int64_t row0 = static_cast<int64_t>(blockIdx.x) * RPB; row0 < a.rows;
@@ -793,9 +802,14 @@ row_quant_kernel(RowQuantArgs a) {
                     if (r >= a.rows) break;
                     const T* xs = static_cast<const T*>(a.src) + r * a.ld;
                     __half* xo = a.x_outlier + r * a.ldo;
-                    for_each_outlier(oruns, [&](int64_t c, int rank) { xo[rank] = xs[c]; });
-                    for (int j = oruns.total + static_cast<int>(threadIdx.x); j < cpad; j += kBlock)
-                        xo[j] = __float2half_rn(0.0f);
+                    if (olist) {
+                        for (int j = static_cast<int>(threadIdx.x); j < cpad; j += kBlock)
+                            xo[j] = j < oruns.total ? xs[s_oidx[j]] : __float2half_rn(0.0f);
+                    } else {
+                        for_each_outlier(oruns, [&](int64_t c, int rank) { xo[rank] = xs[c]; });
+                        for (int j = oruns.total + static_cast<int>(threadIdx.x); j < cpad; j += kBlock)
+                            xo[j] = __float2half_rn(0.0f);
+                    }
                 }
             }
         }
@@ -805,25 +819,34 @@ row_quant_kernel(RowQuantArgs a) {
     // zero-padded like X's: W16's own columns, or the dequantized codes
     // fp16(fl32(S (q - Z))) when only the 8-bit weight is kept.
     if constexpr (kSkip) {
-        for (int64_t r = blockIdx.x; r < a.w_rows; r += gridDim.x) {
-            __half* wo = a.w_outlier + r * a.ldo;
-            const float S = a.w_scale[r];
-            const float Zr = a.w_zero ? a.w_zero[r] : 0.0f;
-            for_each_outlier(oruns, [&](int64_t c, int rank) {
-                __half h;
-                if (a.w16 != nullptr) {
-                    h = a.w16[r * a.w_ld + c];
-                } else {
-                    const float q = a.w_codes_u8
-                                        ? static_cast<float>(static_cast<const uint8_t*>(a.w_codes)[r * a.w_ld + c])
-                                        : static_cast<float>(static_cast<const int8_t*>(a.w_codes)[r * a.w_ld + c]);
-                    const float d = a.w_zero ? __fsub_rn(q, Zr) : q;
-                    h = __float2half_rn(__fmul_rn(S, d));
-                }
-                wo[rank] = h;
-            });
-            for (int j = oruns.total + static_cast<int>(threadIdx.x); j < cpad; j += kBlock)
-                wo[j] = __float2half_rn(0.0f);
+        auto w16_of = [&](int64_t r, int64_t c, float S, float Zr) -> __half {
+            if (a.w16 != nullptr) return a.w16[r * a.w_ld + c];
+            const float q = a.w_codes_u8
+                                ? static_cast<float>(static_cast<const uint8_t*>(a.w_codes)[r * a.w_ld + c])
+                                : static_cast<float>(static_cast<const int8_t*>(a.w_codes)[r * a.w_ld + c]);
+            const float d = a.w_zero ? __fsub_rn(q, Zr) : q;
+            return __float2half_rn(__fmul_rn(S, d));
+        };
+        if (olist) {
+            // One weight row per warp at a time, so the rows' loads overlap.
+            const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+            for (int64_t r = static_cast<int64_t>(blockIdx.x) * (kBlock / 32) + warp; r < a.w_rows;
+                 r += static_cast<int64_t>(gridDim.x) * (kBlock / 32)) {
+                __half* wo = a.w_outlier + r * a.ldo;
+                const float S = a.w_scale[r];
+                const float Zr = a.w_zero ? a.w_zero[r] : 0.0f;
+                for (int j = lane; j < cpad; j += 32)
+                    wo[j] = j < oruns.total ? w16_of(r, s_oidx[j], S, Zr) : __float2half_rn(0.0f);
+            }
+        } else {
+            for (int64_t r = blockIdx.x; r < a.w_rows; r += gridDim.x) {
+                __half* wo = a.w_outlier + r * a.ldo;
+                const float S = a.w_scale[r];
+                const float Zr = a.w_zero ? a.w_zero[r] : 0.0f;
+                for_each_outlier(oruns, [&](int64_t c, int rank) { wo[rank] = w16_of(r, c, S, Zr); });
+                for (int j = oruns.total + static_cast<int>(threadIdx.x); j < cpad; j += kBlock)
+                    wo[j] = __float2half_rn(0.0f);
+            }
         }
     }
 }
@@ -933,11 +956,19 @@ __global__ void __launch_bounds__(kBlock) outlier_colmax_kernel(const T* __restr
 #pragma unroll
     for (int e = 0; e < 8; ++e) mx[e] = 0.f;
     if (col0 < k) {
-        for (int64_t r = rl; r < m; r += 64) {
-            float v[8];
-            load_vec<T>(X + r * ldx + col0, v);
+        // Four rows' loads in flight per thread at a time.
+        for (int64_t r0 = rl; r0 < m; r0 += 4 * 64) {
+            uint4 u[4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], fabsf(v[e]));
+            for (int i = 0; i < 4; ++i)
+                u[i] = r0 + i * 64 < m ? ld_stream16(X + (r0 + i * 64) * ldx + col0) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float v[8];
+                unpack_vec<T>(u[i], v);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], fabsf(v[e]));
+            }
         }
     }
 #pragma unroll
