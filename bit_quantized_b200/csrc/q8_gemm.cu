@@ -39,6 +39,7 @@
 #include <climits>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "q8_device.cuh"
 #include "q8_internal.h"
@@ -713,26 +714,29 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 // cta_group::2 TMA); the MMA's commits arrive on the stage-empty and
 // accumulator-full barriers of both CTAs; the accumulator-empty barriers of
 // the even CTA take one arrival from each epilogue warp of both CTAs.
-template <int BN>
+template <int BN, bool MIXED = false>
 struct PairCfg {
     static constexpr int A_BYTES = kBM * kBKB;            // this CTA's 128 activation rows
     static constexpr int B_BYTES = (BN / 2) * kBKB;       // this CTA's BN/2 weight rows
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int STAGES_RAW = kSmemBudget / STAGE;
     static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
-    static constexpr int BUF_COLS = BN;
-    static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+    static constexpr int BUF_COLS = MIXED ? 2 * BN : BN;  // int32 acc (+ fp32 outlier acc)
+    static constexpr int TMEM_COLS = 2 * BUF_COLS <= 256 ? 256 : 512;
+    static_assert(2 * BUF_COLS <= 512, "TMEM holds 512 columns");
     static constexpr int SMEM = STAGES * STAGE + kEpiStageBytes + kEpiConstBytes + 1024;
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "BN");
     static_assert((BN / 2) % 8 == 0, "weight half-tile rows: whole 8-row swizzle atoms");
 };
 
-template <int BN, int KIND, bool QOUT, bool GROUPED = false>
+template <int BN, int KIND, bool QOUT, bool GROUPED = false, bool MIXED = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmA16, const __grid_constant__ CUtensorMap tmB16,
                  const __grid_constant__ CUtensorMap tmY, int use_tmy, const EpiParams p, int num_kb,
                  int tiles_m, int tiles_n, const int32_t* group_offsets, int experts) {
-    using C = PairCfg<BN>;
+    using C = PairCfg<BN, MIXED>;
+    static_assert(!(GROUPED && MIXED), "grouped tiles carry no outlier stream");
     __shared__ int g_off[GROUPED ? kMaxGroupedExperts + 1 : 1];
     __shared__ int g_mt[GROUPED ? kMaxGroupedExperts + 1 : 1];
     extern __shared__ uint8_t smem_raw[];
@@ -782,6 +786,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     pdl_launch_dependents();
 
     const int num_tiles = GROUPED ? g_mt[GROUPED ? experts : 0] * tiles_n : tiles_m * tiles_n;
+    // LLM.int8: the fp16 outlier K blocks (64 columns each) follow the int8
+    // ones; their count is read on the device (no host round trip).
+    int n16_kb = 0;
+    if constexpr (MIXED) {
+        pdl_wait();
+        n16_kb = (*p.outlier_count + 63) / 64;
+    }
+    const int total_kb = num_kb + n16_kb;
     // A pair tile is 256 activation rows (128 from each CTA) x BN columns.
     auto tile_ref = [&](int tile) -> TileRef {
         if constexpr (GROUPED) return grouped_tile(tile, g_off, g_mt, experts, 2 * kBM, BN, p.n);
@@ -799,7 +811,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
                 const TileRef tr = tile_ref(tile);
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int kb = 0; kb < total_kb; ++kb) {
                     if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
                         ok = false;
                         break;
@@ -808,8 +820,16 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     uint8_t* sb = sa + C::A_BYTES;
                     if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE);
                     const uint32_t fb = full0 + 8u * static_cast<uint32_t>(stage);
-                    tma_load_2d_pair(sa, &tmA, fb, kb * kBKB, tr.a_row + static_cast<int>(rank) * kBM);
-                    tma_load_2d_pair(sb, &tmB, fb, kb * kBKB, tr.b_row + static_cast<int>(rank) * (BN / 2));
+                    const int ya = tr.a_row + static_cast<int>(rank) * kBM;
+                    const int yb = tr.b_row + static_cast<int>(rank) * (BN / 2);
+                    if (!MIXED || kb < num_kb) {
+                        tma_load_2d_pair(sa, &tmA, fb, kb * kBKB, ya);
+                        tma_load_2d_pair(sb, &tmB, fb, kb * kBKB, yb);
+                    } else {
+                        // 64 fp16 columns: the same 128-byte rows
+                        tma_load_2d_pair(sa, &tmA16, fb, (kb - num_kb) * 64, ya);
+                        tma_load_2d_pair(sb, &tmB16, fb, (kb - num_kb) * 64, yb);
+                    }
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1;
@@ -823,6 +843,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         if (rank == 0 && elect_one()) {
             const uint32_t idesc = KIND == kE4M3 ? make_idesc(1, 0, 0, 2 * kBM, BN)
                                                  : make_idesc(2, 1, KIND == kS8U8 ? 0 : 1, 2 * kBM, BN);
+            const uint32_t idesc16 = make_idesc(1, 0, 0, 2 * kBM, BN);   // f16 x f16 -> f32
             int stage = 0;
             uint32_t phase = 0;
             int buf = 0;
@@ -835,7 +856,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 }
                 tc_fence_after();
                 const uint32_t d = tmem_base + buf * C::BUF_COLS;
-                for (int kb = 0; kb < num_kb; ++kb) {
+                for (int kb = 0; kb < total_kb; ++kb) {
                     if (!mbar_wait(&full_bar[stage], phase, &abort_sh, p.status)) {
                         ok = false;
                         break;
@@ -844,12 +865,19 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     const uint32_t sa = smem_addr(smem + stage * C::STAGE);
                     const uint64_t ad = sdesc_kmajor_sw128(sa);
                     const uint64_t bd = sdesc_kmajor_sw128(sa + C::A_BYTES);
+                    if (!MIXED || kb < num_kb) {
 #pragma unroll
-                    for (int ks = 0; ks < kBKB / 32; ++ks) {
-                        if constexpr (KIND == kE4M3)
-                            mma_issue_pair<kKindF8>(d, ad + 2 * ks, bd + 2 * ks, idesc, (kb | ks) != 0);
-                        else
-                            mma_issue_pair<kKindI8>(d, ad + 2 * ks, bd + 2 * ks, idesc, (kb | ks) != 0);
+                        for (int ks = 0; ks < kBKB / 32; ++ks) {
+                            if constexpr (KIND == kE4M3)
+                                mma_issue_pair<kKindF8>(d, ad + 2 * ks, bd + 2 * ks, idesc, (kb | ks) != 0);
+                            else
+                                mma_issue_pair<kKindI8>(d, ad + 2 * ks, bd + 2 * ks, idesc, (kb | ks) != 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < kBKB / 32; ++ks)
+                            mma_issue_pair<kKindF16>(d + BN, ad + 2 * ks, bd + 2 * ks, idesc16,
+                                                     ((kb - num_kb) | ks) != 0);
                     }
                     tc_commit_pair(&empty_bar[stage], 0x3);
                     if (++stage == C::STAGES) {
@@ -905,7 +933,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const TileRef tn = tile_ref(nt);
                 pf.fetch(p, tn.n_tile, tn.col_off, tn.a_row + rbase, tn.row_end);
             }
-            epilogue_tile<BN, KIND, false, QOUT>(p, tb, es.row0 + lane, tr.n_tile, 0, es);
+            epilogue_tile<BN, KIND, MIXED, QOUT>(p, tb, es.row0 + lane, tr.n_tile, n16_kb, es);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(tempty0 + 8u * static_cast<uint32_t>(buf));
@@ -1217,14 +1245,46 @@ bool make_map_y(CUtensorMap* m, const void* y, uint64_t n, uint64_t rows, uint64
 }
 
 int sm_count() {
+    static int cached[64] = {0};
     int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return n;
+    }
+    if (cached[dev] > 0) return cached[dev];
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 148;
+    }
+    cached[dev] = n;
     return n;
 }
 
+// The dynamic shared-memory limit is a per-kernel, per-device attribute: it is
+// set once (to the largest size asked for) instead of on every launch, which
+// keeps the host side of a call short.
 template <typename K>
 cudaError_t set_smem(K kernel, int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    static std::mutex mu;
+    static std::unordered_map<const void*, int> done[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    }
+    const void* key = reinterpret_cast<const void*>(kernel);
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = done[dev].find(key);
+        if (it != done[dev].end() && it->second >= bytes) return cudaSuccess;
+    }
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) {
+        std::lock_guard<std::mutex> lk(mu);
+        int& v = done[dev][key];
+        if (bytes > v) v = bytes;
+    }
+    return e;
 }
 
 template <int BN, int KIND, bool MIXED, bool QOUT = false>
@@ -1297,16 +1357,24 @@ int max_pairs(K kernel, int smem) {
     return n;
 }
 
-template <int BN, int KIND, bool QOUT = false>
+template <int BN, int KIND, bool QOUT = false, bool MIXED = false>
 q8_status run_pair(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
-    using C = PairCfg<BN>;
-    CUtensorMap tA, tB;
+    using C = PairCfg<BN, MIXED>;
+    CUtensorMap tA, tB, tA16, tB16;
     if (!make_map(&tA, a.a_codes, false, a.k, a.m, a.lda, kBKB, kBM) ||
         !make_map(&tB, a.b_codes, false, a.k, a.n, a.ldb, kBKB, BN / 2))
         return Q8_ERR_CUDA;
+    if constexpr (MIXED) {
+        if (!make_map(&tA16, a.xo, true, a.k16_cap, a.m, a.ldxo * 2, 64, kBM) ||
+            !make_map(&tB16, a.wo, true, a.k16_cap, a.n, a.ldwo * 2, 64, BN / 2))
+            return Q8_ERR_CUDA;
+    } else {
+        tA16 = tA;
+        tB16 = tB;
+    }
     CUtensorMap tY = tA;
     const int use_tmy = (!QOUT && a.y != nullptr && make_map_y(&tY, a.y, a.n, a.m, a.ldy)) ? 1 : 0;
-    auto kern = gemm_pair_kernel<BN, KIND, QOUT>;
+    auto kern = gemm_pair_kernel<BN, KIND, QOUT, false, MIXED>;
     if (set_smem(kern, C::SMEM) != cudaSuccess) return Q8_ERR_LAUNCH;
     const int tiles_m = static_cast<int>((a.m + 2 * kBM - 1) / (2 * kBM));
     const int tiles_n = static_cast<int>((a.n + BN - 1) / BN);
@@ -1328,7 +1396,7 @@ q8_status run_pair(const LinearArgs& a, const EpiParams& ep, cudaStream_t s) {
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tY, use_tmy, ep, num_kb, tiles_m, tiles_n,
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tA16, tB16, tY, use_tmy, ep, num_kb, tiles_m, tiles_n,
                            static_cast<const int32_t*>(nullptr), 0) != cudaSuccess) {
         cudaGetLastError();
         return Q8_ERR_LAUNCH;
@@ -1516,7 +1584,7 @@ q8_status run_grouped_pair(const MoeArgs& a, const EpiParams& ep, cudaStream_t s
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tY, use_tmy, ep, num_kb, 0, tiles_n, a.offsets,
+    if (cudaLaunchKernelEx(&cfg, kern, tA, tB, tA, tB, tY, use_tmy, ep, num_kb, 0, tiles_n, a.offsets,
                            static_cast<int>(a.experts)) != cudaSuccess) {
         cudaGetLastError();
         return Q8_ERR_LAUNCH;
@@ -1587,6 +1655,12 @@ q8_status launch_linear(const LinearArgs& a, cudaStream_t s) {
     ep.outlier_count = a.outlier_count;
     ep.status = device_status_ptr();
     if (a.outlier_count != nullptr) {
+        // More than one 128-row tile of tokens: 256-row tiles on CTA pairs
+        // (a quarter fewer operand bytes per SM, which bounds these GEMMs).
+        if (a.m > kBM) {
+            if (a.kind == kS8U8) return run_pair<128, kS8U8, false, true>(a, ep, s);
+            return run_pair<128, kS8S8, false, true>(a, ep, s);
+        }
         if (a.kind == kS8U8) return run_tile<128, kS8U8, true>(a, ep, s);
         return run_tile<128, kS8S8, true>(a, ep, s);
     }

@@ -475,16 +475,25 @@ struct OutlierRuns {
 
 __device__ __forceinline__ OutlierRuns scan_outlier_mask(const uint8_t* mask, int64_t k, int* sh) {
     OutlierRuns r;
-    r.per = static_cast<int>((k + kBlock - 1) / kBlock);
+    // Runs of a multiple of 16 columns, read as 16-byte vectors (the mask is
+    // 16-byte aligned and padded to the vector by the k % 32 == 0 rule).
+    r.per = static_cast<int>((k + 16 * kBlock - 1) / (16 * kBlock)) * 16;
     r.begin = static_cast<int64_t>(threadIdx.x) * r.per;
     int local = 0;
 #pragma unroll
     for (int w = 0; w < 4; ++w) r.bits[w] = 0u;
-    for (int j = 0; j < r.per; ++j) {
-        const int64_t c = r.begin + j;
-        if (c < k && mask[c] != 0) {
-            r.bits[j / 32] |= 1u << (j % 32);
-            ++local;
+    for (int j0 = 0; j0 < r.per; j0 += 16) {
+        const int64_t c0 = r.begin + j0;
+        if (c0 >= k) break;
+        const uint4 v = *reinterpret_cast<const uint4*>(mask + c0);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+            if ((wv[b / 4] >> (8 * (b % 4))) & 0xFFu) {
+                const int j = j0 + b;
+                r.bits[j / 32] |= 1u << (j % 32);
+                ++local;
+            }
         }
     }
     // exclusive scan of `local` over the block
