@@ -225,7 +225,7 @@ def step_functions(q8, w):
         def step(L, X=None):
             q8.q8_linear_int8_mixed(L["X"] if X is None else X, L["qw"], w.threshold,
                                     out=L["Y"], workspace=L["ws"])
-        return step, step, 5
+        return step, step, 3
     scheme = "int8" if w.kind == "w8a8_int8" else "fp8"
 
     def step(L, X=None):
@@ -653,7 +653,7 @@ def extras(q8, dev, pk):
                                                              workspace=ws), flush)
             r["mixed_call_us"] = round(t * 1e3, 2)
             r["tops"] = round(2.0 * w.m * w.n * w.k / (t * 1e-3) / 1e12, 2)
-            r["launches_per_call"] = 5
+            r["launches_per_call"] = 3
         else:
             scheme = "int8" if w.kind == "w8a8_int8" else "fp8"
             qa = q8.q8_quantize_act(Xd, scheme, clip_ub=w.clip_ub)
