@@ -128,24 +128,22 @@ __device__ __forceinline__ uint32_t requant_code(float y, float S) {
            0xFFu;
 }
 
-// The same code without a division per output: the bracket of the
-// quantizers, 1/S rounded down and up and widened by (1 -+ 2^-23), so that
-// y * rlo and y * rhi enclose fl32(y / S).  Where both ends round to the same
-// integer (RN(y r + 1.5 * 2^23), exact product) that is the code; outputs whose
-// bracket lies beyond 127.5 saturate; the rest (near a rounding boundary) take
-// the division.
+// The same code without a division per output.  y is clamped to
+// [-128 S, 128 S] first (128 S is exact; codes beyond it saturate either way),
+// so that q = RN(y / S) comes from R = RN(1/S) with qm::quotient (exact in
+// that range), then q is clamped to [-127, 127] and rounded half to even by
+// RN(q + 1.5 * 2^23), whose low byte is the code.  Scales below 2^-90 divide.
 struct Requant {
-    float S, rlo, rhi;
+    float S, R, T;
+    bool direct;
 };
 
 __device__ __forceinline__ Requant requant_consts(float S) {
     Requant c;
     c.S = S;
-    float rd, ru;
-    qm::reciprocal_bounds(S, rd, ru);
-    const bool exact = rd == ru;   // S a power of two: y * (1/S) = y / S exactly
-    c.rlo = exact ? rd : __fmul_rd(rd, 1.0f - 0x1p-23f);
-    c.rhi = exact ? ru : __fmul_ru(ru, 1.0f + 0x1p-23f);
+    c.R = __frcp_rn(S);
+    c.T = __fmul_rn(S, 128.0f);
+    c.direct = !(S >= qm::kScaleMin);
     return c;
 }
 
@@ -153,33 +151,18 @@ __device__ __forceinline__ Requant requant_consts(float S) {
 // cache with the MMA warp's loop).
 __device__ __noinline__ uint32_t requant_code_slow(float y, float S) { return requant_code(y, S); }
 
-// Branch-free codes of 4 outputs: both ends of the bracket rounded with
-// RN(y r + 1.5 * 2^23) and clamped to the code range in that domain (exact:
-// the bounds are integers there; values too large for the magic constant still
-// clamp on the right side).  A byte where the ends differ is recomputed by the
-// caller; `diff` gets its bit.
-__device__ __forceinline__ uint32_t requant_codes4(const float* y, const Requant& c, uint32_t& diff, int bit0) {
-    constexpr float lo = qm::kMagic - 127.0f, hi = qm::kMagic + 127.0f;
-    uint32_t w = 0u;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float l = fminf(fmaxf(__fmaf_rn(y[e], c.rlo, qm::kMagic), lo), hi);
-        const float h = fminf(fmaxf(__fmaf_rn(y[e], c.rhi, qm::kMagic), lo), hi);
-        w |= (__float_as_uint(l) & 0xFFu) << (8 * e);
-        diff |= (l != h ? 1u : 0u) << (bit0 + e);
-    }
-    return w;
+__device__ __forceinline__ uint32_t requant_code_fast(float y, const Requant& c) {
+    if (c.direct) return requant_code_slow(y, c.S);
+    const float q = qm::quotient(fminf(fmaxf(y, -c.T), c.T), c.S, c.R);
+    return __float_as_uint(__fadd_rn(fminf(fmaxf(q, -127.0f), 127.0f), qm::kMagic)) & 0xFFu;
 }
 
-__device__ __forceinline__ uint32_t requant_code_fast(float y, const Requant& c) {
-    const float a = fabsf(y);
-    if (a * c.rhi < 127.5f) {
-        const float l = __fmaf_rn(y, c.rlo, qm::kMagic), h = __fmaf_rn(y, c.rhi, qm::kMagic);
-        if (l == h) return __float_as_uint(l) & 0xFFu;
-    } else if (a * c.rlo > 127.5f) {
-        return y > 0.f ? 127u : 0x81u;   // -127
-    }
-    return requant_code_slow(y, c.S);
+// Codes of 4 outputs, packed in order.
+__device__ __forceinline__ uint32_t requant_codes4(const float* y, const Requant& c) {
+    uint32_t w = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w |= requant_code_fast(y[e], c) << (8 * e);
+    return w;
 }
 
 // bf16_rne(a) in the low half, bf16_rne(b) in the high half (one conversion).
@@ -348,16 +331,9 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& p, uint32_t tb, i
         } else if (row_ok) {
             if constexpr (QOUT) {
                 const Requant rq = requant_consts(p.out_scale);
-                uint32_t w[8], diff = 0u;
+                uint32_t w[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) w[j] = requant_codes4(&out[4 * j], rq, diff, 4 * j);
-                if (diff != 0u) {   // rare: outputs near a rounding boundary
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if ((diff >> i) & 1u)
-                            w[i / 4] = (w[i / 4] & ~(0xFFu << (8 * (i % 4)))) |
-                                       (requant_code_slow(out[i], rq.S) << (8 * (i % 4)));
-                }
+                for (int j = 0; j < 8; ++j) w[j] = requant_codes4(&out[4 * j], rq);
                 uint4* qp = reinterpret_cast<uint4*>(p.yq + static_cast<int64_t>(row) * p.ldy + n0);
                 qp[0] = make_uint4(w[0], w[1], w[2], w[3]);
                 if (nv > 16) qp[1] = make_uint4(w[4], w[5], w[6], w[7]);

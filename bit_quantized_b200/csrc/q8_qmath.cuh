@@ -1,6 +1,8 @@
-// Scalar pieces of the quantizers: constants of the division-free rounding and
-// the directed reciprocals that bracket the IEEE quotient x / S.
+// Scalar pieces of the quantizers: the IEEE fp32 quotient x / S without a
+// division instruction, and the constant of the integer rounding.
 #pragma once
+
+#include <cuda_runtime.h>
 
 #include <cstdint>
 
@@ -8,18 +10,51 @@ namespace q8 {
 namespace qm {
 
 constexpr float kEps = 1e-8f;
-constexpr float kMagic = 12582912.0f;     // 1.5 * 2^23: x + kMagic rounds x to an integer
-constexpr float kFastLimit = 2097152.0f;  // 2^21: bound on |x * r| for the integer fast path
+constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23: RN(q + kMagic) is q rounded to an integer
 
-// 1/S rounded down and up, from R = RN(1/S) and the sign of the residual
-// 1 - S R, which one FMA gives exactly (|1 - S R| <= 2^-24 fits in a float).
-// Equal when S is a power of two (1/S exact).  S is a positive normal float.
-__device__ __forceinline__ void reciprocal_bounds(float S, float& rd, float& ru) {
-    const float R = __frcp_rn(S);
-    const float res = __fmaf_rn(-S, R, 1.0f);
-    const uint32_t rb = __float_as_uint(R);
-    rd = res < 0.f ? __uint_as_float(rb - 1u) : R;   // R > 1/S: one ulp down
-    ru = res > 0.f ? __uint_as_float(rb + 1u) : R;   // R < 1/S: one ulp up
+// The quotient below is exact when |x / S| < 2^99 and S >= 2^-90 (no overflow,
+// and the residuals of quotients large enough to matter for a code do not
+// underflow); callers divide outside that domain.
+constexpr float kQuotientMax = 0x1p99f;
+constexpr float kScaleMin = 0x1p-90f;
+
+// RN(x / S), the correctly rounded fp32 quotient, from R = RN(1/S) with four
+// fused multiply-adds, after Markstein ("Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990; also
+// Muller et al., Handbook of Floating-Point Arithmetic, the chapter on
+// division with an FMA).
+//   q0 = RN(x R) is within about 1.5 ulp of x / S (R and the product each
+//   round once).
+//   One correction q1 = RN(q0 + RN(x - q0 S) R): the corrected value is
+//   within about 2^-46 relative of x / S, so q1 is a faithful rounding (one
+//   of the two floats around x / S).
+//   Markstein's theorem: with R within half an ulp of 1/S and q1 faithful,
+//   the residual x - q1 S is a float (the FMA computes it exactly) and
+//   RN(q1 + (x - q1 S) R) = RN(x / S).
+// The residuals are kept negated (q S - x) and subtracted, so that x = -0
+// keeps its sign through the corrections (-0 / S = -0).
+__device__ __forceinline__ float quotient(float x, float S, float R) {
+    const float q0 = __fmul_rn(x, R);
+    const float e0 = __fmaf_rn(q0, S, -x);
+    const float q1 = __fmaf_rn(-e0, R, q0);
+    const float e1 = __fmaf_rn(q1, S, -x);
+    return __fmaf_rn(-e1, R, q1);
+}
+
+// The same for two elements with paired fp32 instructions.  The residuals
+// are formed as x - q S (nS = -S), which loses the sign of a zero x; with
+// SIGNED_ZERO the sign of x is put back (every other quotient has it already),
+// for codes that keep the sign of zero (E4M3).
+template <bool SIGNED_ZERO>
+__device__ __forceinline__ float2 quotient2(float2 x, float2 nS, float2 R) {
+    const float2 q0 = __fmul2_rn(x, R);
+    const float2 e0 = __ffma2_rn(q0, nS, x);
+    const float2 q1 = __ffma2_rn(e0, R, q0);
+    const float2 e1 = __ffma2_rn(q1, nS, x);
+    const float2 q2 = __ffma2_rn(e1, R, q1);
+    if constexpr (!SIGNED_ZERO) return q2;
+    return make_float2(__uint_as_float(__float_as_uint(q2.x) | (__float_as_uint(x.x) & 0x80000000u)),
+                       __uint_as_float(__float_as_uint(q2.y) | (__float_as_uint(x.y) & 0x80000000u)));
 }
 
 }  // namespace qm

@@ -38,7 +38,6 @@ namespace q8 {
 namespace {
 
 using qm::kEps;
-using qm::kFastLimit;
 using qm::kMagic;
 constexpr int kBlock = 256;
 constexpr int kMaxVec = 16;   // 16-byte vectors a thread keeps in registers
@@ -160,30 +159,32 @@ __device__ __forceinline__ float clampf(float v, float lo, float hi) {
 // Codes of one 16-byte vector (V elements) without a division per element.
 //
 // The target is a rounding of the IEEE quotient fl32(x / S): rne for integer
-// codes, E4M3 (half to even, saturating) for FP8.  Each row gets two
-// multipliers rlo <= 1/S <= rhi, made with directed roundings and widened so
-// that x * rlo and x * rhi (after the fast path's own rounding) enclose
-// fl32(x / S), with fl32(x / S) strictly inside for integer codes.  Both
-// roundings are monotonic, so where the two ends of the bracket give the same
-// code, that is the code of fl32(x / S).  Elements where they differ lie within
-// a few ulps of a rounding boundary; their codes are recomputed with an exact
-// division.  That is not as rare as the bracket width suggests: with 16-bit
-// inputs, x / S often falls exactly on a boundary (127 x / absmax is a ratio of
-// two short mantissas), about 2 elements in 1000.
-//   Integer codes: one fused multiply-add per end, y = RN(x * r + c), with
-//   c = 1.5 * 2^23 (+ Z + bias for asymmetric codes).  The exact product plus
-//   c lies in [2^23, 2^24), where floats are the integers, so y - c is x * r
-//   rounded to an integer and the low byte of y is the code byte.  With Z
-//   folded into c an exact tie would round to the parity of c, but a tie
-//   strictly inside the bracket makes the two ends differ, so folded ties are
-//   always recomputed.  Rows where |x * r| could leave that range, or whose
-//   codes would need the [-128, 127] clamp, are coded exactly throughout
-//   (constant rows, rows that do not cross zero).
-//   E4M3 codes: t = RN(x * r) per end, then the hardware conversion.
+// codes, E4M3 (half to even, saturating) for FP8.  Each row gets R = RN(1/S),
+// and every element's quotient is formed exactly from it with one multiply and
+// two FMA corrections (qm::quotient: Markstein's correction step).  No element
+// needs a division, and there is no special case for quotients that fall on a
+// rounding boundary (with 16-bit inputs, x / S falls exactly on one about 2
+// times in 1000: 127 x / absmax is a ratio of two short significands).
+//   Integer codes: t = RN(q + 1.5 * 2^23) lies in [2^23, 2^24), where floats
+//   are the integers, so t is q rounded half to even and the low byte of t's
+//   bits is the code's two's-complement byte.  The code range [-127, 127]
+//   (static), or [-128, 127] after adding Z (asymmetric), is applied to q
+//   before the rounding: its bounds are integers, so clamping first and
+//   rounding second give the same code.  Z and the unsigned-storage bias are
+//   added after the rounding (added before it, an odd Z would move the ties).
+//   Dynamic symmetric rows need no clamp: |x| <= absmax makes |q| <= 127
+//   (1 + 2^-23).
+//   E4M3 codes: the hardware conversion of q (round to nearest even,
+//   saturating to 448).
+// Rows whose quotients could reach 2^99 (a static or clipped scale far below
+// the row's values, asymmetric rows far from zero) or whose scale is below
+// 2^-90 are coded with an IEEE division per element instead.
 
 // Internal op for the LLM.int8 regular stream: int8 activations with the
 // outlier columns (mask bytes of 1) left out of the absmax and coded as 0.
 constexpr int kOpActInt8Skip = 5;
+
+__host__ __device__ constexpr bool is_fp8_op(int op) { return op == kOpActFp8 || op == kOpWeightFp8; }
 
 __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
     return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
@@ -194,9 +195,10 @@ __device__ __forceinline__ float2 splat2(float a) { return make_float2(a, a); }
 // Per-row constants.
 struct RowConsts {
     float S, Z, bias;
-    float rlo, rhi;   // bracket multipliers
-    float add;        // integer codes: 1.5 * 2^23 + Z + bias
-    bool fast;        // the row may use the bracket path
+    float R;          // RN(1/S)
+    float qlo, qhi;   // integer codes: bounds of q before the rounding
+    float post;       // integer codes: Z + bias, added after the rounding
+    bool direct;      // code the row with a division per element
 };
 
 template <int OP>
@@ -205,54 +207,32 @@ __device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, 
     RowConsts c;
     c.Z = 0.f;
     c.bias = bias;
+    float vmax = amax;   // largest |x| of the row
     if constexpr (OP == kOpActInt8Static) {
         c.S = static_scale;   // calibrated, > 0 (checked by the caller)
     } else if constexpr (OP == kOpActInt8 || OP == kOpActInt8Skip || OP == kOpActInt8Smooth ||
                          OP == kOpWeightSym) {
         c.S = __fdiv_rn(amax, 127.0f);
-    } else if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
+    } else if constexpr (is_fp8_op(OP)) {
         if (OP == kOpActFp8 && clip_ub > 0.f) amax = fminf(amax, clip_ub);
         c.S = __fdiv_rn(amax, 448.0f);
     } else {
         c.S = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
+        vmax = fmaxf(fabsf(lo), fabsf(hi));
     }
     if (OP != kOpActInt8Static && !(c.S >= kEps)) c.S = kEps;
-    // When S is a power of two, 1/S is exact and so is x * (1/S) = x / S (the
-    // product keeps x's significand): no bracket is needed, except for
-    // asymmetric codes with an odd Z + bias folded into the rounding constant.
-    float rd, ru;
-    qm::reciprocal_bounds(c.S, rd, ru);
-    const bool exact_rcp = rd == ru;
-    if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
-        // t = RN(x * r) adds one more rounding (2^-24) on top of the ends.
-        c.rlo = exact_rcp ? rd : __fmul_rd(rd, 1.0f - 0x1p-22f);
-        c.rhi = exact_rcp ? ru : __fmul_ru(ru, 1.0f + 0x1p-22f);
-        c.add = 0.f;
-        c.fast = true;
-    } else {
-        // fl32(x / S) is within 2^-24 of x / S; the (1 -+ 2^-23) factors put it
-        // strictly inside [x * rlo, x * rhi] (the products are exact in the FMA).
-        c.rlo = __fmul_rd(rd, 1.0f - 0x1p-23f);
-        c.rhi = __fmul_ru(ru, 1.0f + 0x1p-23f);
-        if constexpr (OP == kOpWeightAsym) {
-            c.Z = clampf(__fsub_rn(rintf(__fdiv_rn(-lo, c.S)), 128.0f), -128.0f, 127.0f);
-            // Codes are monotonic in w: the ends of the row bound all of them.
-            const float qlo = __fadd_rn(rintf(__fdiv_rn(lo, c.S)), c.Z);
-            const float qhi = __fadd_rn(rintf(__fdiv_rn(hi, c.S)), c.Z);
-            c.fast = fmaxf(fabsf(lo), fabsf(hi)) * c.rhi <= kFastLimit && qlo >= -128.0f && qhi <= 127.0f;
-            if (exact_rcp && (static_cast<int>(c.Z + bias) & 1) == 0) c.rlo = c.rhi = rd;
-        } else if constexpr (OP == kOpActInt8Static) {
-            // Codes of a static scale may saturate: the fast path (which does
-            // not clamp) needs every |fl32(x / S)| below 127.5, which
-            // absmax * rhi < 127.5 guarantees; other rows are coded exactly.
-            c.fast = amax * c.rhi < 127.5f;
-            if (exact_rcp) c.rlo = c.rhi = rd;
-        } else {
-            c.fast = amax * c.rhi <= kFastLimit;
-            if (exact_rcp) c.rlo = c.rhi = rd;
-        }
-        c.add = kMagic + c.Z + bias;   // an integer below 2^24: exact
+    c.R = __frcp_rn(c.S);
+    c.qlo = -127.0f;
+    c.qhi = 127.0f;
+    c.post = 0.f;
+    if constexpr (OP == kOpWeightAsym) {
+        c.Z = clampf(__fsub_rn(rintf(__fdiv_rn(-lo, c.S)), 128.0f), -128.0f, 127.0f);
+        c.qlo = -128.0f - c.Z;   // integers: exact
+        c.qhi = 127.0f - c.Z;
+        c.post = c.Z + bias;
     }
+    // NaN-safe: a NaN or infinite product also takes the division.
+    c.direct = !(vmax * c.R < qm::kQuotientMax) || !(c.S >= qm::kScaleMin);
     return c;
 }
 
@@ -278,147 +258,55 @@ __device__ __forceinline__ void values_of(const uint4 u, const float* mv, float 
     }
 }
 
-// Fast codes of one vector from the lower end of the bracket, and per word the
-// code bytes where the upper end disagrees.  keep clears the bytes of left-out
-// columns (all ones otherwise); their disagreements do not count.
-template <typename T, int OP>
-__device__ __forceinline__ void fast_codes(const uint4 u, const RowConsts& c, const uint2 keep,
-                                           uint32_t (&words)[2], uint32_t (&diff)[2],
-                                           const float* mv = nullptr) {
+// Codes of one vector, packed in element order (element 4w + b in byte b of
+// word w).  keep clears the bytes of left-out columns (all ones otherwise).
+// DIRECT divides (rows outside the quotient's exact domain).
+template <typename T, int OP, bool DIRECT>
+__device__ __forceinline__ uint2 code_vec(const uint4 u, const RowConsts& c, const uint2 keep,
+                                          const float* mv = nullptr) {
     constexpr int V = VecOf<T>::N;
-    const uint32_t kp[2] = {keep.x, keep.y};
     float v[V];
     values_of<T, OP>(u, mv, v);
-    words[1] = diff[1] = 0u;
-    if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
-        const float2 L = splat2(c.rlo), H = splat2(c.rhi);
+    float2 q[V / 2];
+    if constexpr (DIRECT) {
+#pragma unroll
+        for (int e = 0; e < V / 2; ++e) q[e] = make_float2(__fdiv_rn(v[2 * e], c.S), __fdiv_rn(v[2 * e + 1], c.S));
+    } else {
+        const float2 nS = splat2(-c.S), R = splat2(c.R);
+#pragma unroll
+        for (int e = 0; e < V / 2; ++e)
+            q[e] = qm::quotient2<is_fp8_op(OP)>(make_float2(v[2 * e], v[2 * e + 1]), nS, R);
+    }
+    uint32_t words[2] = {0u, 0u};
+    if constexpr (is_fp8_op(OP)) {
 #pragma unroll
         for (int w = 0; w < V / 4; ++w) {
-            uint32_t cl[2], cd[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float2 x2 = make_float2(v[4 * w + 2 * h], v[4 * w + 2 * h + 1]);
-                cl[h] = __nv_cvt_float2_to_fp8x2(__fmul2_rn(x2, L), __NV_SATFINITE, __NV_E4M3);
-                cd[h] = cl[h] ^ __nv_cvt_float2_to_fp8x2(__fmul2_rn(x2, H), __NV_SATFINITE, __NV_E4M3);
-            }
-            // element 2h in the low byte of each half, 2h + 1 in the high byte
-            words[w] = __byte_perm(cl[0], cl[1], 0x5410);
-            diff[w] = __byte_perm(cd[0], cd[1], 0x5410);
+            const uint32_t c0 = __nv_cvt_float2_to_fp8x2(q[2 * w], __NV_SATFINITE, __NV_E4M3);
+            const uint32_t c1 = __nv_cvt_float2_to_fp8x2(q[2 * w + 1], __NV_SATFINITE, __NV_E4M3);
+            words[w] = __byte_perm(c0, c1, 0x5410);   // element 2h in the low byte of each half
         }
     } else {
-        const float2 L = splat2(c.rlo), H = splat2(c.rhi), A = splat2(c.add);
+        constexpr bool kClamp = OP == kOpActInt8Static || OP == kOpWeightAsym || DIRECT;
+        const float2 M = splat2(kMagic), P = splat2(c.post);
+        float2 t[V / 2];
 #pragma unroll
-        for (int w = 0; w < V / 4; ++w) {
-            const float2 x0 = make_float2(v[4 * w], v[4 * w + 1]);
-            const float2 x1 = make_float2(v[4 * w + 2], v[4 * w + 3]);
-            const float2 l0 = __ffma2_rn(x0, L, A), l1 = __ffma2_rn(x1, L, A);
-            const float2 h0 = __ffma2_rn(x0, H, A), h1 = __ffma2_rn(x1, H, A);
-            const uint32_t lw = pack_low_bytes(__float_as_uint(l0.x), __float_as_uint(l0.y),
-                                               __float_as_uint(l1.x), __float_as_uint(l1.y)) & kp[w];
-            const uint32_t hw = pack_low_bytes(__float_as_uint(h0.x), __float_as_uint(h0.y),
-                                               __float_as_uint(h1.x), __float_as_uint(h1.y)) & kp[w];
-            words[w] = lw;
-            diff[w] = lw ^ hw;
-        }
-    }
-}
-
-// Exact codes, with an IEEE division, for the elements of a vector whose byte
-// in `redo` is nonzero; the other bytes of `words` are kept.  Out of line: it
-// runs for a few elements in a thousand.
-template <typename T, int OP>
-__device__ __noinline__ uint2 exact_codes(const uint4 u, float S, float Z, float bias, uint2 redo,
-                                          uint2 words, const float* mult_vec) {
-    constexpr int V = VecOf<T>::N;
-    float v[V];
-    float mv[V];
-    if constexpr (OP == kOpActInt8Smooth) load_mult<V>(mult_vec, 0, mv);
-    values_of<T, OP>(u, mv, v);
-    uint32_t w[2] = {words.x, words.y};
-    const uint32_t r[2] = {redo.x, redo.y};
-    for (int e = 0; e < V; ++e) {
-        const int sh = 8 * (e % 4);
-        if (((r[e / 4] >> sh) & 0xFFu) == 0u) continue;
-        uint32_t b;
-        if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
-            b = static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(v[e], S), __NV_SATFINITE, __NV_E4M3));
-        } else {
-            const float lo = OP == kOpWeightAsym ? -128.0f : -127.0f;
-            const float q = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(v[e], S)), Z), lo), 127.0f);
-            b = static_cast<uint32_t>(static_cast<int>(__fadd_rn(q, bias))) & 0xFFu;
-        }
-        w[e / 4] = (w[e / 4] & ~(0xFFu << sh)) | (b << sh);
-    }
-    return make_uint2(w[0], w[1]);
-}
-
-// Exact code byte of one element.
-template <int OP>
-__device__ __forceinline__ uint32_t exact_code(float x, float S, float Z, float bias) {
-    if constexpr (OP == kOpActFp8 || OP == kOpWeightFp8) {
-        return static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(x, S), __NV_SATFINITE, __NV_E4M3));
-    } else {
-        const float lo = OP == kOpWeightAsym ? -128.0f : -127.0f;
-        const float q = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(x, S)), Z), lo), 127.0f);
-        return static_cast<uint32_t>(static_cast<int>(__fadd_rn(q, bias))) & 0xFFu;
-    }
-}
-
-// Per-warp queue of elements whose bracket ends disagree: their value, their
-// byte position in the row and the fast code written for them.
-constexpr int kQueueCap = 320;
-constexpr int kDrainAt = 64;   // drained once this full: one step adds at most 32 x 8
-struct FixQueue {
-    float x[kQueueCap];
-    int pos[kQueueCap];
-    int fast[kQueueCap];
-    int n;
-};
-
-// Pushes the flagged elements of one vector (bytes of d that are nonzero).
-// Out of line, so the unrolled pass keeps a small instruction footprint.
-template <typename T, int OP>
-__device__ __noinline__ void push_flagged(const uint4 u, uint2 d, uint2 w, int pos0, FixQueue* q,
-                                          const float* mult_vec) {
-    constexpr int V = VecOf<T>::N;
-    float v[V];
-    float mv[V];
-    if constexpr (OP == kOpActInt8Smooth) load_mult<V>(mult_vec, 0, mv);
-    values_of<T, OP>(u, mv, v);
-    const uint32_t dd[2] = {d.x, d.y}, ww[2] = {w.x, w.y};
-#pragma unroll
-    for (int e = 0; e < V; ++e) {
-        const int sh = 8 * (e % 4);
-        if (((dd[e / 4] >> sh) & 0xFFu) != 0u) {
-            const int slot = atomicAdd(&q->n, 1);
-            if (slot < kQueueCap) {
-                q->x[slot] = v[e];
-                q->pos[slot] = pos0 + e;
-                q->fast[slot] = static_cast<int>(static_cast<int8_t>((ww[e / 4] >> sh) & 0xFFu));
+        for (int e = 0; e < V / 2; ++e) {
+            float2 x = q[e];
+            if constexpr (kClamp) {
+                x.x = clampf(x.x, c.qlo, c.qhi);
+                x.y = clampf(x.y, c.qlo, c.qhi);
             }
+            t[e] = __fadd2_rn(x, M);
+            if constexpr (OP == kOpWeightAsym) t[e] = __fadd2_rn(t[e], P);
         }
+        const uint32_t kp[2] = {keep.x, keep.y};
+#pragma unroll
+        for (int w = 0; w < V / 4; ++w)
+            words[w] = pack_low_bytes(__float_as_uint(t[2 * w].x), __float_as_uint(t[2 * w].y),
+                                      __float_as_uint(t[2 * w + 1].x), __float_as_uint(t[2 * w + 1].y)) &
+                       kp[w];
     }
-}
-
-// Recodes the queued elements, 32 at a time, and empties the queue; returns
-// the change of this lane's share of the row sum (int8 codes).  Called by the
-// whole warp, after the fast codes of the queued elements are stored: the
-// barrier orders those stores before the corrections, which another lane of
-// the warp may write.
-template <int OP>
-__device__ __noinline__ int drain_queue(FixQueue* q, uint8_t* dst_row, float S, float Z, float bias) {
-    __syncwarp();
-    const int n = q->n;
-    int delta = 0;
-    for (int e = threadIdx.x & 31; e < n; e += 32) {
-        const uint32_t b = exact_code<OP>(q->x[e], S, Z, bias);
-        dst_row[q->pos[e]] = static_cast<uint8_t>(b);
-        delta += static_cast<int>(static_cast<int8_t>(b)) - q->fast[e];
-    }
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) q->n = 0;
-    __syncwarp();
-    return delta;
+    return make_uint2(words[0], words[1]);
 }
 
 // Zeroes the 16-bit elements of a vector that are left out; mb holds 0xFF per
@@ -559,19 +447,15 @@ row_quant_kernel(RowQuantArgs a) {
     constexpr bool kSmooth = OP == kOpActInt8Smooth;
     __shared__ float red[3 * (kBlock / 32)];
     __shared__ int redi[kBlock / 32];
-    __shared__ FixQueue fixq[kBlock / 32];
     __shared__ float cshare[kBlock / TPR][8];
     __shared__ int s_oidx[kSkip ? kSmemOutliers : 1];   // LLM.int8: outlier column of each rank
-    FixQueue* q = &fixq[threadIdx.x / 32];
 
     const int g = threadIdx.x / TPR;
     const int t = threadIdx.x % TPR;
     const int64_t nvec = a.k / V;
     const bool cached = nvec <= static_cast<int64_t>(TPR) * MAXV;
-    // Vectors this thread holds when the row is cached, and the most any
-    // thread of its warp holds (the first one).
+    // Vectors this thread holds when the row is cached.
     const int nvl = cached ? static_cast<int>((nvec - t + TPR - 1) / TPR) : 0;
-    const int nvw = cached ? static_cast<int>((nvec - (t & ~31) + TPR - 1) / TPR) : 0;
     const float bias = (OP == kOpWeightAsym && a.codes_u8) ? 128.0f : 0.0f;
     // Launched with programmatic dependent launch: this grid may start while
     // the previous kernel runs, so it waits for it before touching memory.
@@ -622,7 +506,6 @@ row_quant_kernel(RowQuantArgs a) {
         const T* src = src_row + static_cast<int64_t>(t) * V;
         uint8_t* dst = dst_row + static_cast<int64_t>(t) * V;
         const int nv = active ? nvl : 0;
-        const int nvmax = active ? nvw : 0;
         // Every thread of the block holds MAXV vectors: no per-vector guards.
         // (Uniform over the block, as the reductions below synchronize it.)
         const bool full = nvec == static_cast<int64_t>(TPR) * MAXV && row0 + RPB <= a.rows;
@@ -701,90 +584,54 @@ row_quant_kernel(RowQuantArgs a) {
             if (t < 32) {
                 c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias, a.static_scale);
                 if (t == 0) {
-                    cs[0] = c.S; cs[1] = c.Z; cs[2] = c.bias; cs[3] = c.rlo;
-                    cs[4] = c.rhi; cs[5] = c.add; cs[6] = c.fast ? 1.0f : 0.0f;
+                    cs[0] = c.S; cs[1] = c.Z; cs[2] = c.bias; cs[3] = c.R;
+                    cs[4] = c.qlo; cs[5] = c.qhi; cs[6] = c.post; cs[7] = c.direct ? 1.0f : 0.0f;
                 }
             }
             group_sync<TPR>();
-            c.S = cs[0]; c.Z = cs[1]; c.bias = cs[2]; c.rlo = cs[3];
-            c.rhi = cs[4]; c.add = cs[5]; c.fast = cs[6] != 0.0f;
+            c.S = cs[0]; c.Z = cs[1]; c.bias = cs[2]; c.R = cs[3];
+            c.qlo = cs[4]; c.qhi = cs[5]; c.post = cs[6]; c.direct = cs[7] != 0.0f;
         } else {
             c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias, a.static_scale);
         }
 
-        // Pass 2: codes.  c.fast and `cached` are the same for the whole warp.
-        // Elements whose bracket ends disagree go to the warp's queue, which is
-        // drained (32 elements at a time, with exact divisions) whenever it is
-        // half full and at the end of the pass.
+        // Pass 2: codes.  c.direct and `cached` are the same for the whole group.
         int rsum = 0;
-        __syncwarp();   // the previous row's queue is drained
-        if ((threadIdx.x & 31) == 0) q->n = 0;
-        __syncwarp();
-        auto drain = [&]() {
-            __syncwarp();
-            if (q->n != 0) rsum += drain_queue<OP>(q, dst_row, c.S, c.Z, c.bias);   // uniform
-        };
-        auto finish = [&](uint32_t w0, uint32_t w1, uint8_t* p) {
+        auto finish = [&](uint2 w, uint8_t* p) {
             if constexpr (V == 8) {
-                *reinterpret_cast<uint2*>(p) = make_uint2(w0, w1);
+                *reinterpret_cast<uint2*>(p) = w;
             } else {
-                *reinterpret_cast<uint32_t*>(p) = w0;
+                *reinterpret_cast<uint32_t*>(p) = w.x;
             }
             if constexpr (kRowsum) {
-                rsum = __dp4a(static_cast<int>(w0), 0x01010101, rsum);
-                if constexpr (V == 8) rsum = __dp4a(static_cast<int>(w1), 0x01010101, rsum);
+                rsum = __dp4a(static_cast<int>(w.x), 0x01010101, rsum);
+                if constexpr (V == 8) rsum = __dp4a(static_cast<int>(w.y), 0x01010101, rsum);
             }
         };
         auto pass2 = [&](auto full_tag) {
             constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
             for (int i = 0; i < MAXV; ++i) {
-                if (FULL || i < nvmax) {   // uniform over the warp
-                    const bool valid = FULL || i < nv;
-                    const uint2 kp = valid ? keep_of(t + static_cast<int64_t>(i) * TPR) : make_uint2(~0u, ~0u);
-                    uint32_t words[2], d[2];
+                if (FULL || i < nv) {
+                    const int64_t j = t + static_cast<int64_t>(i) * TPR;
                     float mv[V];
-                    if constexpr (kSmooth) {
-                        if (valid) load_mult<V>(a.mult, t + static_cast<int64_t>(i) * TPR, mv);
-                        else for (int e = 0; e < V; ++e) mv[e] = 0.f;
-                    }
-                    fast_codes<T, OP>(raw[i], c, kp, words, d, mv);   // zero vectors: d = 0
-                    if (valid) finish(words[0], words[1], dst + i * TPR * V);
-                    if (__any_sync(0xffffffffu, (d[0] | d[1]) != 0u)) {
-                        if ((d[0] | d[1]) != 0u)
-                            push_flagged<T, OP>(raw[i], make_uint2(d[0], d[1]), make_uint2(words[0], words[1]),
-                                                (t + i * TPR) * V, q,
-                                                kSmooth ? a.mult + (t + static_cast<int64_t>(i) * TPR) * V : nullptr);
-                        __syncwarp();
-                        if (q->n >= kDrainAt) drain();
-                    }
+                    if constexpr (kSmooth) load_mult<V>(a.mult, j, mv);
+                    finish(code_vec<T, OP, false>(raw[i], c, keep_of(j), mv), dst + i * TPR * V);
                 }
             }
         };
-        const bool redo = !(cached && c.fast);
-        if (cached && c.fast) {
+        if (cached && !c.direct) {
             if (full) pass2(std::true_type{}); else pass2(std::false_type{});
-            drain();
-        }
-        if (active && redo) {
-            // Rows longer than the register cache (read again, from L2), rows
-            // the fast path does not cover (every code exact).
-            rsum = 0;
+        } else if (active) {
+            // Rows longer than the register cache (read again, from L2), and
+            // rows coded with divisions.
             for (int64_t j = t; j < nvec; j += TPR) {
                 const uint4 u = ld_stream16(src_row + j * V);
-                const uint2 kp = keep_of(j);
-                uint32_t words[2] = {0u, 0u}, d[2] = {~0u, ~0u};
                 float mv[V];
                 if constexpr (kSmooth) load_mult<V>(a.mult, j, mv);
-                if (c.fast) fast_codes<T, OP>(u, c, kp, words, d, mv);
-                if ((d[0] | d[1]) != 0u) {
-                    const uint2 e = exact_codes<T, OP>(u, c.S, c.Z, c.bias, make_uint2(d[0], d[1]),
-                                                       make_uint2(words[0], words[1]),
-                                                       kSmooth ? a.mult + j * V : nullptr);
-                    words[0] = e.x & kp.x;
-                    words[1] = e.y & kp.y;
-                }
-                finish(words[0], words[1], dst_row + j * V);
+                const uint2 w = c.direct ? code_vec<T, OP, true>(u, c, keep_of(j), mv)
+                                         : code_vec<T, OP, false>(u, c, keep_of(j), mv);
+                finish(w, dst_row + j * V);
             }
         }
         if constexpr (kRowsum) rsum = group_sum<TPR>(rsum, redi);

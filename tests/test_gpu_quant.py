@@ -196,7 +196,7 @@ def test_outlier_act_one_row():
 
 def test_quotient_rounding_at_exact_midpoints():
     """Rows whose scale is exactly 1 put x / S on integer and E4M3 rounding
-    midpoints, where the kernel must fall back to the exact quotient."""
+    midpoints, which must round half to even."""
     ints = [127.0, 62.5, 63.5, -62.5, -63.5, 0.5, 1.5, -0.5, 2.5, -2.5, 100.5, -126.5]
     Xi = torch.zeros(2, 64, dtype=torch.bfloat16)
     Xi[0, :len(ints)] = torch.tensor(ints)
@@ -221,10 +221,8 @@ def test_quotient_rounding_at_exact_midpoints():
 
 def test_ties_with_non_power_of_two_scale():
     """absmax = 127 * 9/64 (fp16-exact) gives S = 9/64 exactly, so
-    x = (n + 1/2) * 9/128 lies exactly on a rounding midpoint of x / S.  Whole
-    16-byte vectors of such elements give a thread more boundary elements than
-    its queue holds, which sends it through the per-vector exact path; single
-    ones go through the queue."""
+    x = (n + 1/2) * 9/128 lies exactly on a rounding midpoint of x / S: whole
+    16-byte vectors of such elements, and single ones among regular values."""
     m, k = 6, 256
     g = torch.Generator().manual_seed(41)
     n = torch.randint(-100, 100, (m, k), generator=g).to(torch.float32)
