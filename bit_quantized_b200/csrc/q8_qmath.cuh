@@ -42,19 +42,14 @@ __device__ __forceinline__ float quotient(float x, float S, float R) {
 }
 
 // The same for two elements with paired fp32 instructions.  The residuals
-// are formed as x - q S (nS = -S), which loses the sign of a zero x; with
-// SIGNED_ZERO the sign of x is put back (every other quotient has it already),
-// for codes that keep the sign of zero (E4M3).
-template <bool SIGNED_ZERO>
+// are formed as x - q S (nS = -S), which returns +0 for x = -0; every other
+// quotient has x's sign.  Callers whose codes keep the sign of zero restore it.
 __device__ __forceinline__ float2 quotient2(float2 x, float2 nS, float2 R) {
     const float2 q0 = __fmul2_rn(x, R);
     const float2 e0 = __ffma2_rn(q0, nS, x);
     const float2 q1 = __ffma2_rn(e0, R, q0);
     const float2 e1 = __ffma2_rn(q1, nS, x);
-    const float2 q2 = __ffma2_rn(e1, R, q1);
-    if constexpr (!SIGNED_ZERO) return q2;
-    return make_float2(__uint_as_float(__float_as_uint(q2.x) | (__float_as_uint(x.x) & 0x80000000u)),
-                       __uint_as_float(__float_as_uint(q2.y) | (__float_as_uint(x.y) & 0x80000000u)));
+    return __ffma2_rn(e1, R, q1);
 }
 
 }  // namespace qm

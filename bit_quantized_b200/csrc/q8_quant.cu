@@ -275,15 +275,25 @@ __device__ __forceinline__ uint2 code_vec(const uint4 u, const RowConsts& c, con
         const float2 nS = splat2(-c.S), R = splat2(c.R);
 #pragma unroll
         for (int e = 0; e < V / 2; ++e)
-            q[e] = qm::quotient2<is_fp8_op(OP)>(make_float2(v[2 * e], v[2 * e + 1]), nS, R);
+            q[e] = qm::quotient2(make_float2(v[2 * e], v[2 * e + 1]), nS, R);
     }
     uint32_t words[2] = {0u, 0u};
     if constexpr (is_fp8_op(OP)) {
+        // The quotient of -0 comes out as +0; every other quotient has x's
+        // sign.  E4M3 keeps the sign of zero, so each code byte takes the sign
+        // bit of its input (bit 7 of the input's top byte).
+        uint32_t sgn[2];
+        if constexpr (V == 8) {
+            sgn[0] = __byte_perm(u.x, u.y, 0x7531);
+            sgn[1] = __byte_perm(u.z, u.w, 0x7531);
+        } else {
+            sgn[0] = __byte_perm(__byte_perm(u.x, u.y, 0x0073), __byte_perm(u.z, u.w, 0x0073), 0x5410);
+        }
 #pragma unroll
         for (int w = 0; w < V / 4; ++w) {
             const uint32_t c0 = __nv_cvt_float2_to_fp8x2(q[2 * w], __NV_SATFINITE, __NV_E4M3);
             const uint32_t c1 = __nv_cvt_float2_to_fp8x2(q[2 * w + 1], __NV_SATFINITE, __NV_E4M3);
-            words[w] = __byte_perm(c0, c1, 0x5410);   // element 2h in the low byte of each half
+            words[w] = __byte_perm(c0, c1, 0x5410) | (sgn[w] & 0x80808080u);   // element 2h low in each half
         }
     } else {
         constexpr bool kClamp = OP == kOpActInt8Static || OP == kOpWeightAsym || DIRECT;
@@ -319,35 +329,45 @@ __device__ __forceinline__ uint4 zero_skipped16(uint4 u, const uint2 mb) {
     return u;
 }
 
-template <typename T, int OP>
-__device__ __forceinline__ void accumulate_stats(const uint4 u, RowStats& st, const float* mv = nullptr) {
-    constexpr int V = VecOf<T>::N;
-    if constexpr (OP == kOpActInt8Smooth) {
+// Row min and max over one thread's vectors.  16-bit inputs (unsmoothed) keep
+// packed 16-bit pairs, since min and max are exact in the input's own format,
+// and widen to fp32 once per row.
+template <typename T, int OP, bool PACKED = (sizeof(T) == 2 && OP != kOpActInt8Smooth)>
+struct StatsAcc {
+    float lo = FLT_MAX, hi = -FLT_MAX;
+    __device__ __forceinline__ void add(const uint4 u, const float* mv = nullptr) {
+        constexpr int V = VecOf<T>::N;
         float v[V];
         values_of<T, OP>(u, mv, v);
 #pragma unroll
         for (int e = 0; e < V; ++e) {
-            st.lo = fminf(st.lo, v[e]);
-            st.hi = fmaxf(st.hi, v[e]);
-        }
-    } else if constexpr (sizeof(T) == 2) {
-        using T2 = typename std::conditional<std::is_same<T, __half>::value, __half2, __nv_bfloat162>::type;
-        const T2* p2 = reinterpret_cast<const T2*>(&u);
-        T2 m2 = __hmax2(p2[0], p2[1]), l2 = __hmin2(p2[0], p2[1]);
-        m2 = __hmax2(m2, __hmax2(p2[2], p2[3]));
-        l2 = __hmin2(l2, __hmin2(p2[2], p2[3]));
-        st.hi = fmaxf(st.hi, fmaxf(static_cast<float>(m2.x), static_cast<float>(m2.y)));
-        st.lo = fminf(st.lo, fminf(static_cast<float>(l2.x), static_cast<float>(l2.y)));
-    } else {
-        float v[V];
-        unpack_vec<T>(u, v);
-#pragma unroll
-        for (int e = 0; e < V; ++e) {
-            st.lo = fminf(st.lo, v[e]);
-            st.hi = fmaxf(st.hi, v[e]);
+            lo = fminf(lo, v[e]);
+            hi = fmaxf(hi, v[e]);
         }
     }
-}
+    __device__ __forceinline__ RowStats get() const { return RowStats{0.f, lo, hi}; }
+};
+
+template <typename T, int OP>
+struct StatsAcc<T, OP, true> {
+    static constexpr bool kHalf = std::is_same<T, __half>::value;
+    using T2 = typename std::conditional<kHalf, __half2, __nv_bfloat162>::type;
+    // the largest finite value of T in both halves, and its negation
+    uint32_t lo = kHalf ? 0x7BFF7BFFu : 0x7F7F7F7Fu;
+    uint32_t hi = kHalf ? 0xFBFFFBFFu : 0xFF7FFF7Fu;
+    __device__ __forceinline__ static T2 as2(uint32_t w) { return *reinterpret_cast<const T2*>(&w); }
+    __device__ __forceinline__ static uint32_t bits(T2 v) { return *reinterpret_cast<const uint32_t*>(&v); }
+    __device__ __forceinline__ void add(const uint4 u, const float* = nullptr) {
+        const T2 a = as2(u.x), b = as2(u.y), c = as2(u.z), d = as2(u.w);
+        hi = bits(__hmax2(as2(hi), __hmax2(__hmax2(a, b), __hmax2(c, d))));
+        lo = bits(__hmin2(as2(lo), __hmin2(__hmin2(a, b), __hmin2(c, d))));
+    }
+    __device__ __forceinline__ RowStats get() const {
+        const T2 h = as2(hi), l = as2(lo);
+        return RowStats{0.f, fminf(static_cast<float>(l.x), static_cast<float>(l.y)),
+                        fmaxf(static_cast<float>(h.x), static_cast<float>(h.y))};
+    }
+};
 
 // The LLM.int8 outlier columns as one block sees them.  Thread i owns the
 // run of `per` consecutive mask bytes from `begin`, held as bits; `before`
@@ -522,7 +542,7 @@ row_quant_kernel(RowQuantArgs a) {
         // end of the row are zero, which leaves absmax unchanged; asymmetric
         // rows only count loaded vectors.  Left-out columns are zeroed.
         uint4 raw[MAXV];
-        RowStats st{0.f, FLT_MAX, -FLT_MAX};
+        StatsAcc<T, OP> acc;
         if constexpr (PF) {
             // This row's vectors were loaded during the previous row; the next
             // row's loads go out now.
@@ -548,9 +568,9 @@ row_quant_kernel(RowQuantArgs a) {
                     if constexpr (kSmooth) {
                         float mv[V];
                         load_mult<V>(a.mult, t + static_cast<int64_t>(i) * TPR, mv);
-                        accumulate_stats<T, OP>(raw[i], st, mv);
+                        acc.add(raw[i], mv);
                     } else {
-                        accumulate_stats<T, OP>(raw[i], st);
+                        acc.add(raw[i]);
                     }
                 }
             }
@@ -567,12 +587,13 @@ row_quant_kernel(RowQuantArgs a) {
                 if constexpr (kSmooth) {
                     float mv[V];
                     load_mult<V>(a.mult, j, mv);
-                    accumulate_stats<T, OP>(u, st, mv);
+                    acc.add(u, mv);
                 } else {
-                    accumulate_stats<T, OP>(u, st);
+                    acc.add(u);
                 }
             }
         }
+        RowStats st = acc.get();
         st.amax = fmaxf(st.hi, -st.lo);
         st = group_reduce<TPR, OP == kOpWeightAsym>(st, red);
         if constexpr (OP != kOpWeightAsym) st.amax = fmaxf(st.amax, 0.0f);

@@ -183,7 +183,8 @@ q4k_expand_kernel(const uint8_t* __restrict__ sub_codes, const float* __restrict
 // ============================================================================
 // W4A16 GEMM
 // ============================================================================
-constexpr int kThreads = 192;
+constexpr int kDqWarps = 8;                     // dequantizing warps (2 .. 9)
+constexpr int kThreads = 64 + 32 * kDqWarps;
 constexpr int kBM = 128;                        // weight rows per CTA (MMA M)
 constexpr int kBK = 64;                         // K elements per stage (128 bytes of 16-bit)
 constexpr int kABytes = kBM * kBK * 2;          // 16 KB dequantized weight slice
@@ -266,7 +267,7 @@ __device__ __forceinline__ uint4 dequant8(uint32_t word, uint64_t s2) {
 }
 
 template <int NT, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmS,
              const __grid_constant__ CUtensorMap tmX, const W4Params p, int num_kb,
              int kb_per_split, int splits, int astages, int qstages, int group) {
@@ -306,7 +307,7 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             mbar_init(&q_empty[s], 1);
         }
         for (int s = 0; s < astages; ++s) {
-            mbar_init(&a_full[s], 4);      // one arrival per dequantizing warp
+            mbar_init(&a_full[s], kDqWarps);   // one arrival per dequantizing warp
             mbar_init(&a_empty[s], 1);
         }
         mbar_init(&tfull_bar, 1);
@@ -410,27 +411,31 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         __syncwarp();
     } else {
         // ---------------- dequantize
-        const int ct = threadIdx.x - 64;           // weight row of the tile
-        const uint32_t a_row = smem_addr(a_ring) + ct * 128;
-        const int sw = ct & 7;
+        // Two threads per weight row, each expanding one half of the row's
+        // 64-value slice (32 values: 16 bytes of codes, one scale group when
+        // groups are 32 wide).  Neighbouring lanes read neighbouring 16-byte
+        // code chunks (no bank conflicts), and the 8 lanes of a quarter warp
+        // write 8 distinct swizzled chunks of 4 rows.
+        const int ct = threadIdx.x - 64;
+        const int row = ct >> 1, half = ct & 1;
+        const uint32_t a_row = smem_addr(a_ring) + row * 128;
+        const int sw = row & 7;
         int qs = 0, as = 0;
         uint32_t qph = 0, aph = 0;
         for (int i = 0; i < my_kb; ++i) {
             if (!mbar_wait(&q_full[qs], qph, &abort_sh, p.status)) break;
             const uint8_t* qsl = q_ring + qs * C::QSLOT + C::X_BYTES;
-            const uint4 c0 = *reinterpret_cast<const uint4*>(qsl + ct * 32);
-            const uint4 c1 = *reinterpret_cast<const uint4*>(qsl + ct * 32 + 16);
+            const uint4 cw = *reinterpret_cast<const uint4*>(qsl + row * 32 + half * 16);
             const float* ssl = reinterpret_cast<const float*>(qsl + kQBytes);
-            const uint32_t s0 = __float_as_uint(ssl[ct]);
-            const uint32_t s1 = gps == 2 ? __float_as_uint(ssl[kBM + ct]) : s0;
+            const uint32_t sc = __float_as_uint(ssl[(gps == 2 ? half * kBM : 0) + row]);
             if (!mbar_wait(&a_empty[as], aph ^ 1, &abort_sh, p.status)) break;
             const uint32_t dst = a_row + as * kABytes;
-            const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-            const uint64_t s20 = pair(s0, s0), s21 = pair(s1, s1);
+            const uint32_t w[4] = {cw.x, cw.y, cw.z, cw.w};
+            const uint64_t s2 = pair(sc, sc);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = dequant8<BF16>(w[c], c < 4 ? s20 : s21);
-                st_shared_v4(dst + ((c ^ sw) << 4), v.x, v.y, v.z, v.w);
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = dequant8<BF16>(w[c], s2);
+                st_shared_v4(dst + (((4 * half + c) ^ sw) << 4), v.x, v.y, v.z, v.w);
             }
             fence_async_smem();
             __syncwarp();
@@ -448,7 +453,10 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         pdl_wait();
 
         // ---------------- epilogue
+        // Warps 2-5 and 6-9 each cover the 128 channels (TMEM lane quarter
+        // warp % 4) and take alternate 16-token column chunks.
         const int q = warp & 3;                    // TMEM lane quarter of this warp
+        const int eh = (warp - 2) >> 2;            // which of the two warp sets
         const int ch = q * 32 + lane;
         const int n = tn * kBM + ch;
         const bool col_ok = n < p.n;
@@ -458,7 +466,7 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         __syncwarp();
         const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
         if (splits == 1) {
-            for (int c = 0; c < NT && m0 + c < p.m; c += 16) {
+            for (int c = 16 * eh; c < NT && m0 + c < p.m; c += 32) {
                 uint32_t r[16];
                 tmem_ld16(tb + c, r);
                 tmem_ld_wait();
@@ -478,7 +486,7 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             const int tpo = (NT + splits - 1) / splits;
             const uint32_t red_base = smem_addr(red);
 #pragma unroll
-            for (int c = 0; c < NT; c += 16) {
+            for (int c = 16 * eh; c < NT; c += 32) {
                 uint32_t r[16];
                 tmem_ld16(tb + c, r);
                 tmem_ld_wait();
@@ -500,12 +508,13 @@ w4a16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
             cluster_sync();
             if (warp >= 2) {
                 const int q = warp & 3;
+                const int eh = (warp - 2) >> 2;
                 const int ch = q * 32 + lane;
                 const int n = tn * kBM + ch;
                 const int tpo = (NT + splits - 1) / splits;
                 if (n < p.n) {
                     const float bias = p.bias ? p.bias[n] : 0.f;
-                    for (int t = static_cast<int>(rank); t < NT && m0 + t < p.m; t += splits) {
+                    for (int t = static_cast<int>(rank) + eh * splits; t < NT && m0 + t < p.m; t += 2 * splits) {
                         const int tl = t / splits;
                         float s = 0.f;
                         for (int r = 0; r < splits; ++r)
