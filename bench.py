@@ -478,38 +478,49 @@ def run_e2e(q8, layers, R, step_fn, args, world, ops_per_step, w):
     """Same step through the public API with the input copied from pinned host
     memory and the bf16 output copied back to pinned host memory every step.
 
-    The steps are replayed as a CUDA graph of R steps, as a serving loop would
-    issue them: each step's host-to-device copy runs on a copy stream and may
-    overlap the previous step's compute, the step's call runs on the compute
-    stream once its input has landed, and the device-to-host copy of its
-    result on a third stream.  Every step still moves its own input and
-    output; a replay ends only when the last step's output is on the host."""
-    steps = min(args.steps, args.e2e_steps)
-    reps = max(1, steps // R)
-    steps = reps * R
+    The steps are replayed as a CUDA graph of S steps (a multiple of the R
+    layers, up to 16), as a serving loop would issue them: each step's
+    host-to-device copy runs on a copy stream and may overlap earlier steps'
+    compute and output copies, the step's call runs on the compute stream once
+    its input has landed, and the device-to-host copy of its result on a third
+    stream.  Step i uses layer i mod R; a copy into a layer's input buffer
+    waits until the step that last read it has finished, and a step waits
+    until the previous output copy of its layer has left the device.  Every
+    step still moves its own input and output; a replay ends only when the
+    last step's output is on the host."""
+    S = R * max(1, min(args.steps, args.e2e_steps, 16) // R)
+    reps = max(1, min(args.steps, args.e2e_steps) // S)
+    steps = reps * S
     hx = [L["X"].cpu().pin_memory() for L in layers]
     hy = [torch.empty((w.m, w.n), dtype=torch.bfloat16).pin_memory() for _ in layers]
     dx = [torch.empty_like(L["X"]) for L in layers]
     s_main, s_in, s_comp, s_out = (torch.cuda.Stream() for _ in range(4))
-    ev_in = [torch.cuda.Event() for _ in range(R)]
-    ev_done = [torch.cuda.Event() for _ in range(R)]
+    ev_in = [torch.cuda.Event() for _ in range(S)]
+    ev_done = [torch.cuda.Event() for _ in range(S)]
+    ev_out = [torch.cuda.Event() for _ in range(S)]
 
     def record_steps():
         fork = torch.cuda.Event()
         fork.record(s_main)
         for st in (s_in, s_comp, s_out):
             st.wait_event(fork)
-        for i in range(R):
+        for i in range(S):
+            j = i % R
             with torch.cuda.stream(s_in):
-                dx[i].copy_(hx[i], non_blocking=True)
+                if i >= R:
+                    s_in.wait_event(ev_done[i - R])      # dx[j] read by step i - R
+                dx[j].copy_(hx[j], non_blocking=True)
                 ev_in[i].record(s_in)
             with torch.cuda.stream(s_comp):
                 s_comp.wait_event(ev_in[i])
-                step_fn(layers[i], dx[i])
+                if i >= R:
+                    s_comp.wait_event(ev_out[i - R])     # Y of layer j copied out
+                step_fn(layers[j], dx[j])
                 ev_done[i].record(s_comp)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_done[i])
-                hy[i].copy_(layers[i]["Y"], non_blocking=True)
+                hy[j].copy_(layers[j]["Y"], non_blocking=True)
+                ev_out[i].record(s_out)
         for st in (s_in, s_comp, s_out):
             s_main.wait_stream(st)
 
@@ -544,7 +555,7 @@ def run_e2e(q8, layers, R, step_fn, args, world, ops_per_step, w):
             "host_output_matches_device": ok,
             "path": "pinned host X -> H2D copy stream -> q8_linear_w8a8_dynamic / q8_linear_int8_mixed "
                     "(C ABI) on a compute stream -> D2H copy stream -> pinned host Y; CUDA graph of "
-                    f"{R} steps, a step's copies overlap its neighbours' compute"}
+                    f"{S} steps over {R} layers, a step's copies overlap other steps' compute and copies"}
 
 
 def load_profile_traffic(kernel_tag: str):
