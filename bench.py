@@ -260,7 +260,8 @@ def dominant_kernel(w, gemm_ms: float, region_ms: float, pk: dict, lib_peaks: di
     peak = bf16 * NOMINAL_INT8_OVER_BF16
     achieved = ops / t / 1e12
     if w.kind == "int8_mixed":
-        kernel = "gemm_tile_kernel (LLM.int8, int32 + fp32 accumulators)"
+        kernel = ("gemm_pair_kernel (LLM.int8, cta_group::2, int32 + fp32 accumulators)" if w.m > 128
+                  else "gemm_tile_kernel (LLM.int8, int32 + fp32 accumulators)")
     elif w.m > 256:
         kernel = "gemm_pair_kernel (cta_group::2, 256-row tiles on SM pairs)"
     else:

@@ -820,7 +820,8 @@ cudaError_t launch_rows_dtype(const RowQuantArgs& a, cudaStream_t s) {
 // ------------------------------------------------------------------ outliers
 
 // Column absmax over all rows for a strip of 32 columns per block:
-// 4 threads x 8 columns across the strip, 64 row lanes down it.
+// 4 threads x 8 columns across the strip, 64 row lanes down it, eight rows'
+// loads in flight per thread (512 rows per round).
 template <typename T>
 __global__ void __launch_bounds__(kBlock) outlier_colmax_kernel(const T* __restrict__ X, int64_t m,
                                                                 int64_t k, int64_t ldx, float thr,
@@ -829,18 +830,22 @@ __global__ void __launch_bounds__(kBlock) outlier_colmax_kernel(const T* __restr
     const int cv = threadIdx.x % 4;        // which 8-column vector of the strip
     const int rl = threadIdx.x / 4;        // row lane 0..63
     const int64_t col0 = static_cast<int64_t>(blockIdx.x) * 32 + cv * 8;
+    // Launched with programmatic dependent launch: X may be the previous
+    // kernel's output.  The row pass that follows may launch right away (it
+    // waits for this grid before reading the mask).
+    pdl_launch_dependents();
+    pdl_wait();
     float mx[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) mx[e] = 0.f;
     if (col0 < k) {
-        // Four rows' loads in flight per thread at a time.
-        for (int64_t r0 = rl; r0 < m; r0 += 4 * 64) {
-            uint4 u[4];
+        for (int64_t r0 = rl; r0 < m; r0 += 8 * 64) {
+            uint4 u[8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+            for (int i = 0; i < 8; ++i)
                 u[i] = r0 + i * 64 < m ? ld_stream16(X + (r0 + i * 64) * ldx + col0) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < 8; ++i) {
                 float v[8];
                 unpack_vec<T>(u[i], v);
 #pragma unroll
@@ -896,14 +901,20 @@ cudaError_t launch_row_quant(const RowQuantArgs& a, cudaStream_t s) {
 
 cudaError_t launch_outlier_columns(const void* X, q8_dtype dt, int64_t m, int64_t k, int64_t ldx,
                                    float threshold, uint8_t* mask, cudaStream_t s) {
-    const unsigned blocks = static_cast<unsigned>((k + 31) / 32);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((k + 31) / 32), 1, 1);
+    cfg.blockDim = dim3(kBlock, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (dt == Q8_F16)
-        outlier_colmax_kernel<__half><<<blocks, kBlock, 0, s>>>(static_cast<const __half*>(X), m, k,
-                                                                ldx, threshold, mask);
-    else
-        outlier_colmax_kernel<__nv_bfloat16><<<blocks, kBlock, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(X), m, k, ldx, threshold, mask);
-    return cudaGetLastError();
+        return cudaLaunchKernelEx(&cfg, outlier_colmax_kernel<__half>, static_cast<const __half*>(X), m, k, ldx,
+                                  threshold, mask);
+    return cudaLaunchKernelEx(&cfg, outlier_colmax_kernel<__nv_bfloat16>, static_cast<const __nv_bfloat16*>(X), m,
+                              k, ldx, threshold, mask);
 }
 
 cudaError_t launch_dequant(const q8_weight& w, q8_dtype out_dtype, void* out, cudaStream_t s) {
