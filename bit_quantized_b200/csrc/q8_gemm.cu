@@ -505,8 +505,12 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 
     int n16_kb = 0;
     if constexpr (MIXED) {
-        pdl_wait();   // the outlier count comes from the previous kernels
-        n16_kb = (*p.outlier_count + 63) / 64;
+        // The outlier count comes from the previous kernels (the producer
+        // reads it after its early weight loads).
+        if (warp != 0) {
+            pdl_wait();
+            n16_kb = (*p.outlier_count + 63) / 64;
+        }
     }
     const int total_kb = num_kb + n16_kb;
     const int num_tiles = GROUPED ? g_mt[GROUPED ? experts : 0] * tiles_n : tiles_m * tiles_n;
@@ -524,7 +528,24 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 tma_prefetch_desc(&tmA16);
                 tma_prefetch_desc(&tmB16);
             }
+            // The weights do not depend on the previous kernel (a weight
+            // quantizer lets no dependent grid start before it completes): the
+            // first ring of the first tile's weight slices goes out before the
+            // programmatic-launch wait, the activation slices after it.
+            int npre = 0;
+            if constexpr (!GROUPED) {
+                if (static_cast<int>(blockIdx.x) < num_tiles) {
+                    const TileRef tr0 = tile_ref(blockIdx.x);
+                    npre = num_kb < C::STAGES ? num_kb : C::STAGES;
+                    for (int s = 0; s < npre; ++s) {
+                        mbar_arrive_expect_tx(&full_bar[s], C::STAGE);
+                        tma_load_2d(smem + s * C::STAGE + C::A_BYTES, &tmB, &full_bar[s], s * kBKB, tr0.b_row);
+                    }
+                }
+            }
             pdl_wait();   // operands may come from the previous kernel
+            int ptotal_kb = total_kb;
+            if constexpr (MIXED) ptotal_kb = num_kb + (*p.outlier_count + 63) / 64;
             uint32_t issued = 0;             // stages that ever received a load
             uint32_t last_par = 0;           // parity of each stage's last load
             int stage = 0;
@@ -532,17 +553,18 @@ gemm_tile_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const TileRef tr = tile_ref(tile);
-                for (int kb = 0; kb < total_kb; ++kb) {
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
+                for (int kb = 0; kb < ptotal_kb; ++kb) {
+                    const bool pre = tile == static_cast<int>(blockIdx.x) && kb < npre;   // weight already out
+                    if (!pre && !mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
                         ok = false;
                         break;
                     }
                     uint8_t* sa = smem + stage * C::STAGE;
                     uint8_t* sb = sa + C::A_BYTES;
-                    mbar_arrive_expect_tx(&full_bar[stage], C::STAGE);
+                    if (!pre) mbar_arrive_expect_tx(&full_bar[stage], C::STAGE);
                     if (!MIXED || kb < num_kb) {
                         tma_load_2d(sa, &tmA, &full_bar[stage], kb * kBKB, tr.a_row);
-                        tma_load_2d(sb, &tmB, &full_bar[stage], kb * kBKB, tr.b_row);
+                        if (!pre) tma_load_2d(sb, &tmB, &full_bar[stage], kb * kBKB, tr.b_row);
                     } else {
                         const int k16 = (kb - num_kb) * 64;
                         tma_load_2d(sa, &tmA16, &full_bar[stage], k16, tr.a_row);
@@ -766,8 +788,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     // ones; their count is read on the device (no host round trip).
     int n16_kb = 0;
     if constexpr (MIXED) {
-        pdl_wait();
-        n16_kb = (*p.outlier_count + 63) / 64;
+        // The producer reads the count after its early weight loads.
+        if (warp != 0) {
+            pdl_wait();
+            n16_kb = (*p.outlier_count + 63) / 64;
+        }
     }
     const int total_kb = num_kb + n16_kb;
     // A pair tile is 256 activation rows (128 from each CTA) x BN columns.
@@ -781,26 +806,45 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
             const uint32_t full0 = map_shared_rank(smem_addr(&full_bar[0]), 0);
+            // The weights do not depend on the previous kernel: the first ring
+            // of the first tile's weight halves goes out before the
+            // programmatic-launch wait, the activation slices after it.
+            int npre = 0;
+            if constexpr (!GROUPED) {
+                if (pair < num_tiles) {
+                    const TileRef tr0 = tile_ref(pair);
+                    const int yb0 = tr0.b_row + static_cast<int>(rank) * (BN / 2);
+                    npre = num_kb < C::STAGES ? num_kb : C::STAGES;
+                    for (int s = 0; s < npre; ++s) {
+                        if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2 * C::STAGE);
+                        tma_load_2d_pair(smem + s * C::STAGE + C::A_BYTES, &tmB, full0 + 8u * static_cast<uint32_t>(s),
+                                         s * kBKB, yb0);
+                    }
+                }
+            }
             pdl_wait();
+            int ptotal_kb = total_kb;
+            if constexpr (MIXED) ptotal_kb = num_kb + (*p.outlier_count + 63) / 64;
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
                 const TileRef tr = tile_ref(tile);
-                for (int kb = 0; kb < total_kb; ++kb) {
-                    if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
+                for (int kb = 0; kb < ptotal_kb; ++kb) {
+                    const bool pre = tile == pair && kb < npre;   // weight half already out
+                    if (!pre && !mbar_wait(&empty_bar[stage], phase ^ 1, &abort_sh, p.status)) {
                         ok = false;
                         break;
                     }
                     uint8_t* sa = smem + stage * C::STAGE;
                     uint8_t* sb = sa + C::A_BYTES;
-                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE);
+                    if (rank == 0 && !pre) mbar_arrive_expect_tx(&full_bar[stage], 2 * C::STAGE);
                     const uint32_t fb = full0 + 8u * static_cast<uint32_t>(stage);
                     const int ya = tr.a_row + static_cast<int>(rank) * kBM;
                     const int yb = tr.b_row + static_cast<int>(rank) * (BN / 2);
                     if (!MIXED || kb < num_kb) {
                         tma_load_2d_pair(sa, &tmA, fb, kb * kBKB, ya);
-                        tma_load_2d_pair(sb, &tmB, fb, kb * kBKB, yb);
+                        if (!pre) tma_load_2d_pair(sb, &tmB, fb, kb * kBKB, yb);
                     } else {
                         // 64 fp16 columns: the same 128-byte rows
                         tma_load_2d_pair(sa, &tmA16, fb, (kb - num_kb) * 64, ya);
