@@ -41,15 +41,23 @@ __device__ __forceinline__ float quotient(float x, float S, float R) {
     return __fmaf_rn(-e1, R, q1);
 }
 
-// The same for two elements with paired fp32 instructions.  The residuals
-// are formed as x - q S (nS = -S), which returns +0 for x = -0; every other
-// quotient has x's sign.  Callers whose codes keep the sign of zero restore it.
-__device__ __forceinline__ float2 quotient2(float2 x, float2 nS, float2 R) {
-    const float2 q0 = __fmul2_rn(x, R);
+// The same for two elements with paired fp32 instructions and one correction
+// instead of two: with 1/S carried as R + Rlo (Rlo = RN(RN(1 - S R) R), the
+// next 24 bits of the reciprocal), q0 = RN(x R + RN(x Rlo)) is within 2^-47
+// relative of x / S before its rounding, so q0 is faithful and Markstein's
+// step gives RN(x / S) directly.  The residual is formed as x - q0 S
+// (nS = -S), which returns +0 for x = -0; every other quotient has x's sign,
+// and callers whose codes keep the sign of zero restore it.
+__device__ __forceinline__ float2 quotient2(float2 x, float2 nS, float2 R, float2 Rlo) {
+    const float2 q0 = __ffma2_rn(x, R, __fmul2_rn(x, Rlo));
     const float2 e0 = __ffma2_rn(q0, nS, x);
-    const float2 q1 = __ffma2_rn(e0, R, q0);
-    const float2 e1 = __ffma2_rn(q1, nS, x);
-    return __ffma2_rn(e1, R, q1);
+    return __ffma2_rn(e0, R, q0);
+}
+
+// The low part of 1/S for quotient2: 1 - S R is exact in an FMA (R = RN(1/S)),
+// and (1 - S R) / S = 1/S - R.
+__device__ __forceinline__ float reciprocal_low(float S, float R) {
+    return __fmul_rn(__fmaf_rn(-S, R, 1.0f), R);
 }
 
 }  // namespace qm

@@ -159,9 +159,10 @@ __device__ __forceinline__ float clampf(float v, float lo, float hi) {
 // Codes of one 16-byte vector (V elements) without a division per element.
 //
 // The target is a rounding of the IEEE quotient fl32(x / S): rne for integer
-// codes, E4M3 (half to even, saturating) for FP8.  Each row gets R = RN(1/S),
-// and every element's quotient is formed exactly from it with one multiply and
-// two FMA corrections (qm::quotient: Markstein's correction step).  No element
+// codes, E4M3 (half to even, saturating) for FP8.  Each row gets R = RN(1/S)
+// and the next 24 bits of 1/S, and every element's quotient is formed exactly
+// from them with a multiply, an FMA and one FMA correction (qm::quotient2:
+// Markstein's correction step from a faithful first quotient).  No element
 // needs a division, and there is no special case for quotients that fall on a
 // rounding boundary (with 16-bit inputs, x / S falls exactly on one about 2
 // times in 1000: 127 x / absmax is a ratio of two short significands).
@@ -195,7 +196,7 @@ __device__ __forceinline__ float2 splat2(float a) { return make_float2(a, a); }
 // Per-row constants.
 struct RowConsts {
     float S, Z, bias;
-    float R;          // RN(1/S)
+    float R, Rlo;     // RN(1/S) and the next bits of 1/S
     float qlo, qhi;   // integer codes: bounds of q before the rounding
     float post;       // integer codes: Z + bias, added after the rounding
     bool direct;      // code the row with a division per element
@@ -222,6 +223,7 @@ __device__ __forceinline__ RowConsts row_consts(float amax, float lo, float hi, 
     }
     if (OP != kOpActInt8Static && !(c.S >= kEps)) c.S = kEps;
     c.R = __frcp_rn(c.S);
+    c.Rlo = qm::reciprocal_low(c.S, c.R);
     c.qlo = -127.0f;
     c.qhi = 127.0f;
     c.post = 0.f;
@@ -272,10 +274,10 @@ __device__ __forceinline__ uint2 code_vec(const uint4 u, const RowConsts& c, con
 #pragma unroll
         for (int e = 0; e < V / 2; ++e) q[e] = make_float2(__fdiv_rn(v[2 * e], c.S), __fdiv_rn(v[2 * e + 1], c.S));
     } else {
-        const float2 nS = splat2(-c.S), R = splat2(c.R);
+        const float2 nS = splat2(-c.S), R = splat2(c.R), Rlo = splat2(c.Rlo);
 #pragma unroll
         for (int e = 0; e < V / 2; ++e)
-            q[e] = qm::quotient2(make_float2(v[2 * e], v[2 * e + 1]), nS, R);
+            q[e] = qm::quotient2(make_float2(v[2 * e], v[2 * e + 1]), nS, R, Rlo);
     }
     uint32_t words[2] = {0u, 0u};
     if constexpr (is_fp8_op(OP)) {
@@ -467,7 +469,7 @@ row_quant_kernel(RowQuantArgs a) {
     constexpr bool kSmooth = OP == kOpActInt8Smooth;
     __shared__ float red[3 * (kBlock / 32)];
     __shared__ int redi[kBlock / 32];
-    __shared__ float cshare[kBlock / TPR][8];
+    __shared__ float cshare[kBlock / TPR][9];
     __shared__ int s_oidx[kSkip ? kSmemOutliers : 1];   // LLM.int8: outlier column of each rank
 
     const int g = threadIdx.x / TPR;
@@ -607,11 +609,13 @@ row_quant_kernel(RowQuantArgs a) {
                 if (t == 0) {
                     cs[0] = c.S; cs[1] = c.Z; cs[2] = c.bias; cs[3] = c.R;
                     cs[4] = c.qlo; cs[5] = c.qhi; cs[6] = c.post; cs[7] = c.direct ? 1.0f : 0.0f;
+                    cs[8] = c.Rlo;
                 }
             }
             group_sync<TPR>();
             c.S = cs[0]; c.Z = cs[1]; c.bias = cs[2]; c.R = cs[3];
             c.qlo = cs[4]; c.qhi = cs[5]; c.post = cs[6]; c.direct = cs[7] != 0.0f;
+            c.Rlo = cs[8];
         } else {
             c = row_consts<OP>(st.amax, st.lo, st.hi, a.clip_ub, bias, a.static_scale);
         }
