@@ -860,9 +860,21 @@ __global__ void __launch_bounds__(kBlock) outlier_colmax_kernel(const T* __restr
 #pragma unroll
     for (int e = 0; e < 8; ++e) part[rl][cv * 8 + e] = mx[e];
     __syncthreads();
+    // Two-level reduction of the 64 row lanes: each warp folds 8 of them for
+    // the strip's 32 columns (independent loads), then one warp folds the 8.
+    __shared__ float part2[8][32];
+    {
+        const int w = threadIdx.x / 32, c = threadIdx.x % 32;
+        float v = 0.f;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) v = fmaxf(v, part[w * 8 + r][c]);
+        part2[w][c] = v;
+    }
+    __syncthreads();
     if (threadIdx.x < 32) {
         float c = 0.f;
-        for (int r = 0; r < 64; ++r) c = fmaxf(c, part[r][threadIdx.x]);
+#pragma unroll
+        for (int w = 0; w < 8; ++w) c = fmaxf(c, part2[w][threadIdx.x]);
         const int64_t col = static_cast<int64_t>(blockIdx.x) * 32 + threadIdx.x;
         if (col < k) mask[col] = (thr > 0.f && c > thr) ? 1 : 0;
     }
