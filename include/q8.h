@@ -258,13 +258,14 @@ q8_status q8_outlier_quantize_act(const void *X, q8_dtype x_dtype, int64_t m, in
  * Launch overlap: the quantize and GEMM kernels are launched with
  * programmatic dependent launch, and each waits for the kernel before it
  * before reading anything that kernel may write.  The one exception is the
- * weight: when the kernel right before the GEMM is this library's activation
- * quantizer, the GEMM starts loading the weight early, while that quantizer
- * and the kernel before it may still run.  The weight must therefore not be
- * written by a kernel that triggers programmatic launch early
- * (griddepcontrol.launch_dependents) and runs just before the quantizer.  This
- * library's weight quantizer does not trigger, so quantize_weight followed by
- * any sequence of these calls is safe.
+ * weight: every GEMM kernel requests its first weight slices before that
+ * wait, so when the kernel right before it triggers programmatic launch early
+ * (this library's activation quantizers and LLM.int8 row pass do), the weight
+ * loads overlap that kernel and the one before it.  The weight must therefore
+ * not be written by a kernel that triggers programmatic launch early
+ * (griddepcontrol.launch_dependents) and runs just before the GEMM or its
+ * quantizer.  This library's weight quantizers do not trigger, so
+ * quantize_weight followed by any sequence of these calls is safe.
  */
 q8_status q8_linear_w8a8(const q8_act *x, const q8_weight *w, const float *bias, void *Y,
                          int64_t ldy, void *acc_debug, void *workspace, size_t ws_bytes,
