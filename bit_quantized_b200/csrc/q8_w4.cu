@@ -190,7 +190,7 @@ constexpr int kBK = 64;                         // K elements per stage (128 byt
 constexpr int kABytes = kBM * kBK * 2;          // 16 KB dequantized weight slice
 constexpr int kQBytes = kBM * kBK / 2;          // 4 KB packed codes
 constexpr int kSBytes = 2 * kBM * 4;            // room for two groups of scales
-constexpr int kMaxA = 4;
+constexpr int kMaxA = 8;
 constexpr int kMaxQ = 8;
 
 // Staging slot of one K slice: [activation tile, 128-byte swizzled][codes][scales].
@@ -607,7 +607,10 @@ q8_status run_w4(const W4Args& a, cudaStream_t s) {
         astages = NT == 64 ? 3 : 2;
         qstages = NT == 32 ? 6 : 8;
     } else {
-        astages = NT == 128 ? 3 : 2;
+        // Deep rings of dequantized slices: the dequantizing warps refill a
+        // slot only after the MMAs that read it completed, so with two slots
+        // the tensor pipe idled for that round trip on every K slice.
+        astages = NT == 128 ? 5 : 4;
         qstages = NT == 128 ? 6 : 4;
     }
     if (astages > per) astages = per;
