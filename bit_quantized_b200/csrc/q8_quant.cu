@@ -794,6 +794,10 @@ cudaError_t launch_rows_t(const RowQuantArgs& a, cudaStream_t s) {
     // unrolled for just those keeps the code short, which matters when each
     // SM runs it once (small batches: the instructions are fetched cold).
     if (tpr == 256 && nvec <= 256 * 2) return go(T256{}, C2{}, N{});
+    // The LLM.int8 row pass also gathers the outlier columns of X and W by
+    // block and by warp: one row per block gives those gathers twice the
+    // blocks (512 x 4096 fp16: 32.1 -> 30.9 us per call).
+    if (OP == kOpActInt8Skip && tpr >= 128 && nvec <= 256 * 2) return go(T256{}, C2{}, N{});
     if (tpr >= 128 && nvec <= 128 * 4) return go(T128{}, C4{}, N{});
     if (tpr == 256 && nvec <= 256 * 4) return go(T256{}, C4{}, N{});
     if (tpr == 32) return go(std::integral_constant<int, 32>{}, C16{}, N{});
